@@ -1,0 +1,92 @@
+"""Seeded synthetic workloads: shapes, distributions and input generation.
+
+This module holds no attention arithmetic; it only draws inputs.  Both the CUDA
+path's tests/bench and the fp64 oracle's tests take their inputs from here.
+
+Each workload draws Q, K, V and dO, in that order, as float32 normals from
+``torch.Generator('cpu').manual_seed(seed)``, multiplies Q and K by ``qk_std``,
+and rounds all four to bf16.  The oracle receives the same bf16 values upcast
+exactly to float64.
+"""
+
+from __future__ import annotations
+
+import math
+from dataclasses import dataclass
+
+import torch
+
+
+@dataclass(frozen=True)
+class Workload:
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    N: int
+    d: int
+    causal: bool
+    qk_std: float = 1.0
+    seed: int = 1000
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    def fwd_flops(self) -> float:
+        """4·B·Hq·N²·d, halved when causal."""
+        f = 4.0 * self.B * self.Hq * self.N * self.N * self.d
+        return f / 2 if self.causal else f
+
+    def bwd_flops(self) -> float:
+        return 2.5 * self.fwd_flops()
+
+    def describe(self) -> str:
+        return (f"B={self.B} Hq={self.Hq} Hkv={self.Hkv} N={self.N} d={self.d} "
+                f"{'causal' if self.causal else 'non-causal'} qk_std={self.qk_std:g}")
+
+
+# The five reference workloads (seed = 1000 + index).  C2 runs both causal and
+# non-causal; the non-causal variant is the benchmark workload.
+WORKLOADS = {
+    "tiny_b1_h2_n128_d64": Workload("tiny_b1_h2_n128_d64", 1, 2, 2, 128, 64, False, 1.0, 1000),
+    "train_b8_h16_n2048_d128": Workload("train_b8_h16_n2048_d128", 8, 16, 16, 2048, 128, False, 1.0, 1001),
+    "train_b8_h16_n2048_d128_causal": Workload("train_b8_h16_n2048_d128_causal", 8, 16, 16, 2048, 128, True, 1.0, 1001),
+    "long_b1_h16_n16384_d128_causal": Workload("long_b1_h16_n16384_d128_causal", 1, 16, 16, 16384, 128, True, 1.0, 1002),
+    "gqa_b4_hq32_hkv8_n4096_d128_causal": Workload("gqa_b4_hq32_hkv8_n4096_d128_causal", 4, 32, 8, 4096, 128, True, 1.0, 1003),
+    "wide_b2_h8_n8192_d256_bigqk": Workload("wide_b2_h8_n8192_d256_bigqk", 2, 8, 8, 8192, 256, False, 3.0, 1004),
+}
+
+BENCH_WORKLOAD = "train_b8_h16_n2048_d128"
+
+
+def make_inputs(w: Workload, device="cpu", seed: int | None = None):
+    """Draw (q, k, v, do) as bf16 tensors with shapes [B,Hq,N,d], [B,Hkv,N,d],
+    [B,Hkv,N,d], [B,Hq,N,d] from the workload's seed, then move them to
+    ``device``."""
+    g = torch.Generator("cpu").manual_seed(w.seed if seed is None else seed)
+    q = torch.randn(w.B, w.Hq, w.N, w.d, generator=g, dtype=torch.float32)
+    k = torch.randn(w.B, w.Hkv, w.N, w.d, generator=g, dtype=torch.float32)
+    v = torch.randn(w.B, w.Hkv, w.N, w.d, generator=g, dtype=torch.float32)
+    do = torch.randn(w.B, w.Hq, w.N, w.d, generator=g, dtype=torch.float32)
+    if w.qk_std != 1.0:
+        q.mul_(w.qk_std)
+        k.mul_(w.qk_std)
+    out = [t.to(torch.bfloat16) for t in (q, k, v, do)]
+    return tuple(t.to(device) for t in out)
+
+
+def shard_units(B: int, Hkv: int, rank: int, world: int):
+    """Split the independent (batch, kv-head) units of a workload across
+    ``world`` ranks: contiguous blocks of the flattened B·Hkv index, the first
+    ``B·Hkv % world`` ranks taking one extra.  Query heads travel with their
+    kv head, so no rank needs another rank's data."""
+    total = B * Hkv
+    base, extra = divmod(total, world)
+    start = rank * base + min(rank, extra)
+    count = base + (1 if rank < extra else 0)
+    return [(u // Hkv, u % Hkv) for u in range(start, start + count)]

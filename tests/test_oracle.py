@@ -1,0 +1,361 @@
+"""Pins for the fp64 oracle, checked against what the pages and the mathematics
+fix rather than against the oracle itself:
+
+* the worked online-softmax example printed in "深度学习进阶（三十一）FlashAttention：
+  IO 感知的精确注意力" §2.1 (golden fixture) and its closed forms;
+* the page's claim in the same section that the online result equals safe
+  softmax exactly, extended to the blockwise attention update of §2.2;
+* rows of P sum to one (the softmax row-sum invariant the "Flash-Attention"
+  concept page cites as an SDC check, "Key observations");
+* closed forms of the definition (Q = 0, V = 1);
+* the library special case: torch's fp64 CPU ``scaled_dot_product_attention``
+  and its autograd (the handbook page "FlashAttention", "如何使用 FlashAttention",
+  names PyTorch SDPA as the standard entry point);
+* central finite differences and gradient invariants for the backward pass;
+* planted mistakes in the oracle, which must make at least one pin fail.
+"""
+
+import math
+import os
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from oracle import attention as oa
+
+GOLDEN = os.path.join(os.path.dirname(__file__), "golden", "online_softmax_example.txt")
+
+
+def _read_golden(path):
+    out = {}
+    with open(path) as f:
+        for line in f:
+            line = line.strip()
+            if not line or line.startswith("#"):
+                continue
+            key, val = line.split("=", 1)
+            out[key.strip()] = [float(t) for t in val.split(",")]
+    return out
+
+
+# ---------------------------------------------------------------------------
+# Online softmax worked example
+# ---------------------------------------------------------------------------
+
+def test_online_softmax_worked_example_matches_page():
+    g = _read_golden(GOLDEN)
+    dec = int(g["decimals"][0])
+    m_tr, d_tr, y = oracle.online_softmax(g["x"])
+    tol = 0.5 * 10 ** (-dec) + 1e-12
+    np.testing.assert_allclose(m_tr, g["m_after_each_step"], atol=tol, rtol=0)
+    np.testing.assert_allclose(d_tr, g["d_after_each_step"], atol=tol, rtol=0)
+    np.testing.assert_allclose(y, g["softmax"], atol=tol, rtol=0)
+
+
+def test_online_softmax_worked_example_closed_forms():
+    # d_2 = 1 + e^{-1};  d_3 = d_2·e^{-1} + 1;  y = e^{x-3} / d_3
+    _, d_tr, y = oracle.online_softmax([2.0, 1.0, 3.0])
+    e1 = math.exp(-1.0)
+    assert d_tr[0] == 1.0
+    assert abs(d_tr[1] - (1 + e1)) < 1e-15
+    assert abs(d_tr[2] - ((1 + e1) * e1 + 1)) < 1e-15
+    d3 = (1 + e1) * e1 + 1
+    np.testing.assert_allclose(y, [math.exp(-1) / d3, math.exp(-2) / d3, 1 / d3], rtol=1e-15)
+
+
+def test_online_softmax_equals_safe_softmax():
+    rng = np.random.default_rng(0)
+    for n in (1, 2, 7, 64, 300):
+        for sd in (1.0, 30.0, 300.0):
+            x = rng.normal(0, sd, n)
+            _, d_tr, y = oracle.online_softmax(x)
+            np.testing.assert_allclose(y, oracle.safe_softmax(x), rtol=1e-12, atol=1e-300)
+            assert abs(d_tr[-1] - np.exp(x - x.max()).sum()) <= 1e-12 * d_tr[-1]
+
+
+def test_safe_softmax_reduces_to_textbook_and_survives_large_inputs():
+    rng = np.random.default_rng(1)
+    x = rng.normal(0, 3, (5, 40))
+    np.testing.assert_allclose(oracle.safe_softmax(x), oracle.naive_softmax(x), rtol=1e-13)
+    big = np.array([1000.0, 999.0, 990.0])
+    y = oracle.safe_softmax(big)
+    assert np.all(np.isfinite(y)) and abs(y.sum() - 1) < 1e-15
+    np.testing.assert_allclose(y, oracle.safe_softmax(big - 1000.0), rtol=1e-15)
+
+
+# ---------------------------------------------------------------------------
+# Blockwise online update inside attention (§2.2) == two-pass safe softmax
+# ---------------------------------------------------------------------------
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("sd", [1.0, 3.0])
+def test_blockwise_online_attention_equals_two_pass(causal, sd):
+    rng = np.random.default_rng(2 + int(causal))
+    N, d = 37, 8
+    q = rng.normal(0, sd, (N, d))
+    k = rng.normal(0, sd, (N, d))
+    v = rng.normal(0, 1, (N, d))
+    scale = 1 / math.sqrt(d)
+    o_ref, lse_ref, p_ref = oracle.head_forward_rows(q, k, v, scale, causal)
+    for trial in range(6):
+        cuts = np.sort(rng.choice(np.arange(1, N), size=rng.integers(0, 8), replace=False))
+        sizes = np.diff(np.concatenate([[0], cuts, [N]])).tolist()
+        o, m, dsum = oracle.blockwise_online_attention(q, k, v, scale, sizes, causal)
+        np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+        np.testing.assert_allclose(m + np.log(dsum), lse_ref, rtol=1e-12, atol=1e-12)
+    # fixed block size form, including a ragged last block
+    o, _, _ = oracle.blockwise_online_attention(q, k, v, scale, 16, causal)
+    np.testing.assert_allclose(o, o_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_blockwise_update_running_max_and_normaliser():
+    # after the last block m is the row max of the scaled scores and d = Σ e^{S - m}
+    rng = np.random.default_rng(4)
+    q = rng.normal(0, 2, (5, 4))
+    k = rng.normal(0, 2, (11, 4))
+    v = rng.normal(0, 1, (11, 4))
+    _, m, dsum = oracle.blockwise_online_attention(q, k, v, 0.5, [3, 3, 5])
+    s = 0.5 * q @ k.T
+    np.testing.assert_allclose(m, s.max(axis=1), rtol=1e-15)
+    np.testing.assert_allclose(dsum, np.exp(s - s.max(axis=1, keepdims=True)).sum(axis=1), rtol=1e-13)
+
+
+# ---------------------------------------------------------------------------
+# Forward: invariants, closed forms, library special case
+# ---------------------------------------------------------------------------
+
+def _rand(shape, seed, sd=1.0):
+    return np.random.default_rng(seed).normal(0, sd, shape)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_probability_rows_sum_to_one(causal):
+    q, k, v = _rand((16, 8), 5), _rand((16, 8), 6), _rand((16, 8), 7)
+    _, _, p = oracle.head_forward_rows(q, k, v, 0.3, causal)
+    np.testing.assert_allclose(p.sum(axis=1), 1.0, rtol=0, atol=1e-13)
+    if causal:
+        assert np.all(np.triu(p, 1) == 0)
+
+
+def test_zero_queries_give_mean_of_values_and_log_n():
+    B, H, N, d = 1, 2, 12, 4
+    q = np.zeros((B, H, N, d))
+    k, v = _rand((B, H, N, d), 8), _rand((B, H, N, d), 9)
+    o, lse = oracle.attention_forward(q, k, v, 0.7, causal=False)
+    np.testing.assert_allclose(o, np.broadcast_to(v.mean(axis=2, keepdims=True), o.shape), rtol=1e-13, atol=1e-15)
+    np.testing.assert_allclose(lse, math.log(N), rtol=1e-14)
+    o, lse = oracle.attention_forward(q, k, v, 0.7, causal=True)
+    prefix_mean = np.cumsum(v, axis=2) / np.arange(1, N + 1)[None, None, :, None]
+    np.testing.assert_allclose(o, prefix_mean, rtol=1e-12, atol=1e-14)
+    np.testing.assert_allclose(lse, np.broadcast_to(np.log(np.arange(1, N + 1)), lse.shape), rtol=1e-14)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_constant_values_give_constant_output(causal):
+    q, k = _rand((1, 1, 20, 8), 10, 3.0), _rand((1, 1, 20, 8), 11, 3.0)
+    v = np.ones((1, 1, 20, 8))
+    o, _ = oracle.attention_forward(q, k, v, 1 / math.sqrt(8), causal)
+    np.testing.assert_allclose(o, 1.0, rtol=0, atol=1e-13)
+
+
+def _torch_sdpa(q, k, v, scale, causal):
+    G = q.shape[1] // k.shape[1]
+    tq = torch.tensor(q)
+    tk = torch.tensor(k).repeat_interleave(G, dim=1)
+    tv = torch.tensor(v).repeat_interleave(G, dim=1)
+    return torch.nn.functional.scaled_dot_product_attention(tq, tk, tv, is_causal=causal, scale=scale).numpy()
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 2), (3, 1)])
+def test_forward_matches_torch_sdpa_fp64(causal, Hq, Hkv):
+    B, N, d = 2, 19, 8
+    q = _rand((B, Hq, N, d), 12)
+    k = _rand((B, Hkv, N, d), 13)
+    v = _rand((B, Hkv, N, d), 14)
+    o, lse = oracle.attention_forward(q, k, v, 1 / math.sqrt(d), causal)
+    np.testing.assert_allclose(o, _torch_sdpa(q, k, v, 1 / math.sqrt(d), causal), rtol=1e-12, atol=1e-13)
+    # LSE against torch.logsumexp of the masked scaled scores
+    G = Hq // Hkv
+    s = torch.einsum("bhid,bhjd->bhij", torch.tensor(q),
+                     torch.tensor(k).repeat_interleave(G, dim=1)) / math.sqrt(d)
+    if causal:
+        s = s.masked_fill(torch.ones(N, N, dtype=torch.bool).triu(1), -math.inf)
+    np.testing.assert_allclose(lse, torch.logsumexp(s, dim=-1).numpy(), rtol=1e-13)
+
+
+def test_gqa_equals_repeated_heads():
+    B, Hq, Hkv, N, d = 1, 4, 2, 10, 4
+    q = _rand((B, Hq, N, d), 15)
+    k, v = _rand((B, Hkv, N, d), 16), _rand((B, Hkv, N, d), 17)
+    o, lse = oracle.attention_forward(q, k, v, 0.5, True)
+    o2, lse2 = oracle.attention_forward(q, np.repeat(k, 2, axis=1), np.repeat(v, 2, axis=1), 0.5, True)
+    np.testing.assert_array_equal(o, o2)
+    np.testing.assert_array_equal(lse, lse2)
+
+
+def test_head_forward_rows_subset_equals_full():
+    q, k, v = _rand((30, 4), 18), _rand((30, 4), 19), _rand((30, 4), 20)
+    rows = np.array([0, 7, 29])
+    o, lse, _ = oracle.head_forward_rows(q, k, v, 0.4, True)
+    o_r, lse_r, _ = oracle.head_forward_rows(q, k, v, 0.4, True, rows)
+    np.testing.assert_array_equal(o_r, o[rows])
+    np.testing.assert_array_equal(lse_r, lse[rows])
+
+
+# ---------------------------------------------------------------------------
+# Backward: finite differences, invariants, library autograd
+# ---------------------------------------------------------------------------
+
+def _loss(q, k, v, do, scale, causal):
+    o, _ = oracle.attention_forward(q, k, v, scale, causal)
+    return float(np.sum(o * do))
+
+
+@pytest.mark.parametrize("N,d,Hq,Hkv,causal", [
+    (1, 1, 1, 1, False), (3, 4, 1, 1, True), (8, 4, 2, 1, False), (17, 1, 2, 2, True), (8, 4, 2, 1, True),
+])
+def test_backward_matches_central_finite_differences(N, d, Hq, Hkv, causal):
+    B = 1
+    scale = 1 / math.sqrt(d)
+    q = _rand((B, Hq, N, d), 21)
+    k = _rand((B, Hkv, N, d), 22)
+    v = _rand((B, Hkv, N, d), 23)
+    do = _rand((B, Hq, N, d), 24)
+    dq, dk, dv, _, _ = oracle.attention_backward(q, k, v, do, scale, causal)
+    h = 1e-6
+    for name, x, g in (("q", q, dq), ("k", k, dk), ("v", v, dv)):
+        num = np.zeros_like(x)
+        it = np.nditer(x, flags=["multi_index"])
+        for _ in it:
+            idx = it.multi_index
+            xp, xm = x.copy(), x.copy()
+            xp[idx] += h
+            xm[idx] -= h
+            args = {"q": q, "k": k, "v": v}
+            args[name] = xp
+            fp = _loss(args["q"], args["k"], args["v"], do, scale, causal)
+            args[name] = xm
+            fm = _loss(args["q"], args["k"], args["v"], do, scale, causal)
+            num[idx] = (fp - fm) / (2 * h)
+        err = np.linalg.norm(num - g) / max(np.linalg.norm(g), 1e-30)
+        assert err <= 1e-6, (name, err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_invariants(causal):
+    # rows of P sum to one  =>  Σ_keys dV = Σ_queries dO (per kv head, over its
+    # query heads) and Σ_keys dS = 0 per query row  =>  Σ_keys dK = 0.
+    B, Hq, Hkv, N, d = 2, 4, 2, 24, 8
+    q, k, v = _rand((B, Hq, N, d), 25), _rand((B, Hkv, N, d), 26), _rand((B, Hkv, N, d), 27)
+    do = _rand((B, Hq, N, d), 28)
+    dq, dk, dv, _, _ = oracle.attention_backward(q, k, v, do, 0.35, causal)
+    G = Hq // Hkv
+    do_sum = do.reshape(B, Hkv, G, N, d).sum(axis=(2, 3))
+    np.testing.assert_allclose(dv.sum(axis=2), do_sum, rtol=1e-12, atol=1e-12)
+    np.testing.assert_allclose(dk.sum(axis=2), 0.0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_matches_torch_autograd_fp64(causal):
+    B, Hq, Hkv, N, d = 1, 4, 2, 21, 8
+    scale = 1 / math.sqrt(d)
+    q, k, v = _rand((B, Hq, N, d), 29), _rand((B, Hkv, N, d), 30), _rand((B, Hkv, N, d), 31)
+    do = _rand((B, Hq, N, d), 32)
+    dq, dk, dv, o, _ = oracle.attention_backward(q, k, v, do, scale, causal)
+    tq, tk, tv = (torch.tensor(x, requires_grad=True) for x in (q, k, v))
+    G = Hq // Hkv
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(G, 1), tv.repeat_interleave(G, 1), is_causal=causal, scale=scale)
+    out.backward(torch.tensor(do))
+    np.testing.assert_allclose(o, out.detach().numpy(), rtol=1e-12, atol=1e-13)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy(), rtol=1e-10, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_sampled_backward_equals_full(causal):
+    B, Hq, Hkv, N, d = 1, 2, 1, 40, 4
+    q, k, v = _rand((B, Hq, N, d), 33), _rand((B, Hkv, N, d), 34), _rand((B, Hkv, N, d), 35)
+    do = _rand((B, Hq, N, d), 36)
+    dq, dk, dv, _, _ = oracle.attention_backward(q, k, v, do, 0.5, causal)
+    qr, kr = np.array([0, 5, 39]), np.array([1, 20, 39])
+    dq_r, dk_r, dv_r = oracle.head_backward_sampled(q[0], k[0, 0], v[0, 0], do[0], 0.5, causal, qr, kr, row_chunk=16)
+    np.testing.assert_allclose(dq_r, dq[0][:, qr], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dk_r, dk[0, 0][kr], rtol=1e-12, atol=1e-13)
+    np.testing.assert_allclose(dv_r, dv[0, 0][kr], rtol=1e-12, atol=1e-13)
+
+
+def test_flop_count():
+    # 4·B·Hq·N²·d, halved when causal
+    assert oracle.attention_flops(8, 16, 2048, 128, False) == 274877906944.0
+    assert oracle.attention_flops(8, 16, 2048, 128, True) == 137438953472.0
+    assert oracle.attention_flops(1, 2, 128, 64, False) == 8388608.0
+
+
+# ---------------------------------------------------------------------------
+# Planted mistakes: each must be caught by one of the pins above
+# ---------------------------------------------------------------------------
+
+def _pins_pass():
+    """Run a compact subset of the pins; return False if any fails."""
+    checks = [
+        lambda: test_forward_matches_torch_sdpa_fp64(True, 4, 2),
+        lambda: test_forward_matches_torch_sdpa_fp64(False, 2, 2),
+        lambda: test_zero_queries_give_mean_of_values_and_log_n(),
+        lambda: test_backward_matches_torch_autograd_fp64(True),
+        lambda: test_backward_invariants(True),
+    ]
+    for c in checks:
+        try:
+            c()
+        except AssertionError:
+            return False
+    return True
+
+
+def test_pins_pass_on_unmodified_oracle():
+    assert _pins_pass()
+
+
+def _mut_scores_no_scale(qh, kh, scale, causal, rows=None, _orig=oa._scores):
+    return _orig(qh, kh, 1.0, causal, rows)
+
+
+def _mut_scores_wrong_mask(qh, kh, scale, causal, rows=None, _orig=oa._scores):
+    # masks j >= i instead of j > i (drops the diagonal), keeping row 0 alive
+    s = _orig(qh, kh, scale, False, rows)
+    if causal:
+        r = np.arange(qh.shape[0]) if rows is None else rows
+        mask = (np.arange(kh.shape[0])[None, :] >= r[:, None]) & (r[:, None] > 0)
+        s = np.where(mask, -np.inf, s)
+    return s
+
+
+def _mut_scores_transposed(qh, kh, scale, causal, rows=None, _orig=oa._scores):
+    return _orig(kh, qh, scale, causal, rows)
+
+
+@pytest.mark.parametrize("mutant", [_mut_scores_no_scale, _mut_scores_wrong_mask, _mut_scores_transposed])
+def test_planted_score_mistakes_are_caught(monkeypatch, mutant):
+    monkeypatch.setattr(oa, "_scores", mutant)
+    assert not _pins_pass()
+
+
+def test_planted_backward_mistake_is_caught(monkeypatch):
+    # drop the D term of dS = P ∘ (dP − D) by zeroing dO·O inside the oracle
+    orig_sum = np.sum
+
+    def bad_sum(a, *args, **kw):
+        out = orig_sum(a, *args, **kw)
+        if kw.get("keepdims") and kw.get("axis") == 1:
+            return out * 0.0
+        return out
+
+    monkeypatch.setattr(oa.np, "sum", bad_sum)
+    try:
+        assert not _pins_pass()
+    finally:
+        monkeypatch.setattr(oa.np, "sum", orig_sum)
