@@ -1,0 +1,401 @@
+"""Benchmark: exact attention forward + backward on B200, through the C ABI.
+
+One step = one forward pass (fa_fwd) and one backward pass (fa_bwd) over the
+whole workload, with inputs resident in HBM.  The default workload is
+B=8, Hq=Hkv=16, N=2048, d=128, non-causal, bf16, seeded synthetic N(0,1)
+inputs.  Prints ONE JSON line (rank 0).
+
+  python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
+                  [--workload NAME] [--no-e2e] [--no-cpu-baseline]
+
+Multi-GPU (launched by torchrun): every rank runs its own independent problem
+of the same size (weak scaling; attention over distinct batches needs no data
+exchange), timed with CUDA events, max over ranks.
+
+--impl reference times the fp64 CPU oracle on this host's cores on a bounded
+sample of the same workload (one (batch, head) slice per step).
+"""
+
+from __future__ import annotations
+
+import argparse
+import json
+import math
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import threading
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+if ROOT not in sys.path:
+    sys.path.insert(0, ROOT)
+
+METRIC = "attention fwd and fwd+bwd TFLOPS (bf16) and % of B200 dense BF16 tensor peak"
+NOMINAL_PEAK_TFLOPS = 2250.0
+
+
+def _peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"bf16_tflops": float(d["bf16_tflops"]), "bf16_tflops_sustained": float(d["bf16_tflops_sustained"]),
+                "hbm_gbs": float(d["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def _blas_threads():
+    try:
+        from threadpoolctl import threadpool_info
+        n = [i.get("num_threads", 1) for i in threadpool_info() if i.get("user_api") == "blas"]
+        return max(n) if n else 1
+    except Exception:
+        return os.cpu_count() or 1
+
+
+# ----------------------------------------------------------------- clocks
+class ClockSampler:
+    """Samples nvidia-smi clocks and throttle reasons while running."""
+
+    FIELDS = ("index,clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,"
+              "clocks_event_reasons.hw_slowdown,clocks_event_reasons.hw_thermal_slowdown,"
+              "clocks_event_reasons.sw_thermal_slowdown,clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, gpu_index: int):
+        self.gpu = gpu_index
+        self.proc = None
+        self.out = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+
+    def __enter__(self):
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", f"--id={self.gpu}", f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "100"], stdout=self.out, stderr=subprocess.DEVNULL)
+            time.sleep(0.3)
+        except Exception:
+            self.proc = None
+        return self
+
+    def __exit__(self, *a):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except Exception:
+                self.proc.kill()
+
+    def summary(self):
+        self.out.flush()
+        try:
+            lines = open(self.out.name).read().strip().splitlines()
+        except Exception:
+            lines = []
+        os.unlink(self.out.name)
+        mhz, maxes, reasons, power = [], [], set(), []
+        for ln in lines:
+            parts = [p.strip() for p in ln.split(",")]
+            if len(parts) < 9:
+                continue
+            try:
+                sm, smax = float(parts[1]), float(parts[2])
+            except ValueError:
+                continue
+            mhz.append(sm)
+            maxes.append(smax)
+            try:
+                power.append(float(parts[3]))
+            except ValueError:
+                pass
+            for name, val in zip(("hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"),
+                                 parts[5:9]):
+                if val.lower().startswith("active"):
+                    reasons.add(name)
+        if not mhz:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": [], "samples": 0}
+        return {"sm_mhz": statistics.median(mhz), "sm_max_mhz": max(maxes), "reasons": sorted(reasons),
+                "samples": len(mhz), "power_w_max": max(power) if power else None}
+
+
+# ------------------------------------------------------------- CPU oracle
+def cpu_oracle_sample(w, seconds: float, max_heads: int | None = None):
+    """Time the fp64 oracle's forward+backward on (batch 0, head h) slices of
+    the workload until `seconds` of CPU work have been spent.  Returns
+    (TFLOPS, heads, elapsed seconds)."""
+    import numpy as np
+
+    import oracle
+    from exact_attention_104_b200.workloads import make_inputs
+
+    q, k, v, do = make_inputs(w, "cpu")
+    G = w.G
+    heads, t_total = 0, 0.0
+    while True:
+        h = heads % w.Hq
+        sl = lambda t, hh: t[0:1, hh:hh + 1].float().numpy().astype(np.float64)  # noqa: E731
+        qs, dos = sl(q, h), sl(do, h)
+        ks, vs = sl(k, h // G), sl(v, h // G)
+        t0 = time.perf_counter()
+        oracle.attention_backward(qs, ks, vs, dos, w.scale, w.causal)
+        t_total += time.perf_counter() - t0
+        heads += 1
+        if t_total >= seconds or (max_heads is not None and heads >= max_heads):
+            break
+    flops_per_head = 3.5 * oracle.attention_flops(1, 1, w.N, w.d, w.causal)
+    return flops_per_head * heads / t_total / 1e12, heads, t_total
+
+
+def run_reference(args, w, rank, world):
+    """The reference arm: the fp64 oracle on the host cores, one (b, h) slice
+    of the workload per step.  Rank 0 only."""
+    if rank != 0:
+        return
+    import oracle
+
+    flops_per_step = 3.5 * oracle.attention_flops(1, 1, w.N, w.d, w.causal)
+    for _ in range(args.warmup):
+        cpu_oracle_sample(w, 0.0, max_heads=1)
+    times = []
+    for _ in range(args.steps):
+        _, _, t = cpu_oracle_sample(w, 0.0, max_heads=1)
+        times.append(t)
+    total = sum(times)
+    value = flops_per_step * args.steps / total / 1e12
+    cores = _blas_threads()
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
+                   "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
+                         "sample": f"one (batch 0, head h) slice of {w.describe()} per step, fwd+bwd in fp64"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
+# ------------------------------------------------------------------- ours
+def run_ours(args, w, rank, world, local_rank):
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_104_b200 import binding
+    from exact_attention_104_b200.workloads import make_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    stream = torch.cuda.current_stream()
+
+    # independent problem per rank (weak scaling): same shape, rank-specific seed
+    q, k, v, do = make_inputs(w, dev, seed=w.seed + 7919 * rank)
+    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
+    o = torch.empty_like(q)
+    lse = torch.empty(B, Hq, N, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    ws_bytes = binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d)
+    ws = torch.empty(ws_bytes, dtype=torch.uint8, device=dev)
+    scale = w.scale
+
+    def fwd(prof=None):
+        if prof is not None:
+            binding.fa_profile_next(*prof)
+        st = binding.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, w.causal, scale, stream)
+        if st:
+            raise binding.FAError(st, "fa_fwd")
+
+    def bwd(prof=None):
+        if prof is not None:
+            binding.fa_profile_next(*prof)
+        st = binding.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, w.causal, scale, ws, ws_bytes,
+                            stream)
+        if st:
+            raise binding.FAError(st, "fa_bwd")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        fwd()
+        bwd()
+    torch.cuda.synchronize()
+    if binding.fa_device_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+
+    # timed region: K whole steps, plus per-kernel events on the same stream
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    f_ev = [(ev(), ev()) for _ in range(K)]
+    b_ev = [(ev(), ev()) for _ in range(K)]
+    start, stop = ev(), ev()
+    for e in [x for pair in f_ev + b_ev for x in pair] + [start, stop]:
+        e.record(stream)  # creates the event handles before the timed region
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        start.record(stream)
+        for i in range(K):
+            fwd(f_ev[i])
+            bwd(b_ev[i])
+        stop.record(stream)
+        barrier()
+    clocks = clk.summary()
+    if binding.fa_device_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_total = max_over_ranks(start.elapsed_time(stop))
+    ms_fwd_kernel = max_over_ranks(sum(a.elapsed_time(b) for a, b in f_ev) / K)
+    ms_bwd_kernel = max_over_ranks(sum(a.elapsed_time(b) for a, b in b_ev) / K)
+
+    F = w.fwd_flops()
+    step_flops = 3.5 * F
+    ms_step = ms_total / K
+    value = step_flops * world * K / (ms_total * 1e-3) / 1e12
+    fwd_tflops = F / (ms_fwd_kernel * 1e-3) / 1e12
+    bwd_main_tflops = 2.5 * F / (ms_bwd_kernel * 1e-3) / 1e12
+    peaks = _peaks()
+
+    # separate fwd-only and bwd-only throughput (whole calls), outside the main timed region
+    def time_calls(fn, reps):
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(reps):
+            fn()
+        b.record(stream)
+        barrier()
+        return max_over_ranks(a.elapsed_time(b)) / reps
+
+    reps = max(3, min(K, 50))
+    ms_fwd_call = time_calls(fwd, reps)
+    ms_bwd_call = time_calls(bwd, reps)
+
+    # end to end through the public API with host buffers
+    e2e = None
+    if not args.no_e2e:
+        hq = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        outs = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+        h2d = sum(t.numel() * t.element_size() for t in hq)
+        d2h = sum(t.numel() * t.element_size() for t in outs)
+        dev_in = (q, k, v, do)
+        ke = max(3, min(K, 30))
+
+        def e2e_step():
+            for hsrc, ddst in zip(hq, dev_in):
+                ddst.copy_(hsrc, non_blocking=True)
+            fwd()
+            bwd()
+            for ddst, dsrc in zip(outs, (o, lse, dq, dk, dv)):
+                ddst.copy_(dsrc, non_blocking=True)
+
+        e2e_step()
+        ms_e2e = time_calls(e2e_step, ke)
+        e2e = {"value": step_flops * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tflops, heads, secs = cpu_oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": tflops, "unit": "TFLOPS", "cores": _blas_threads(), "kind": "oracle",
+               "sample": f"{heads} (batch 0, head) slices of {w.describe()}, fwd+bwd in fp64, {secs:.1f} s"}
+
+    # dominant kernel: the backward dK/dV/dQ kernel (2.5x the forward FLOPs)
+    bwd_main_flops = 2.5 * F
+    roof = {
+        "kernel": "fa_bwd_kernel",
+        "bound": "tensor",
+        "achieved": bwd_main_tflops,
+        "peak": peaks["bf16_tflops"],
+        "unit": "TFLOP/s",
+        "frac": bwd_main_tflops / peaks["bf16_tflops"],
+        "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
+        "flops_per_launch": bwd_main_flops,
+        "ms_per_launch": ms_bwd_kernel,
+        "traffic": args.traffic_bytes if args.traffic_bytes else None,
+    }
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": B, "Hq": Hq, "Hkv": Hkv, "N": N, "d": d, "causal": w.causal,
+                   "qk_std": w.qk_std, "global_batch": B * world, "seq_len": N,
+                   "parallelism": f"dp{world} (independent problem per GPU)",
+                   "l2": "inputs larger than L2 (Q,K,V,O,dO 64 MiB each; no flush needed)"},
+        "fwd_tflops": fwd_tflops,
+        "bwd_tflops": 2.5 * F / (ms_bwd_call * 1e-3) / 1e12,
+        "fwd_bwd_tflops": value / world,
+        "pct_of_peak": {"fwd_vs_2250_nominal": fwd_tflops / NOMINAL_PEAK_TFLOPS,
+                        "fwd_vs_measured": fwd_tflops / peaks["bf16_tflops"],
+                        "fwd_bwd_vs_2250_nominal": value / world / NOMINAL_PEAK_TFLOPS,
+                        "fwd_bwd_vs_measured": value / world / peaks["bf16_tflops"]},
+        "ms": {"fwd_kernel": ms_fwd_kernel, "bwd_main_kernel": ms_bwd_kernel, "fwd_call": ms_fwd_call,
+               "bwd_call": ms_bwd_call},
+        "roofline": roof,
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 4 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=200)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--workload", default=None)
+    ap.add_argument("--no-e2e", action="store_true")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-seconds", type=float, default=10.0)
+    ap.add_argument("--traffic-bytes", type=float, default=0.0,
+                    help="DRAM bytes per launch of the dominant kernel from an ncu capture, if known")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+
+    from exact_attention_104_b200.workloads import BENCH_WORKLOAD, WORKLOADS
+
+    w = WORKLOADS[args.workload or BENCH_WORKLOAD]
+    rank = int(os.environ.get("RANK", "0"))
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    local_rank = int(os.environ.get("LOCAL_RANK", "0"))
+
+    if args.impl == "reference":
+        run_reference(args, w, rank, world)
+        return
+
+    if world > 1:
+        import datetime
+
+        import torch
+        import torch.distributed as dist
+
+        torch.cuda.set_device(local_rank)
+        dist.init_process_group("nccl", timeout=datetime.timedelta(seconds=120),
+                                device_id=torch.device("cuda", local_rank))
+    try:
+        run_ours(args, w, rank, world, local_rank)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

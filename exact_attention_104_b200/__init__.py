@@ -1,0 +1,19 @@
+"""Exact attention (FlashAttention-style forward and backward) for NVIDIA B200.
+
+The compute lives in ``libfa_b200.so`` (hand-written sm_100a CUDA behind the C
+ABI declared in ``include/fa.h``); this package only marshals arguments.
+"""
+
+from .binding import (  # noqa: F401
+    FAError,
+    fa_fwd,
+    fa_bwd,
+    fa_bwd_workspace_bytes,
+    fa_device_status,
+    fa_profile_next,
+    fa_status_string,
+    attention_forward,
+    attention_backward,
+    lib,
+    LIB_PATH,
+)

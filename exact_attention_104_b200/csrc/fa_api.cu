@@ -1,0 +1,350 @@
+// Host side of libfa_b200.so: argument checks, TMA descriptor encoding and
+// kernel launches behind the C ABI declared in include/fa.h.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+// Device error word: kernels that abandon a bounded wait record it here.
+__device__ int g_fa_err = 0;
+
+namespace {
+
+constexpr int kMaxDevices = 64;
+long long g_wait_cap = 1LL << 31;
+
+// pending one-shot profiling events of this host thread (fa_profile_next)
+thread_local cudaEvent_t t_prof_start = nullptr;
+thread_local cudaEvent_t t_prof_stop = nullptr;
+
+struct ProfileScope {
+  cudaEvent_t start, stop;
+  cudaStream_t stream;
+  explicit ProfileScope(cudaStream_t s) : start(t_prof_start), stop(t_prof_stop), stream(s) {
+    t_prof_start = t_prof_stop = nullptr;
+    if (start) cudaEventRecord(start, stream);
+  }
+  ~ProfileScope() {
+    if (stop) cudaEventRecord(stop, stream);
+  }
+};
+
+typedef CUresult (*EncodeTiledFn)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                  const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                  CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static std::once_flag once;
+  std::call_once(once, [] {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(p);
+  });
+  return fn;
+}
+
+// 2-D view [rows, d] of a bf16 tensor; boxes of 64 columns (128 bytes, the
+// swizzle span) by `box_rows` rows, 128-byte swizzled in shared memory.
+bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, int d, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 2};
+  cuuint32_t box[2] = {64, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
+struct DeviceInfo {
+  bool checked = false;
+  bool sm100 = false;
+  int sms = 0;
+  int* err = nullptr;
+};
+DeviceInfo g_dev[kMaxDevices];
+std::mutex g_dev_mu;
+
+// Checks for an sm_100 device and resolves the error word's device address
+// (once per device, with that device current).
+fa_status current_device(DeviceInfo** out) {
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lk(g_dev_mu);
+  DeviceInfo& di = g_dev[dev];
+  if (!di.checked) {
+    int major = 0, minor = 0, sms = 0;
+    cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, dev);
+    cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, dev);
+    cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev);
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_err) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    di.sm100 = (major == 10 && minor == 0);
+    di.sms = sms;
+    di.err = static_cast<int*>(p);
+    di.checked = true;
+  }
+  if (!di.sm100) return FA_ERR_UNSUPPORTED;
+  *out = &di;
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+struct Range {
+  uintptr_t lo, hi;  // [lo, hi)
+};
+Range span(const void* p, size_t bytes) {
+  const uintptr_t a = reinterpret_cast<uintptr_t>(p);
+  return Range{a, a + bytes};
+}
+bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
+
+// Size checks shared by both passes.  Returns FA_OK, or the status to report;
+// sets *empty for a problem with nothing to compute.
+fa_status check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* empty) {
+  *empty = false;
+  if (B < 0 || N < 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || N == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || Hq > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * N >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
+                     int B, int Hq, cudaStream_t stream) {
+  using C = fa::FwdCfg<D>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  dim3 grid((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
+  ProfileScope prof(stream);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL>
+fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
+  using C = fa::BwdCfg<D>;
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  dim3 grid((p.N / C::BC) * C::NDH, Hkv, B);
+  ProfileScope prof(stream);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_bwd_pre(const void* o, const void* dout, const float* lse, float* dvec, float* lse2, float* dqacc,
+                         long long rows, int sms, cudaStream_t stream) {
+  const long long dq_vec4 = rows * D / 4;
+  long long want = rows * (D / 8);
+  if (dq_vec4 > want) want = dq_vec4;
+  long long blocks = (want + 255) / 256;
+  const long long cap = (long long)sms * 8;
+  if (blocks > cap) blocks = cap;
+  if (blocks < 1) blocks = 1;
+  fa::fa_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc, rows,
+      dq_vec4);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+}  // namespace
+
+extern "C" {
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument";
+    case FA_ERR_UNSUPPORTED: return "unsupported configuration";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device wait timed out";
+  }
+  return "unknown status";
+}
+
+fa_status fa_profile_next(void* start_event, void* stop_event) {
+  if ((start_event == nullptr) != (stop_event == nullptr)) return FA_ERR_INVALID_ARG;
+  t_prof_start = static_cast<cudaEvent_t>(start_event);
+  t_prof_stop = static_cast<cudaEvent_t>(stop_event);
+  return FA_OK;
+}
+
+fa_status fa_set_wait_cap(long long cycles) {
+  if (cycles < 0) return FA_ERR_INVALID_ARG;
+  g_wait_cap = cycles == 0 ? (1LL << 31) : cycles;
+  return FA_OK;
+}
+
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
+  bool empty = false;
+  if (check_sizes(B, Hq, Hkv, N, d, 1.f, &empty) != FA_OK) return 0;
+  const size_t rows = (size_t)B * Hq * N;
+  return 2 * round256(rows * 4) + round256(rows * (size_t)d * 4);
+}
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
+                 int d, int causal, float scale, void* stream) {
+  bool empty = false;
+  fa_status st = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
+  const Range rq = span(q, qbytes), rk = span(k, kvbytes), rv = span(v, kvbytes);
+  const Range ro = span(o, qbytes), rl = span(lse, (size_t)B * Hq * N * 4);
+  for (Range out : {ro, rl})
+    for (Range in : {rq, rk, rv})
+      if (overlap(out, in)) return FA_ERR_INVALID_ARG;
+  if (overlap(ro, rl)) return FA_ERR_INVALID_ARG;
+
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+
+  CUtensorMap tq, tk, tv;
+  const uint64_t qrows = (uint64_t)B * Hq * N, kvrows = (uint64_t)B * Hkv * N;
+  if (!make_map(&tq, q, qrows, d, 128) || !make_map(&tk, k, kvrows, d, 128) || !make_map(&tv, v, kvrows, d, 128))
+    return FA_ERR_CUDA;
+  fa::FwdParams p;
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = N / 128;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.wait_cap = g_wait_cap;
+  p.err = di->err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return causal ? launch_fwd<64, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<64, false>(tq, tk, tv, p, B, Hq, s);
+    case 128: return causal ? launch_fwd<128, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<128, false>(tq, tk, tv, p, B, Hq, s);
+    case 256: return causal ? launch_fwd<256, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<256, false>(tq, tk, tv, p, B, Hq, s);
+  }
+  return FA_ERR_UNSUPPORTED;
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,
+                 void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status st = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !workspace) return FA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)lse, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_workspace_bytes(B, Hq, Hkv, N, d);
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)B * Hq * N;
+  const size_t qbytes = rows * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
+  const Range ins[6] = {span(q, qbytes), span(k, kvbytes), span(v, kvbytes),
+                        span(o, qbytes), span(lse, rows * 4), span(dout, qbytes)};
+  const Range outs[4] = {span(dq, qbytes), span(dk, kvbytes), span(dv, kvbytes), span(workspace, need)};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 6; ++j)
+      if (overlap(outs[i], ins[j])) return FA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outs[i], outs[j])) return FA_ERR_INVALID_ARG;
+  }
+
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  float* dvec = reinterpret_cast<float*>(ws);
+  float* lse2 = reinterpret_cast<float*>(ws + round256(rows * 4));
+  float* dqacc = reinterpret_cast<float*>(ws + 2 * round256(rows * 4));
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  switch (d) {
+    case 64: st = launch_bwd_pre<64>(o, dout, lse, dvec, lse2, dqacc, (long long)rows, di->sms, s); break;
+    case 128: st = launch_bwd_pre<128>(o, dout, lse, dvec, lse2, dqacc, (long long)rows, di->sms, s); break;
+    default: st = launch_bwd_pre<256>(o, dout, lse, dvec, lse2, dqacc, (long long)rows, di->sms, s); break;
+  }
+  if (st != FA_OK) return st;
+
+  CUtensorMap tq, tk, tv, tdo;
+  const uint64_t kvrows = (uint64_t)B * Hkv * N;
+  if (!make_map(&tq, q, rows, d, 64) || !make_map(&tdo, dout, rows, d, 64) || !make_map(&tk, k, kvrows, d, 128) ||
+      !make_map(&tv, v, kvrows, d, 128))
+    return FA_ERR_CUDA;
+  fa::BwdParams p;
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dqacc = dqacc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.wait_cap = g_wait_cap;
+  p.err = di->err;
+  switch (d) {
+    case 64: st = causal ? launch_bwd_main<64, true>(tq, tk, tv, tdo, p, B, Hkv, s) : launch_bwd_main<64, false>(tq, tk, tv, tdo, p, B, Hkv, s); break;
+    case 128: st = causal ? launch_bwd_main<128, true>(tq, tk, tv, tdo, p, B, Hkv, s) : launch_bwd_main<128, false>(tq, tk, tv, tdo, p, B, Hkv, s); break;
+    default: st = causal ? launch_bwd_main<256, true>(tq, tk, tv, tdo, p, B, Hkv, s) : launch_bwd_main<256, false>(tq, tk, tv, tdo, p, B, Hkv, s); break;
+  }
+  if (st != FA_OK) return st;
+
+  const long long n_vec4 = (long long)rows * d / 4;
+  long long blocks = (n_vec4 + 255) / 256;
+  if (blocks > (long long)di->sms * 8) blocks = (long long)di->sms * 8;
+  fa::fa_dq_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(dqacc, static_cast<__nv_bfloat16*>(dq), scale, n_vec4);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_device_status(void* stream) {
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  int host = 0;
+  const int zero = 0;
+  if (cudaMemcpy(&host, di->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
+  if (host != 0 && cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
+    return FA_ERR_CUDA;
+  return host != 0 ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,466 @@
+// Exact-attention backward pass for sm_100a.
+//
+// The pages only state that the backward pass does not keep the probability
+// matrix but recomputes it from Q, K, V and a few per-row statistics
+// ("Flash-Attention" concept page, "Core idea").  The formulas are the chain
+// rule on O = softmax(s·Q Kᵀ) V, with LSE saved by the forward pass:
+//   P = exp(s·Q Kᵀ − LSE),  dV = Pᵀ dO,  dP = dO Vᵀ,  D = rowsum(dO ∘ O),
+//   dS = P ∘ (dP − D),      dQ = s·dS K, dK = s·dSᵀ Q.
+//
+// Kernels:
+//   fa_bwd_pre_kernel   D = rowsum(dO∘O), LSE·log2e, zero the fp32 dQ accumulator
+//   fa_bwd_kernel       one CTA per (128-key tile, batch, kv head[, d-half]);
+//                       streams 64-row query tiles of every query head of the
+//                       GQA group; dK, dV accumulate in TMEM, dQ partials are
+//                       added to the fp32 accumulator in global memory
+//   fa_dq_convert_kernel dQ = bf16(s · accumulator)
+//
+// In fa_bwd_kernel every product runs on tcgen05 with fp32 TMEM accumulators:
+//   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ        (A, B from shared memory)
+//   dV += Pᵀ dO, dK += dSᵀ Q       (A = bf16 Pᵀ / dSᵀ written back to TMEM)
+//   dQᵀ = Kᵀ dSᵀ                   (A = K tile read MN-major, B = dSᵀ in smem)
+// Roles: warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 4-7 compute
+// (thread = key row: Pᵀ, dSᵀ), warps 8-11 drain (thread = d row of dQᵀ).
+// For d = 256, dK/dV/dQ do not fit TMEM for a full row, so two CTAs share a
+// key tile, each owning 128 of the 256 output columns and both recomputing Sᵀ
+// and dPᵀ over the full head dimension.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+template <int D>
+struct BwdCfg {
+  static constexpr int DH = D < 128 ? D : 128;  // output columns owned by one CTA
+  static constexpr int NDH = D / DH;            // CTAs per key tile
+  static constexpr int BR = 64;                 // query rows per step
+  static constexpr int BC = 128;                // keys per CTA
+  static constexpr int THREADS = 384;
+  static constexpr int KV_PANEL = BC * 128;     // 64 columns x 128 rows (bytes)
+  static constexpr int Q_PANEL = BR * 128;      // 64 columns x 64 rows
+  static constexpr int KV_BYTES = BC * D * 2;
+  static constexpr int Q_BYTES = BR * D * 2;
+  static constexpr int NSTAGE = (D == 64) ? 4 : (D == 128 ? 3 : 1);
+  static constexpr int LA = NSTAGE >= 2 ? 2 : 1;  // Sᵀ lookahead in steps
+  static constexpr int K_OFF = 0;
+  static constexpr int V_OFF = KV_BYTES;
+  static constexpr int DS_OFF = 2 * KV_BYTES;   // dSᵀ: 128 key rows x 64 queries (bf16), 16 KB
+  static constexpr int Q_OFF = DS_OFF + 16384;
+  static constexpr int DO_OFF = Q_OFF + NSTAGE * Q_BYTES;
+  static constexpr int LS_OFF = DO_OFF + NSTAGE * Q_BYTES;  // per stage: lse2[64], Dvec[64]
+  static constexpr int BAR_OFF = LS_OFF + NSTAGE * 512;
+  static constexpr int B_KVFULL = 0;
+  static constexpr int B_QFULL = 1;                  // + stage
+  static constexpr int B_QEMPTY = 1 + NSTAGE;        // + stage
+  static constexpr int B_SFULL = 1 + 2 * NSTAGE;     // + {0,1}
+  static constexpr int B_DPFULL = B_SFULL + 2;
+  static constexpr int B_PFULL = B_DPFULL + 1;   // + {0,1}: by step parity
+  static constexpr int B_DSFULL = B_PFULL + 2;
+  static constexpr int B_DQFULL = B_DSFULL + 1;
+  static constexpr int B_DQEMPTY = B_DQFULL + 1;
+  static constexpr int B_ACC = B_DQEMPTY + 1;
+  static constexpr int B_DRAIN = B_ACC + 1;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int DK_COL = 0;
+  static constexpr int DV_COL = DH;
+  static constexpr int ST_COL = 2 * DH;        // two 64-column Sᵀ buffers
+  static constexpr int DP_COL = 2 * DH + 128;  // dPᵀ (later dSᵀ bf16)
+  static constexpr int DQ_COL = 2 * DH + 192;  // dQᵀ
+  static constexpr uint32_t IDESC_ST = idesc_bf16_f32(128, BR, false, false);
+  static constexpr uint32_t IDESC_DKV = idesc_bf16_f32(128, DH, false, true);
+  static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, BR, true, true);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(DQ_COL + 64 <= TMEM_COLS, "TMEM budget");
+};
+
+// ------------------------------------------------------------ preprocess
+// One group of D/8 threads per row: D_i = Σ_c dO_ic·O_ic in fp32, and
+// lse2_i = LSE_i·log2e.  Also zeroes the fp32 dQ accumulator.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
+                                                         const __nv_bfloat16* __restrict__ dout,
+                                                         const float* __restrict__ lse, float* __restrict__ dvec,
+                                                         float* __restrict__ lse2, float* __restrict__ dqacc,
+                                                         long long rows, long long dq_vec4) {
+  constexpr int TPR = D / 8;
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  // zero the accumulator
+  float4* acc4 = reinterpret_cast<float4*>(dqacc);
+  for (long long i = tid; i < dq_vec4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
+  // row dots: rows are processed in rounds so that every lane of a group stays together
+  const long long groups = nthreads / TPR;
+  const long long gid = tid / TPR;
+  const int sub = (int)(tid % TPR);
+  for (long long r0 = 0; r0 < rows; r0 += groups) {
+    const long long r = r0 + gid;
+    float acc = 0.f;
+    if (r < rows && gid < groups) {
+      const uint4 ov = *reinterpret_cast<const uint4*>(o + r * D + sub * 8);
+      const uint4 dv = *reinterpret_cast<const uint4*>(dout + r * D + sub * 8);
+      const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
+      const __nv_bfloat162* d2 = reinterpret_cast<const __nv_bfloat162*>(&dv);
+#pragma unroll
+      for (int e = 0; e < 4; ++e) {
+        const float2 a = __bfloat1622float2(o2[e]);
+        const float2 c = __bfloat1622float2(d2[e]);
+        acc = fmaf(a.x, c.x, acc);
+        acc = fmaf(a.y, c.y, acc);
+      }
+    }
+#pragma unroll
+    for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+    if (r < rows && gid < groups && sub == 0) {
+      dvec[r] = acc;
+      lse2[r] = lse[r] * kLog2e;
+    }
+  }
+}
+
+__global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float* __restrict__ dqacc,
+                                                            __nv_bfloat16* __restrict__ dq, float scale,
+                                                            long long n_vec4) {
+  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
+  const long long nthreads = (long long)gridDim.x * blockDim.x;
+  for (long long i = tid; i < n_vec4; i += nthreads) {
+    const float4 a = reinterpret_cast<const float4*>(dqacc)[i];
+    uint2 w;
+    w.x = pack_bf16(a.x * scale, a.y * scale);
+    w.y = pack_bf16(a.z * scale, a.w * scale);
+    reinterpret_cast<uint2*>(dq)[i] = w;
+  }
+}
+
+struct BwdParams {
+  const float* lse2;
+  const float* dvec;
+  float* dqacc;
+  __nv_bfloat16* dk;
+  __nv_bfloat16* dv;
+  int N, Hq, Hkv, G;
+  float scale, scale_log2;
+  long long wait_cap;
+  int* err;
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8 * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int jt = blockIdx.x / C::NDH;  // key tile
+  const int dh = blockIdx.x % C::NDH;  // output column half
+  const int hkv = blockIdx.y;
+  const int b = blockIdx.z;
+  const int nqt = p.N / C::BR;
+  const int i_start = CAUSAL ? (jt * C::BC) / C::BR : 0;
+  const int per_head = nqt - i_start;
+  const int n = p.G * per_head;  // steps
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_KVFULL), 1);
+    for (int i = 0; i < C::NSTAGE; ++i) {
+      mbar_init(BAR(C::B_QFULL + i), 1);
+      mbar_init(BAR(C::B_QEMPTY + i), 1);
+    }
+    mbar_init(BAR(C::B_SFULL + 0), 1);
+    mbar_init(BAR(C::B_SFULL + 1), 1);
+    mbar_init(BAR(C::B_DPFULL), 1);
+    mbar_init(BAR(C::B_PFULL + 0), 4);
+    mbar_init(BAR(C::B_PFULL + 1), 4);
+    mbar_init(BAR(C::B_DSFULL), 4);
+    mbar_init(BAR(C::B_DQFULL), 1);
+    mbar_init(BAR(C::B_DQEMPTY), 4);
+    mbar_init(BAR(C::B_ACC), 1);
+    mbar_init(BAR(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const WaitCtx wc{abort_flag, p.err, p.wait_cap};
+
+  auto step_head = [&](int s) { return hkv * p.G + s / per_head; };
+  auto step_q0 = [&](int s) { return (i_start + s % per_head) * C::BR; };
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmDO);
+      const int kv_row = (b * p.Hkv + hkv) * p.N + jt * C::BC;
+      mbar_expect_tx(BAR(C::B_KVFULL), 2 * C::KV_BYTES);
+#pragma unroll
+      for (int pn = 0; pn < D / 64; ++pn) {
+        tma_load_2d(sbase + C::K_OFF + pn * C::KV_PANEL, &tmK, BAR(C::B_KVFULL), pn * 64, kv_row);
+        tma_load_2d(sbase + C::V_OFF + pn * C::KV_PANEL, &tmV, BAR(C::B_KVFULL), pn * 64, kv_row);
+      }
+      for (int s = 0; s < n; ++s) {
+        const int st = s % C::NSTAGE;
+        if (!mbar_wait(BAR(C::B_QEMPTY + st), ((s / C::NSTAGE) & 1) ^ 1, wc, 11)) break;
+        const int q_row = (b * p.Hq + step_head(s)) * p.N + step_q0(s);
+        const uint32_t bar = BAR(C::B_QFULL + st);
+        mbar_expect_tx(bar, 2 * C::Q_BYTES + 512);
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn) {
+          tma_load_2d(sbase + C::Q_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmQ, bar, pn * 64, q_row);
+          tma_load_2d(sbase + C::DO_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmDO, bar, pn * 64, q_row);
+        }
+        bulk_load(sbase + C::LS_OFF + st * 512, p.lse2 + q_row, 256, bar);
+        bulk_load(sbase + C::LS_OFF + st * 512 + 256, p.dvec + q_row, 256, bar);
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(BAR(C::B_KVFULL), 0, wc, 12);
+      tc_fence_after();
+      auto wait_q = [&](int s) -> bool {
+        const bool r = mbar_wait(BAR(C::B_QFULL + s % C::NSTAGE), (s / C::NSTAGE) & 1, wc, 13);
+        tc_fence_after();
+        return r;
+      };
+      // Sᵀ / dPᵀ: [128 keys x 64 queries] = (K or V tile) · (Q or dO tile)ᵀ over D
+      auto issue_xt = [&](uint32_t a_off, uint32_t b_off, int dcol) {
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int koff = (kk & 3) * 32;
+          const uint64_t da = sdesc_sw128(sbase + a_off + (kk >> 2) * C::KV_PANEL + koff, 16, 1024);
+          const uint64_t db = sdesc_sw128(sbase + b_off + (kk >> 2) * C::Q_PANEL + koff, 16, 1024);
+          mma_ss(tbase + dcol, da, db, C::IDESC_ST, kk > 0 ? 1u : 0u);
+        }
+      };
+      // dV or dK [128 keys x DH] += (Pᵀ or dSᵀ in TMEM) · (dO or Q tile)[:, dh half]
+      auto issue_acc = [&](int a_col, uint32_t b_off, int dcol, bool first) {
+#pragma unroll
+        for (int kk = 0; kk < C::BR / 16; ++kk) {
+          const uint64_t db =
+              sdesc_sw128(sbase + b_off + (dh * C::DH / 64) * C::Q_PANEL + kk * 2048, C::Q_PANEL, 1024);
+          mma_ts(tbase + dcol, tbase + a_col + kk * 8, db, C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+      // dQᵀ [128 d-rows x 64 queries] = K[:, dh half]ᵀ · dSᵀ over the 128 keys
+      auto issue_dq = [&]() {
+#pragma unroll
+        for (int kk = 0; kk < C::BC / 16; ++kk) {
+          const uint64_t da =
+              sdesc_sw128(sbase + C::K_OFF + (dh * C::DH / 64) * C::KV_PANEL + kk * 2048, C::KV_PANEL, 1024);
+          const uint64_t db = sdesc_sw128(sbase + C::DS_OFF + kk * 2048, 16384, 1024);
+          mma_ss(tbase + C::DQ_COL, da, db, C::IDESC_DQ, kk > 0 ? 1u : 0u);
+        }
+      };
+      auto q_off = [&](int s) -> uint32_t { return C::Q_OFF + (s % C::NSTAGE) * C::Q_BYTES; };
+      auto do_off = [&](int s) -> uint32_t { return C::DO_OFF + (s % C::NSTAGE) * C::Q_BYTES; };
+
+      if (ok) {
+        for (int k = 0; k < C::LA && k < n && ok; ++k) {
+          ok = wait_q(k);
+          if (!ok) break;
+          issue_xt(C::K_OFF, q_off(k), C::ST_COL + 64 * (k & 1));
+          tc_commit(BAR(C::B_SFULL + (k & 1)));
+        }
+        if (ok) {
+          issue_xt(C::V_OFF, do_off(0), C::DP_COL);
+          tc_commit(BAR(C::B_DPFULL));
+        }
+        for (int s = 0; s < n && ok; ++s) {
+          if (!mbar_wait(BAR(C::B_PFULL + (s & 1)), (s >> 1) & 1, wc, 14)) { ok = false; break; }
+          tc_fence_after();
+          issue_acc(C::ST_COL + 64 * (s & 1), do_off(s), C::DV_COL, s == 0);
+          if (!mbar_wait(BAR(C::B_DSFULL), s & 1, wc, 15)) { ok = false; break; }
+          tc_fence_after();
+          issue_acc(C::DP_COL, q_off(s), C::DK_COL, s == 0);
+          tc_commit(BAR(C::B_QEMPTY + s % C::NSTAGE));
+          if (s > 0) {
+            if (!mbar_wait(BAR(C::B_DQEMPTY), (s - 1) & 1, wc, 16)) { ok = false; break; }
+            tc_fence_after();
+          }
+          issue_dq();
+          tc_commit(BAR(C::B_DQFULL));
+          if (s + C::LA < n) {
+            const int s2 = s + C::LA;
+            if (!wait_q(s2)) { ok = false; break; }
+            issue_xt(C::K_OFF, q_off(s2), C::ST_COL + 64 * (s2 & 1));
+            tc_commit(BAR(C::B_SFULL + (s2 & 1)));
+          }
+          if (s + 1 < n) {
+            issue_xt(C::V_OFF, do_off(s + 1), C::DP_COL);
+            tc_commit(BAR(C::B_DPFULL));
+          }
+        }
+        if (ok) tc_commit(BAR(C::B_ACC));
+      }
+      tc_commit(BAR(C::B_DRAIN));
+      mbar_wait(BAR(C::B_DRAIN), 0, wc, 17);
+    }
+  } else if (warp >= 4 && warp < 8) {
+    // ------------------------------------------- compute: Pᵀ and dSᵀ rows
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // key row within the tile
+    const int key = jt * C::BC + r;
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+    const float sl2 = p.scale_log2;
+    bool ok = true;
+    for (int s = 0; s < n; ++s) {
+      const int st = s % C::NSTAGE;
+      const int q0 = step_q0(s);
+      if (!mbar_wait_warp(BAR(C::B_QFULL + st), (s / C::NSTAGE) & 1, wc, 21)) { ok = false; break; }
+      if (!mbar_wait_warp(BAR(C::B_SFULL + (s & 1)), (s >> 1) & 1, wc, 22)) { ok = false; break; }
+      tc_fence_after();
+      const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512);
+      const float* dv = lse2 + 64;
+      uint32_t x0[32], x1[32];
+      const int scol = C::ST_COL + 64 * (s & 1);
+      tmem_ld32(tl + scol, x0);
+      tmem_ld32(tl + scol + 32, x1);
+      tmem_ld_wait();
+      reg_fence(x0);
+      reg_fence(x1);
+      float pr[64];
+      const bool diag = CAUSAL && (q0 < jt * C::BC + C::BC);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        pr[c] = ex2(fmaf(__uint_as_float(x0[c]), sl2, -lse2[c]));
+        pr[32 + c] = ex2(fmaf(__uint_as_float(x1[c]), sl2, -lse2[32 + c]));
+      }
+      if (diag) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (key > q0 + c) pr[c] = 0.f;
+      }
+      uint32_t pk[32];
+#pragma unroll
+      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+      tmem_st32(tl + scol, pk);
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_PFULL + (s & 1)));
+
+      if (!mbar_wait_warp(BAR(C::B_DPFULL), s & 1, wc, 23)) { ok = false; break; }
+      tc_fence_after();
+      tmem_ld32(tl + C::DP_COL, x0);
+      tmem_ld32(tl + C::DP_COL + 32, x1);
+      tmem_ld_wait();
+      reg_fence(x0);
+      reg_fence(x1);
+#pragma unroll
+      for (int c = 0; c < 32; ++c) {
+        const float d0 = pr[2 * c] * (__uint_as_float(c < 16 ? x0[2 * c] : x1[2 * c - 32]) - dv[2 * c]);
+        const float d1 = pr[2 * c + 1] * (__uint_as_float(c < 16 ? x0[2 * c + 1] : x1[2 * c + 1 - 32]) - dv[2 * c + 1]);
+        pk[c] = pack_bf16(d0, d1);
+      }
+      tmem_st32(tl + C::DP_COL, pk);
+      // the previous dQᵀ product must be done reading the dSᵀ tile in smem
+      if (s > 0 && !mbar_wait_warp(BAR(C::B_DQFULL), (s - 1) & 1, wc, 24)) { ok = false; break; }
+      {
+        uint8_t* rowp = smem + C::DS_OFF + r * 128;
+#pragma unroll
+        for (int ch = 0; ch < 8; ++ch) {
+          uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) * 16)) = v;
+        }
+      }
+      fence_proxy_async_smem();
+      tmem_st_wait();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DSFULL));
+    }
+    // dK epilogue (scaled by s)
+    if (ok && mbar_wait_warp(BAR(C::B_ACC), 0, wc, 25)) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dk + ((size_t)(b * p.Hkv + hkv) * p.N + key) * D + dh * C::DH;
+#pragma unroll
+      for (int oc = 0; oc < C::DH / 32; ++oc) {
+        uint32_t v[32];
+        tmem_ld32(tl + C::DK_COL + oc * 32, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c)
+          w[c] = pack_bf16(__uint_as_float(v[2 * c]) * p.scale, __uint_as_float(v[2 * c + 1]) * p.scale);
+        uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      }
+    }
+    tc_fence_before();
+  } else if (warp >= 8) {
+    // ------------------------------------------ drain: dQᵀ rows -> global
+    const int quarter = warp & 3;
+    const int r = quarter * 32 + lane;  // d row of dQᵀ, key row of dV
+    const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+    bool ok = true;
+    for (int s = 0; s < n; ++s) {
+      if (!mbar_wait_warp(BAR(C::B_DQFULL), s & 1, wc, 31)) { ok = false; break; }
+      tc_fence_after();
+      uint32_t x0[32], x1[32];
+      tmem_ld32(tl + C::DQ_COL, x0);
+      tmem_ld32(tl + C::DQ_COL + 32, x1);
+      tmem_ld_wait();
+      reg_fence(x0);
+      reg_fence(x1);
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(BAR(C::B_DQEMPTY));
+      if (r < C::DH) {
+        float* base = p.dqacc + ((size_t)(b * p.Hq + step_head(s)) * p.N + step_q0(s)) * D + dh * C::DH + r;
+#pragma unroll
+        for (int c = 0; c < 32; ++c) red_add_f32(base + (size_t)c * D, __uint_as_float(x0[c]));
+#pragma unroll
+        for (int c = 0; c < 32; ++c) red_add_f32(base + (size_t)(32 + c) * D, __uint_as_float(x1[c]));
+      }
+    }
+    // dV epilogue
+    if (ok && mbar_wait_warp(BAR(C::B_ACC), 0, wc, 32)) {
+      tc_fence_after();
+      __nv_bfloat16* dst = p.dv + ((size_t)(b * p.Hkv + hkv) * p.N + jt * C::BC + r) * D + dh * C::DH;
+#pragma unroll
+      for (int oc = 0; oc < C::DH / 32; ++oc) {
+        uint32_t v[32];
+        tmem_ld32(tl + C::DV_COL + oc * 32, v);
+        tmem_ld_wait();
+        reg_fence(v);
+        uint32_t w[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) w[c] = pack_bf16(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
+        uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
+#pragma unroll
+        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+      }
+    }
+    tc_fence_before();
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,457 @@
+// Fused exact-attention forward pass for sm_100a.
+//
+// Computes O = softmax(s·Q Kᵀ [+ causal mask]) V and the per-row log-sum-exp,
+// keeping the score and probability tiles on chip (TMEM / registers) as the
+// FlashAttention pages describe: "深度学习进阶（三十一）FlashAttention：IO 感知的精确
+// 注意力" §2.2 (fix a Q block, stream every K/V block, update the per-row running
+// max m, normaliser d and output O after each block) and the "Flash-Attention"
+// concept page, "Core idea" (tile into on-chip memory, write only O and a few
+// per-row statistics).
+//
+// One CTA owns NQ query tiles of 128 rows of one (batch, head):
+//   warp 0        TMA producer: Q tiles once, then K/V chunks through a ring
+//   warp 1        MMA issuer (one thread) + TMEM owner
+//   warps 4..     one softmax warpgroup per query tile; thread = query row
+// S = Q Kᵀ and O += P V both run on tcgen05 with fp32 accumulators in TMEM.
+// P (bf16) is written back over the first half of its S columns and read by
+// the PV MMA directly from TMEM.  The O rescale is conditional: a row keeps a
+// stale reference max until the true max exceeds it by more than kRescaleTau
+// (log2 units); l and O share that reference, so the result is unchanged.
+#pragma once
+
+#include "sm100.cuh"
+
+namespace fa {
+
+constexpr float kRescaleTau = 8.0f;
+
+template <int D>
+struct FwdCfg {
+  static constexpr int BM = 128;                 // query rows per tile (MMA M)
+  static constexpr int BN = 128;                 // keys per K/V tile (MMA N of QKᵀ)
+  static constexpr int NQ = (D <= 128) ? 2 : 1;  // query tiles per CTA
+  static constexpr int THREADS = 128 + 128 * NQ;
+  static constexpr int CH = D < 128 ? D : 128;   // K/V chunk width in columns
+  static constexpr int NCH = D / CH;             // chunks per K or V tile
+  static constexpr int PANEL = 128 * 128;        // one 64-column panel of a 128-row tile (bytes)
+  static constexpr int Q_BYTES = BM * D * 2;
+  static constexpr int SLOT_BYTES = BN * CH * 2;
+  static constexpr int NSLOT = (D == 64) ? 8 : 4;
+  static constexpr int Q_OFF = 0;
+  static constexpr int KV_OFF = NQ * Q_BYTES;
+  static constexpr int BAR_OFF = KV_OFF + NSLOT * SLOT_BYTES;
+  // barrier indices
+  static constexpr int B_QFULL = 0;
+  static constexpr int B_KVFULL = 1;                 // + slot
+  static constexpr int B_KVEMPTY = 1 + NSLOT;        // + slot
+  static constexpr int B_SFULL = 1 + 2 * NSLOT;      // + {0,1}
+  static constexpr int B_PFULL = B_SFULL + 2;        // + {0,1}
+  static constexpr int B_ODONE = B_PFULL + 2;        // + {0,1}
+  static constexpr int B_DRAIN = B_ODONE + 2;
+  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
+  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;  // + slack to align the base to 1024
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int S_COL = 0;    // S buffer x at S_COL + 128*x
+  static constexpr int O_COL = 256;  // O of query tile t at O_COL + t*D
+  static constexpr uint32_t IDESC_S = idesc_bf16_f32(128, BN, false, false);
+  static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, CH, false, true);
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
+};
+
+struct FwdParams {
+  __nv_bfloat16* o;
+  float* lse;
+  int N, Hq, Hkv, G, n_qtiles;
+  float scale_log2;
+  long long wait_cap;
+  int* err;
+};
+
+// Load-order of K/V tiles ("units"; each unit is NCH chunks).  With two query
+// tiles the MMA warp first uses K(j) then V(j); with one query tile it keeps
+// two S tiles in flight and first uses K(0), K(1), V(0), K(2), V(1), ...
+template <int NQ>
+struct KVOrder {
+  __device__ static int unitK(int j, int n) {
+    if (NQ == 2) return 2 * j;
+    return j == 0 ? 0 : 2 * j - 1;
+  }
+  __device__ static int unitV(int j, int n) {
+    if (NQ == 2) return 2 * j + 1;
+    return (j == n - 1) ? 2 * n - 1 : 2 * j + 2;
+  }
+  // inverse: unit u -> (is_v, j)
+  __device__ static void decode(int u, int n, bool& is_v, int& j) {
+    if (NQ == 2) {
+      is_v = (u & 1);
+      j = u >> 1;
+      return;
+    }
+    if (u == 0) { is_v = false; j = 0; }
+    else if (u == 2 * n - 1) { is_v = true; j = n - 1; }
+    else if (u & 1) { is_v = false; j = (u + 1) >> 1; }
+    else { is_v = true; j = (u >> 1) - 1; }
+  }
+};
+
+template <int D, bool CAUSAL>
+__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+    fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
+  using C = FwdCfg<D>;
+  using Ord = KVOrder<C::NQ>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8 * i; };
+  uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+  const int h = blockIdx.y;
+  const int b = blockIdx.z;
+  const int hkv = h / p.G;
+  // causal: heaviest query tiles first so the tail of the grid is short
+  const int unit = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int qt0 = unit * C::NQ;
+  int n_t[2] = {0, 0};
+#pragma unroll
+  for (int t = 0; t < C::NQ; ++t) {
+    const int qt = qt0 + t;
+    n_t[t] = (qt < p.n_qtiles) ? (CAUSAL ? qt + 1 : p.n_qtiles) : 0;
+  }
+  const int nmax = n_t[0] > n_t[1] ? n_t[0] : n_t[1];
+
+  if (threadIdx.x == 0) {
+    mbar_init(BAR(C::B_QFULL), 1);
+    for (int i = 0; i < C::NSLOT; ++i) {
+      mbar_init(BAR(C::B_KVFULL + i), 1);
+      mbar_init(BAR(C::B_KVEMPTY + i), 1);
+    }
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(C::B_SFULL + i), 1);
+      mbar_init(BAR(C::B_PFULL + i), 4);
+      mbar_init(BAR(C::B_ODONE + i), 1);
+    }
+    mbar_init(BAR(C::B_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 1) {
+    tmem_alloc(smem_u32(tmem_holder), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tbase = *tmem_holder;
+  const WaitCtx wc{abort_flag, p.err, p.wait_cap};
+
+  if (warp == 0) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      const uint64_t pol_kv = policy_evict_last();
+      const uint64_t pol_q = policy_evict_first();
+      const int q_row_base = (b * p.Hq + h) * p.N;
+      const int kv_row_base = (b * p.Hkv + hkv) * p.N;
+      int nvalid = 0;
+#pragma unroll
+      for (int t = 0; t < C::NQ; ++t) nvalid += (n_t[t] > 0);
+      mbar_expect_tx(BAR(C::B_QFULL), nvalid * C::Q_BYTES);
+#pragma unroll
+      for (int t = 0; t < C::NQ; ++t) {
+        if (n_t[t] == 0) continue;
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn)
+          tma_load_2d_hint(sbase + C::Q_OFF + t * C::Q_BYTES + pn * C::PANEL, &tmQ, BAR(C::B_QFULL), pn * 64,
+                           q_row_base + (qt0 + t) * C::BM, pol_q);
+      }
+      bool ok = true;
+      for (int u = 0; u < 2 * nmax && ok; ++u) {
+        bool is_v;
+        int j;
+        Ord::decode(u, nmax, is_v, j);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int seq = u * C::NCH + c;
+          const int slot = seq % C::NSLOT;
+          const int round = seq / C::NSLOT;
+          if (!mbar_wait(BAR(C::B_KVEMPTY + slot), (round & 1) ^ 1, wc, 1)) { ok = false; break; }
+          mbar_expect_tx(BAR(C::B_KVFULL + slot), C::SLOT_BYTES);
+#pragma unroll
+          for (int pp = 0; pp < C::CH / 64; ++pp)
+            tma_load_2d_hint(sbase + C::KV_OFF + slot * C::SLOT_BYTES + pp * C::PANEL, is_v ? &tmV : &tmK,
+                             BAR(C::B_KVFULL + slot), c * C::CH + pp * 64, kv_row_base + j * C::BN, pol_kv);
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ---------------------------------------------------------- MMA issuer
+    if (lane == 0) {
+      bool ok = mbar_wait(BAR(C::B_QFULL), 0, wc, 2);
+      tc_fence_after();
+      int k_ready = -1, v_ready = -1;
+      auto wait_unit = [&](int u) -> bool {
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int seq = u * C::NCH + c;
+          if (!mbar_wait(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 3)) return false;
+        }
+        tc_fence_after();
+        return true;
+      };
+      auto release_unit = [&](int u) {
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) tc_commit(BAR(C::B_KVEMPTY + (u * C::NCH + c) % C::NSLOT));
+      };
+      auto need_k = [&](int j) -> bool {
+        if (j <= k_ready) return true;
+        k_ready = j;
+        return wait_unit(Ord::unitK(j, nmax));
+      };
+      auto need_v = [&](int j) -> bool {
+        if (j <= v_ready) return true;
+        v_ready = j;
+        return wait_unit(Ord::unitV(j, nmax));
+      };
+      // S[scol] = Q_t · K_jᵀ   (M=128 queries, N=128 keys, K=D)
+      auto issue_s = [&](int t, int j, int scol) {
+        const int uk = Ord::unitK(j, nmax);
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int koff = (kk & 3) * 32;
+          const uint64_t da = sdesc_sw128(sbase + C::Q_OFF + t * C::Q_BYTES + (kk >> 2) * C::PANEL + koff, 16, 1024);
+          const int col = kk * 16;
+          const int seq = uk * C::NCH + col / C::CH;
+          const int slot = seq % C::NSLOT;
+          const uint64_t db = sdesc_sw128(
+              sbase + C::KV_OFF + slot * C::SLOT_BYTES + ((col % C::CH) / 64) * C::PANEL + koff, 16, 1024);
+          mma_ss(tbase + scol, da, db, C::IDESC_S, kk > 0 ? 1u : 0u);
+        }
+      };
+      // O_t[:, c*CH..] (+)= P(TMEM at scol) · V_j[:, c*CH..]   (K = 128 keys)
+      auto issue_pv = [&](int j, int scol, int ocol) {
+        const int uv = Ord::unitV(j, nmax);
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const int slot = (uv * C::NCH + c) % C::NSLOT;
+#pragma unroll
+          for (int kk = 0; kk < C::BN / 16; ++kk) {
+            const uint64_t db = sdesc_sw128(sbase + C::KV_OFF + slot * C::SLOT_BYTES + kk * 2048, C::PANEL, 1024);
+            mma_ts(tbase + ocol + c * C::CH, tbase + scol + kk * 8, db, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
+          }
+        }
+      };
+
+      if (ok) {
+        if (C::NQ == 2) {
+          for (int t = 0; t < 2 && ok; ++t) {
+            if (n_t[t] == 0) continue;
+            ok = need_k(0);
+            if (!ok) break;
+            issue_s(t, 0, C::S_COL + 128 * t);
+            tc_commit(BAR(C::B_SFULL + t));
+          }
+          if (ok) release_unit(Ord::unitK(0, nmax));
+          for (int j = 0; j < nmax && ok; ++j) {
+            for (int t = 0; t < 2; ++t) {
+              if (j >= n_t[t]) continue;
+              if (!mbar_wait(BAR(C::B_PFULL + t), j & 1, wc, 4)) { ok = false; break; }
+              tc_fence_after();
+              if (!need_v(j)) { ok = false; break; }
+              issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D);
+              tc_commit(BAR(C::B_ODONE + t));
+              if (j + 1 < n_t[t]) {
+                if (!need_k(j + 1)) { ok = false; break; }
+                issue_s(t, j + 1, C::S_COL + 128 * t);
+                tc_commit(BAR(C::B_SFULL + t));
+              }
+            }
+            if (!ok) break;
+            release_unit(Ord::unitV(j, nmax));
+            if (j + 1 < nmax) release_unit(Ord::unitK(j + 1, nmax));
+          }
+        } else {
+          const int n = n_t[0];
+          ok = need_k(0);
+          if (ok) {
+            issue_s(0, 0, C::S_COL);
+            tc_commit(BAR(C::B_SFULL + 0));
+            release_unit(Ord::unitK(0, n));
+          }
+          if (ok && n > 1) {
+            ok = need_k(1);
+            if (ok) {
+              issue_s(0, 1, C::S_COL + 128);
+              tc_commit(BAR(C::B_SFULL + 1));
+              release_unit(Ord::unitK(1, n));
+            }
+          }
+          for (int j = 0; j < n && ok; ++j) {
+            const int x = j & 1;
+            if (!mbar_wait(BAR(C::B_PFULL + x), (j >> 1) & 1, wc, 4)) { ok = false; break; }
+            tc_fence_after();
+            if (!need_v(j)) { ok = false; break; }
+            issue_pv(j, C::S_COL + 128 * x, C::O_COL);
+            tc_commit(BAR(C::B_ODONE + x));
+            release_unit(Ord::unitV(j, n));
+            if (j + 2 < n) {
+              if (!need_k(j + 2)) { ok = false; break; }
+              issue_s(0, j + 2, C::S_COL + 128 * x);
+              tc_commit(BAR(C::B_SFULL + x));
+              release_unit(Ord::unitK(j + 2, n));
+            }
+          }
+        }
+      }
+      // no MMA may still be running when TMEM is released
+      tc_commit(BAR(C::B_DRAIN));
+      mbar_wait(BAR(C::B_DRAIN), 0, wc, 8);
+    }
+  } else if (warp >= 4) {
+    // ------------------------------------------------------------- softmax
+    const int t = (warp - 4) >> 2;
+    const int quarter = warp & 3;
+    const int row = quarter * 32 + lane;
+    const int n = n_t[t];
+    if (n > 0) {
+      const int qt = qt0 + t;
+      const int q_row = qt * C::BM + row;
+      const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+      const float sl2 = p.scale_log2;
+      const int ocol = C::O_COL + t * D;
+      float m_ref = -INFINITY;
+      float l = 0.f;
+      bool ok = true;
+      // Completion of PV(j) is signalled on o_done[t] (two query tiles: PV(t, j+1)
+      // cannot start before this warpgroup has seen S(t, j+1), which follows
+      // PV(t, j)) or on o_done[j & 1] (one query tile: S(j+1) is issued before
+      // PV(j), so one barrier could run two phases ahead of a waiter and make
+      // its parity test ambiguous).
+      auto odone_idx = [&](int jj) { return C::NQ == 2 ? t : (jj & 1); };
+      auto odone_par = [&](int jj) -> uint32_t { return C::NQ == 2 ? (jj & 1) : ((jj >> 1) & 1); };
+      for (int j = 0; j < n; ++j) {
+        const int x = (C::NQ == 2) ? t : (j & 1);
+        const uint32_t par = (C::NQ == 2) ? (j & 1) : ((j >> 1) & 1);
+        const int scol = C::S_COL + 128 * x;
+        if (!mbar_wait_warp(BAR(C::B_SFULL + x), par, wc, 5)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t r0[32], r1[32], r2[32], r3[32];
+        tmem_ld32(tl + scol + 0, r0);
+        tmem_ld32(tl + scol + 32, r1);
+        tmem_ld32(tl + scol + 64, r2);
+        tmem_ld32(tl + scol + 96, r3);
+        tmem_ld_wait();
+        reg_fence(r0);
+        reg_fence(r1);
+        reg_fence(r2);
+        reg_fence(r3);
+        float s[128];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          s[c] = __uint_as_float(r0[c]);
+          s[32 + c] = __uint_as_float(r1[c]);
+          s[64 + c] = __uint_as_float(r2[c]);
+          s[96 + c] = __uint_as_float(r3[c]);
+        }
+        if (CAUSAL && j == qt) {
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c > row) s[c] = -INFINITY;
+        }
+        float mx = s[0];
+#pragma unroll
+        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        const float m_new = fmaxf(m_ref, mx * sl2);
+        if (j == 0) {
+          m_ref = m_new;
+        } else {
+          const bool need = m_new > m_ref + kRescaleTau;
+          if (__any_sync(0xffffffffu, need)) {
+            const float alpha = need ? ex2(m_ref - m_new) : 1.f;
+            if (need) m_ref = m_new;
+            l *= alpha;
+            // O must hold the previous block's product before it is scaled
+            if (!mbar_wait_warp(BAR(C::B_ODONE + odone_idx(j - 1)), odone_par(j - 1), wc, 6)) { ok = false; break; }
+            tc_fence_after();
+#pragma unroll
+            for (int oc = 0; oc < D / 32; ++oc) {
+              uint32_t ov[32];
+              tmem_ld32(tl + ocol + oc * 32, ov);
+              tmem_ld_wait();
+              reg_fence(ov);
+#pragma unroll
+              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+              tmem_st32(tl + ocol + oc * 32, ov);
+            }
+            tmem_st_wait();
+          }
+        }
+        const float neg_m = -m_ref;
+        float rs0 = 0.f, rs1 = 0.f;
+        uint32_t pk0[32], pk1[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float a0 = ex2(fmaf(s[2 * c], sl2, neg_m));
+          const float a1 = ex2(fmaf(s[2 * c + 1], sl2, neg_m));
+          rs0 += a0;
+          rs1 += a1;
+          pk0[c] = pack_bf16(a0, a1);
+        }
+#pragma unroll
+        for (int c = 0; c < 32; ++c) {
+          const float a0 = ex2(fmaf(s[64 + 2 * c], sl2, neg_m));
+          const float a1 = ex2(fmaf(s[64 + 2 * c + 1], sl2, neg_m));
+          rs0 += a0;
+          rs1 += a1;
+          pk1[c] = pack_bf16(a0, a1);
+        }
+        l += rs0 + rs1;
+        tmem_st32(tl + scol + 0, pk0);
+        tmem_st32(tl + scol + 32, pk1);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_PFULL + x));
+      }
+      if (ok) ok = mbar_wait_warp(BAR(C::B_ODONE + odone_idx(n - 1)), odone_par(n - 1), wc, 7);
+      if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l;
+        __nv_bfloat16* orow = p.o + ((size_t)(b * p.Hq + h) * p.N + q_row) * D;
+#pragma unroll
+        for (int oc = 0; oc < D / 32; ++oc) {
+          uint32_t ov[32];
+          tmem_ld32(tl + ocol + oc * 32, ov);
+          tmem_ld_wait();
+          reg_fence(ov);
+          uint32_t w[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c)
+            w[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
+          uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
+#pragma unroll
+          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        }
+        float lg;
+        asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
+        p.lse[(size_t)(b * p.Hq + h) * p.N + q_row] = (m_ref + lg) * kLn2;
+      }
+      tc_fence_before();
+    }
+  }
+
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tbase, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

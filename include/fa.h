@@ -1,0 +1,110 @@
+/*
+ * fa.h — C ABI of libfa_b200.so: exact scaled-dot-product attention
+ * (forward and backward) for NVIDIA B200 (sm_100a).
+ *
+ * What it computes.  For every batch b and query head h, with key/value head
+ * g = h / (Hq / Hkv) (grouped-query attention; contiguous groups):
+ *
+ *     S   = scale · Q[b,h] · K[b,g]ᵀ            (N × N, never stored)
+ *     S_ij = -inf  where causal and j > i
+ *     P   = softmax(S) row-wise                  (never stored)
+ *     O[b,h]   = P · V[b,g]
+ *     LSE[b,h,i] = log Σ_j exp(S_ij)             (natural log)
+ *
+ * The standard definition is on the page "FlashAttention" (LLM inference
+ * handbook, kernel-optimization chapter), section "attention 为什么一开始就很慢";
+ * the tiled online-softmax evaluation that keeps S and P on chip is section
+ * 2.2 of "深度学习进阶（三十一）FlashAttention：IO 感知的精确注意力"; the backward
+ * pass recomputes P from Q, K and the saved LSE ("Flash-Attention" concept
+ * page, "Core idea") and returns the chain-rule gradients dQ, dK, dV.
+ *
+ * Layouts (all row-major, contiguous, 16-byte aligned device pointers):
+ *   q, o, dout, dq : bf16 [B, Hq,  N, d]
+ *   k, v, dk, dv   : bf16 [B, Hkv, N, d]
+ *   lse            : fp32 [B, Hq,  N]
+ *
+ * Ownership.  The caller allocates every buffer (device memory) and keeps it
+ * alive until the work on `stream` has finished.  The library allocates no
+ * memory.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * stream).  Every call only enqueues work and returns; errors found on the
+ * device are reported by fa_device_status().
+ *
+ * Errors.  Arguments are checked before anything is enqueued:
+ *   FA_ERR_INVALID_ARG  null or misaligned pointer, negative size, Hq not a
+ *                       multiple of Hkv, non-finite or non-positive scale,
+ *                       an output overlapping an input or another output,
+ *                       workspace too small;
+ *   FA_ERR_UNSUPPORTED  d not in {64, 128, 256}, N not a multiple of 128,
+ *                       sizes beyond the index limits (B, Hq ≤ 65535,
+ *                       B·Hq·N < 2^31), or no sm_100 device;
+ *   FA_ERR_CUDA         a CUDA launch or attribute call failed;
+ *   FA_ERR_TIMEOUT      (fa_device_status only) a kernel gave up a bounded
+ *                       wait and returned early; its outputs are invalid.
+ * A problem with B == 0 or N == 0 is empty: nothing is enqueued, FA_OK.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4
+} fa_status;
+
+/* Forward pass: writes O (bf16) and LSE (fp32, natural log).
+ * One fused kernel; S and P stay on chip.  `causal` != 0 masks keys after
+ * the query.  `scale` multiplies the scores before masking and softmax
+ * (usually 1/sqrt(d)). */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                 void* stream);
+
+/* Bytes of device workspace fa_bwd needs: two fp32 [B,Hq,N] row vectors
+ * (D = rowsum(dO∘O) and LSE·log2 e) and an fp32 [B,Hq,N,d] dQ accumulator,
+ * each rounded up to 256 bytes.  Returns 0 for invalid sizes. */
+size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
+
+/* Backward pass: given q, k, v, the forward outputs o and lse, and the output
+ * gradient dout, writes dq, dk, dv (bf16).  dk and dv are summed over the
+ * query heads that share a key/value head.  `workspace` (device, 256-byte
+ * aligned, at least fa_bwd_workspace_bytes) is scratch owned by the caller;
+ * its contents on entry do not matter.  Enqueues three kernels on `stream`. */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dout, void* dq, void* dk, void* dv,
+                 int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                 void* workspace, size_t workspace_bytes, void* stream);
+
+/* Synchronises `stream`, then reads and clears the current device's error
+ * word.  FA_ERR_TIMEOUT if a kernel abandoned a bounded wait since the last
+ * call, FA_ERR_CUDA if the stream reported a CUDA error, else FA_OK. */
+fa_status fa_device_status(void* stream);
+
+/* Static English description of a status code; never NULL. */
+const char* fa_status_string(fa_status s);
+
+/* Cycle budget (SM clock cycles) after which a kernel's wait on an on-chip
+ * barrier gives up, records FA_ERR_TIMEOUT and returns.  0 restores the
+ * default (2^31 cycles, about one second).  Affects later launches only. */
+fa_status fa_set_wait_cap(long long cycles);
+
+/* One-shot profiling hook for the calling host thread: the next fa_fwd or
+ * fa_bwd call records `start_event` on its stream immediately before its
+ * attention kernel (fa_fwd's fused kernel; fa_bwd's dK/dV/dQ kernel, after
+ * the preprocessing kernel) and `stop_event` immediately after it, then
+ * forgets both.  The events are cudaEvent_t handles owned by the caller;
+ * NULL for both cancels a pending request. */
+fa_status fa_profile_next(void* start_event, void* stop_event);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */

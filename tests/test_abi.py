@@ -1,0 +1,120 @@
+"""C-ABI checks that need no GPU: the library loads, exports every function
+``include/fa.h`` declares, and rejects invalid arguments before touching CUDA."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from exact_attention_104_b200 import binding
+from exact_attention_104_b200.build import build
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "fa.h")
+
+
+@pytest.fixture(scope="module")
+def lib():
+    build()
+    return binding.lib()
+
+
+def _declared_functions():
+    src = open(HEADER).read()
+    src = re.sub(r"/\*.*?\*/", "", src, flags=re.S)
+    return sorted(set(re.findall(r"^\s*(?:[A-Za-z_][\w\s\*]*?)\b(fa_\w+)\s*\(", src, flags=re.M)))
+
+
+def test_header_declares_the_entry_points():
+    names = _declared_functions()
+    for required in ("fa_fwd", "fa_bwd", "fa_bwd_workspace_bytes", "fa_device_status", "fa_status_string"):
+        assert required in names
+
+
+def test_library_exports_every_declared_symbol(lib):
+    for name in _declared_functions():
+        assert hasattr(lib, name), name
+        assert ctypes.cast(getattr(lib, name), ctypes.c_void_p).value
+
+
+def test_status_strings(lib):
+    for code in range(5):
+        assert binding.fa_status_string(code)
+    assert binding.fa_status_string(99) == "unknown status"
+
+
+def test_workspace_bytes_formula(lib):
+    # two fp32 row vectors and an fp32 [B,Hq,N,d] accumulator, each 256-rounded
+    B, Hq, Hkv, N, d = 8, 16, 16, 2048, 128
+    rows = B * Hq * N
+    assert binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) == 2 * rows * 4 + rows * d * 4
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 128, 64) == 2 * 512 + 128 * 64 * 4
+    assert binding.fa_bwd_workspace_bytes(1, 3, 2, 128, 64) == 0      # Hq % Hkv != 0
+    assert binding.fa_bwd_workspace_bytes(1, 2, 2, 128, 96) == 0      # unsupported d
+
+
+FAKE = 1 << 20  # an aligned, non-null address; validation must reject before any use
+
+
+def _fwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5,
+             B=1, Hq=2, Hkv=2, N=128, d=64, causal=0, scale=0.125, stream=0)
+    a.update(kw)
+    return binding.fa_fwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["N"], a["d"],
+                          a["causal"], a["scale"], a["stream"])
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), binding.FA_ERR_INVALID_ARG),
+    (dict(lse=0), binding.FA_ERR_INVALID_ARG),
+    (dict(k=FAKE * 2 + 8), binding.FA_ERR_INVALID_ARG),          # misaligned
+    (dict(Hq=3, Hkv=2), binding.FA_ERR_INVALID_ARG),
+    (dict(Hq=0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=0.0), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=float("nan")), binding.FA_ERR_INVALID_ARG),
+    (dict(scale=float("inf")), binding.FA_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=0), binding.FA_ERR_INVALID_ARG),
+    (dict(N=200), binding.FA_ERR_UNSUPPORTED),                   # ragged tail
+    (dict(B=70000), binding.FA_ERR_UNSUPPORTED),
+    (dict(B=1024, Hq=1024, Hkv=1024, N=4096), binding.FA_ERR_UNSUPPORTED),
+    (dict(o=FAKE), binding.FA_ERR_INVALID_ARG),                  # output aliases q
+    (dict(lse=FAKE * 4 + 64), binding.FA_ERR_INVALID_ARG),       # lse overlaps o
+    (dict(B=0, q=0, k=0, v=0, o=0, lse=0), binding.FA_OK),       # empty problem: nothing to do
+    (dict(N=0), binding.FA_OK),
+])
+def test_fwd_argument_validation(lib, kw, expect):
+    assert _fwd(lib, **kw) == expect
+
+
+def _bwd(lib, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5, do=FAKE * 6, dq=FAKE * 7, dk=FAKE * 8,
+             dv=FAKE * 9, B=1, Hq=2, Hkv=2, N=128, d=64, causal=0, scale=0.125, ws=FAKE * 10, wsb=1 << 20)
+    a.update(kw)
+    return binding.fa_bwd(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"], a["dv"],
+                          a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["causal"], a["scale"], a["ws"], a["wsb"], 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(do=0), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=0), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=FAKE * 10 + 16), binding.FA_ERR_INVALID_ARG),       # workspace not 256-aligned
+    (dict(wsb=100), binding.FA_ERR_INVALID_ARG),                 # workspace too small
+    (dict(dq=FAKE), binding.FA_ERR_INVALID_ARG),                 # dq aliases q
+    (dict(dk=FAKE * 7), binding.FA_ERR_INVALID_ARG),             # dk aliases dq
+    (dict(ws=FAKE * 9), binding.FA_ERR_INVALID_ARG),             # workspace aliases dv
+    (dict(Hq=4, Hkv=3), binding.FA_ERR_INVALID_ARG),
+    (dict(d=32), binding.FA_ERR_UNSUPPORTED),
+    (dict(N=130), binding.FA_ERR_UNSUPPORTED),
+    (dict(B=0), binding.FA_OK),
+])
+def test_bwd_argument_validation(lib, kw, expect):
+    assert _bwd(lib, **kw) == expect
+
+
+def test_wait_cap_setter(lib):
+    assert lib.fa_set_wait_cap(-1) == binding.FA_ERR_INVALID_ARG
+    assert lib.fa_set_wait_cap(1 << 28) == binding.FA_OK
+    assert lib.fa_set_wait_cap(0) == binding.FA_OK

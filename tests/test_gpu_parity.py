@@ -1,0 +1,121 @@
+"""GPU parity: the CUDA path (through the C ABI) against the fp64 oracle on the
+same seeded bf16 inputs, element by element, at sizes the oracle finishes in
+seconds that still span several tiles.  Tolerances are the specification's
+(see tests/_parity.py)."""
+
+import math
+
+import numpy as np
+import pytest
+import torch
+
+from exact_attention_104_b200 import FAError, attention_backward, attention_forward, binding, lib
+from exact_attention_104_b200.workloads import WORKLOADS, Workload, make_inputs
+
+from _parity import assert_within_tolerance, compare_full, f64, run_gpu
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _short_waits():
+    # a broken pipeline reports FA_ERR_TIMEOUT quickly instead of after ~1 s
+    lib().fa_set_wait_cap(1 << 28)
+    yield
+    lib().fa_set_wait_cap(0)
+
+
+def test_tiny_config_fwd_bwd():
+    w = WORKLOADS["tiny_b1_h2_n128_d64"]
+    err = compare_full(w, run_gpu(w))
+    assert_within_tolerance(err)
+
+
+SMALL = []
+for d in (64, 128, 256):
+    for causal in (False, True):
+        for (B, Hq, Hkv, N) in ((1, 2, 2, 256), (2, 2, 1, 384), (1, 4, 2, 640)):
+            SMALL.append(Workload(f"s_d{d}_{'c' if causal else 'nc'}_{B}_{Hq}_{Hkv}_{N}", B, Hq, Hkv, N, d, causal,
+                                  1.0, 7 + d + N))
+
+
+@pytest.mark.parametrize("w", SMALL, ids=lambda w: w.name)
+def test_small_shapes_fwd_bwd(w):
+    err = compare_full(w, run_gpu(w))
+    assert_within_tolerance(err)
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+@pytest.mark.parametrize("causal", [False, True])
+def test_large_logits(d, causal):
+    # Q, K ~ N(0, 3²): peaked rows with frequent running-max changes
+    w = Workload(f"big_d{d}", 1, 2, 2, 512, d, causal, 3.0, 99 + d)
+    err = compare_full(w, run_gpu(w))
+    assert_within_tolerance(err)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_forward_is_bitwise_deterministic_and_dkdv_too(causal):
+    w = Workload("det", 2, 4, 2, 512, 128, causal, 1.0, 5)
+    q, k, v, do = make_inputs(w, "cuda")
+    o1, l1 = attention_forward(q, k, v, causal=causal)
+    o2, l2 = attention_forward(q, k, v, causal=causal)
+    assert torch.equal(o1, o2) and torch.equal(l1, l2)
+    g1 = attention_backward(q, k, v, o1, l1, do, causal=causal)
+    g2 = attention_backward(q, k, v, o1, l1, do, causal=causal)
+    assert torch.equal(g1[1], g2[1]) and torch.equal(g1[2], g2[2])
+    # dQ sums fp32 partials with atomics: order may vary, value within tolerance
+    assert (g1[0].float() - g2[0].float()).abs().max().item() <= 1e-2
+
+
+@pytest.mark.parametrize("d", [64, 128, 256])
+def test_constant_values_give_constant_output(d):
+    # rows of P sum to one, so V = 1 gives O = 1 for any Q, K
+    w = Workload("ones", 1, 2, 2, 384, d, True, 2.0, 3)
+    q, k, _, _ = make_inputs(w, "cuda")
+    v = torch.ones_like(k)
+    o, _ = attention_forward(q, k, v, causal=True)
+    assert (o.float() - 1).abs().max().item() <= 4e-3
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_zero_queries_give_uniform_attention(causal):
+    w = Workload("zq", 1, 2, 2, 256, 128, causal, 1.0, 4)
+    _, k, v, _ = make_inputs(w, "cuda")
+    q = torch.zeros(1, 2, 256, 128, dtype=torch.bfloat16, device="cuda")
+    o, lse = attention_forward(q, k, v, causal=causal)
+    vf = f64(v)
+    if causal:
+        ref = np.cumsum(vf, axis=2) / np.arange(1, 257)[None, None, :, None]
+        lse_ref = np.log(np.arange(1, 257))[None, None, :]
+    else:
+        ref = np.broadcast_to(vf.mean(axis=2, keepdims=True), vf.shape)
+        lse_ref = np.full((1, 2, 256), math.log(256))
+    assert np.abs(f64(o) - ref).max() <= 2e-2
+    assert np.abs(f64(lse) - lse_ref).max() <= 1e-5
+
+
+def test_unsupported_and_invalid_are_reported():
+    q = torch.zeros(1, 2, 200, 64, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(FAError) as e:
+        attention_forward(q, q.clone(), q.clone())
+    assert e.value.status == binding.FA_ERR_UNSUPPORTED
+    q = torch.zeros(1, 2, 128, 96, dtype=torch.bfloat16, device="cuda")
+    with pytest.raises(FAError) as e:
+        attention_forward(q, q.clone(), q.clone())
+    assert e.value.status == binding.FA_ERR_UNSUPPORTED
+    q = torch.zeros(1, 2, 128, 64, dtype=torch.bfloat16, device="cuda")
+    o = torch.empty_like(q)
+    lse = torch.empty(1, 2, 128, device="cuda")
+    # output aliasing an input is rejected
+    st = binding.fa_fwd(q, q.clone(), q.clone(), q, lse, 1, 2, 2, 128, 64, 0, 0.125)
+    assert st == binding.FA_ERR_INVALID_ARG
+    st = binding.fa_fwd(q, q.clone(), q.clone(), o, lse, 1, 2, 2, 128, 64, 0, 0.125)
+    assert st == binding.FA_OK
+    assert binding.fa_device_status() == binding.FA_OK
+
+
+def test_empty_problem_is_a_no_op():
+    q = torch.zeros(0, 2, 128, 64, dtype=torch.bfloat16, device="cuda")
+    o, lse = attention_forward(q, q, q)
+    assert o.numel() == 0 and lse.numel() == 0
