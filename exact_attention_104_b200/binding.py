@@ -50,6 +50,8 @@ def lib() -> ctypes.CDLL:
     L.fa_set_wait_cap.restype = i
     L.fa_profile_next.argtypes = [vp, vp]
     L.fa_profile_next.restype = i
+    L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.fa_bwd_noalloc.restype = i
     _lib = L
     return L
 
@@ -99,6 +101,18 @@ def fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, wor
     return lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                         B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _ptr(workspace),
                         int(workspace_bytes), _stream_handle(stream))
+
+
+FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024
+
+
+def fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, stream=None) -> int:
+    """Raw C-ABI call of the backward pass that uses the library's fixed
+    device scratch array instead of a caller workspace (for callers that
+    cannot allocate device memory).  Returns the status."""
+    return lib().fa_bwd_noalloc(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                                _ptr(dv), B, Hq, Hkv, N, d, int(bool(causal)), float(scale),
+                                _stream_handle(stream))
 
 
 def fa_profile_next(start_event=None, stop_event=None) -> int:

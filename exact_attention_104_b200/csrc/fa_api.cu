@@ -14,6 +14,11 @@
 // Device error word: kernels that abandon a bounded wait record it here.
 __device__ int g_fa_err = 0;
 
+// Scratch of fa_bwd_noalloc: a fixed device array instead of a caller buffer.
+// Host code must not pass this symbol to a kernel (on the host it names a
+// stand-in, not device memory); noalloc_scratch() resolves its device address.
+static __device__ __align__(256) unsigned char g_fa_noalloc_scratch[FA_NOALLOC_SCRATCH_BYTES];
+
 namespace {
 
 constexpr int kMaxDevices = 64;
@@ -176,6 +181,29 @@ fa_status launch_bwd_pre(const void* o, const void* dout, const float* lse, floa
       static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc, rows,
       dq_vec4);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// Device address of g_fa_noalloc_scratch on the current device, looked up
+// once per device (with that device current) and cached.
+fa_status noalloc_scratch(void** out) {
+  static void* addr[kMaxDevices] = {};
+  static std::mutex mu;
+  int dev = -1;
+  if (cudaGetDevice(&dev) != cudaSuccess || dev < 0 || dev >= kMaxDevices) {
+    cudaGetLastError();
+    return FA_ERR_UNSUPPORTED;
+  }
+  std::lock_guard<std::mutex> lk(mu);
+  if (addr[dev] == nullptr) {
+    void* p = nullptr;
+    if (cudaGetSymbolAddress(&p, g_fa_noalloc_scratch) != cudaSuccess || p == nullptr) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    addr[dev] = p;
+  }
+  *out = addr[dev];
+  return FA_OK;
 }
 
 }  // namespace
@@ -345,6 +373,21 @@ fa_status fa_device_status(void* stream) {
   if (host != 0 && cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return FA_ERR_CUDA;
   return host != 0 ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv, int B, int Hq, int Hkv, int N, int d,
+                         int causal, float scale, void* stream) {
+  bool empty = false;
+  fa_status st = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  const size_t need = fa_bwd_workspace_bytes(B, Hq, Hkv, N, d);
+  if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  void* scratch = nullptr;
+  st = noalloc_scratch(&scratch);
+  if (st != FA_OK) return st;
+  return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, scratch,
+                (size_t)FA_NOALLOC_SCRATCH_BYTES, stream);
 }
 
 }  // extern "C"

@@ -103,6 +103,40 @@ fa_status fa_set_wait_cap(long long cycles);
  * NULL for both cancels a pending request. */
 fa_status fa_profile_next(void* start_event, void* stop_event);
 
+/* Size in bytes of the fixed device scratch array used by fa_bwd_noalloc. */
+#define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
+
+/* Backward pass without caller-provided scratch.  (The FlashAttention pages
+ * have no counterpart to this entry point; it exists for callers, not for
+ * the method.)
+ *
+ * Same arguments, layouts and results as fa_bwd, minus the workspace.  It is
+ * meant for callers that cannot hand the library a device buffer: code that
+ * runs inside a host framework which owns all device memory and offers its
+ * plugins no allocator, or a latency-critical loop where calling cudaMalloc
+ * (which can synchronise the whole device) is not acceptable.  Instead of a
+ * workspace it uses one file-scope device array of FA_NOALLOC_SCRATCH_BYTES
+ * (64 MiB), which every GPU that loads the library holds until the process
+ * exits.  Nothing is allocated or freed per call.
+ *
+ * Limit: the problem's fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) must not
+ * exceed FA_NOALLOC_SCRATCH_BYTES (for d = 128 that is B·Hq·N ≤ 129,055
+ * query rows); larger problems return FA_ERR_UNSUPPORTED and enqueue nothing.
+ *
+ * Set-up: the first call on each device, with that device current, looks up
+ * the array's device address (cudaGetSymbolAddress).  Make that first call
+ * before any stream capture on that device.
+ *
+ * Sharing: all calls on a device use the same array, and it keeps whatever
+ * the last call left in it (the dQ accumulator is zeroed by every call before
+ * use).  Two calls whose work overlaps on the GPU — different streams, or
+ * different host threads without ordering — race on the array and give wrong
+ * results; order them on one stream or with events. */
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dout, void* dq, void* dk, void* dv,
+                         int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                         void* stream);
+
 #ifdef __cplusplus
 }
 #endif
