@@ -71,6 +71,20 @@ bool make_map(CUtensorMap* m, const void* ptr, uint64_t rows, int d, int box_row
              CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
 }
 
+// 2-D view [rows, d] of an fp32 tensor, unswizzled boxes of box_cols x box_rows
+// (used as the destination of TMA reduce-adds).
+bool make_map_f32(CUtensorMap* m, const void* ptr, uint64_t rows, int d, int box_cols, int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return false;
+  cuuint64_t dims[2] = {(cuuint64_t)d, (cuuint64_t)rows};
+  cuuint64_t strides[1] = {(cuuint64_t)d * 4};
+  cuuint32_t box[2] = {(cuuint32_t)box_cols, (cuuint32_t)box_rows};
+  cuuint32_t estr[2] = {1, 1};
+  return enc(m, CU_TENSOR_MAP_DATA_TYPE_FLOAT32, 2, const_cast<void*>(ptr), dims, strides, box, estr,
+             CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_NONE, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+             CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE) == CUDA_SUCCESS;
+}
+
 struct DeviceInfo {
   bool checked = false;
   bool sm100 = false;
@@ -159,11 +173,13 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
   using C = fa::BwdCfg<D>;
   auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  CUtensorMap tdq;
+  if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.N, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
   dim3 grid((p.N / C::BC) * C::NDH, Hkv, B);
   ProfileScope prof(stream);
-  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, p);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

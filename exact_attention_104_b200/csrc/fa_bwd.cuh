@@ -49,7 +49,11 @@ struct BwdCfg {
   static constexpr int Q_OFF = DS_OFF + 16384;
   static constexpr int DO_OFF = Q_OFF + NSTAGE * Q_BYTES;
   static constexpr int LS_OFF = DO_OFF + NSTAGE * Q_BYTES;  // per stage: lse2[64], Dvec[64]
-  static constexpr int BAR_OFF = LS_OFF + NSTAGE * 512;
+  // dQᵀ staging for the TMA reduce-add: STG_ROWS query rows x DH fp32, row-major
+  static constexpr int STG_ROWS = (D == 256) ? 32 : 64;
+  static constexpr int STG_OFF = LS_OFF + NSTAGE * 512 + ((1024 - (NSTAGE * 512) % 1024) % 1024);
+  static constexpr int STG_BYTES = STG_ROWS * DH * 4;
+  static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
   static constexpr int B_KVFULL = 0;
   static constexpr int B_QFULL = 1;                  // + stage
   static constexpr int B_QEMPTY = 1 + NSTAGE;        // + stage
@@ -59,7 +63,9 @@ struct BwdCfg {
   static constexpr int B_DSFULL = B_PFULL + 2;
   static constexpr int B_DQFULL = B_DSFULL + 1;
   static constexpr int B_DQEMPTY = B_DQFULL + 1;
-  static constexpr int B_ACC = B_DQEMPTY + 1;
+  static constexpr int B_STGFREE = B_DQEMPTY + 1;  // staging may be overwritten
+  static constexpr int B_STGFULL = B_STGFREE + 1;  // staging written by all drain threads
+  static constexpr int B_ACC = B_STGFULL + 1;
   static constexpr int B_DRAIN = B_ACC + 1;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
@@ -151,7 +157,7 @@ template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
-                  const BwdParams p) {
+                  const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg<D>;
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
@@ -185,6 +191,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(BAR(C::B_DSFULL), 4);
     mbar_init(BAR(C::B_DQFULL), 1);
     mbar_init(BAR(C::B_DQEMPTY), 4);
+    mbar_init(BAR(C::B_STGFREE), 1);
+    mbar_init(BAR(C::B_STGFULL), 128);
     mbar_init(BAR(C::B_ACC), 1);
     mbar_init(BAR(C::B_DRAIN), 1);
     *abort_flag = 0;
@@ -299,15 +307,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
           issue_dq();
           tc_commit(BAR(C::B_DQFULL));
-          if (s + C::LA < n) {
-            const int s2 = s + C::LA;
-            if (!wait_q(s2)) { ok = false; break; }
-            issue_xt(C::K_OFF, q_off(s2), C::ST_COL + 64 * (s2 & 1));
-            tc_commit(BAR(C::B_SFULL + (s2 & 1)));
-          }
+          // dPᵀ of the next step first: the compute warps are waiting for it
           if (s + 1 < n) {
+            if (C::LA == 1 && !wait_q(s + 1)) { ok = false; break; }
             issue_xt(C::V_OFF, do_off(s + 1), C::DP_COL);
             tc_commit(BAR(C::B_DPFULL));
+          }
+          if (s + C::LA < n) {
+            const int s2 = s + C::LA;
+            if (C::LA > 1 && !wait_q(s2)) { ok = false; break; }
+            issue_xt(C::K_OFF, q_off(s2), C::ST_COL + 64 * (s2 & 1));
+            tc_commit(BAR(C::B_SFULL + (s2 & 1)));
           }
         }
         if (ok) tc_commit(BAR(C::B_ACC));
@@ -360,27 +370,31 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (lane == 0) mbar_arrive(BAR(C::B_PFULL + (s & 1)));
 
       if (!mbar_wait_warp(BAR(C::B_DPFULL), s & 1, wc, 23)) { ok = false; break; }
-      tc_fence_after();
-      tmem_ld32(tl + C::DP_COL, x0);
-      tmem_ld32(tl + C::DP_COL + 32, x1);
-      tmem_ld_wait();
-      reg_fence(x0);
-      reg_fence(x1);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        const float d0 = pr[2 * c] * (__uint_as_float(c < 16 ? x0[2 * c] : x1[2 * c - 32]) - dv[2 * c]);
-        const float d1 = pr[2 * c + 1] * (__uint_as_float(c < 16 ? x0[2 * c + 1] : x1[2 * c + 1 - 32]) - dv[2 * c + 1]);
-        pk[c] = pack_bf16(d0, d1);
-      }
-      tmem_st32(tl + C::DP_COL, pk);
       // the previous dQᵀ product must be done reading the dSᵀ tile in smem
       if (s > 0 && !mbar_wait_warp(BAR(C::B_DQFULL), (s - 1) & 1, wc, 24)) { ok = false; break; }
-      {
-        uint8_t* rowp = smem + C::DS_OFF + r * 128;
+      tc_fence_after();
+      uint8_t* rowp = smem + C::DS_OFF + r * 128;
+      // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: bf16 over the
+      // consumed dPᵀ columns (A operand of dK) and into the smem tile (dQᵀ)
 #pragma unroll
-        for (int ch = 0; ch < 8; ++ch) {
-          uint4 v = make_uint4(pk[4 * ch], pk[4 * ch + 1], pk[4 * ch + 2], pk[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(rowp + ((ch ^ (r & 7)) * 16)) = v;
+      for (int hf = 0; hf < 2; ++hf) {
+        tmem_ld32(tl + C::DP_COL + 32 * hf, x0);
+        tmem_ld_wait();
+        reg_fence(x0);
+        uint32_t dk16[16];
+#pragma unroll
+        for (int c = 0; c < 16; ++c) {
+          const int q = 32 * hf + 2 * c;
+          const float d0 = pr[q] * (__uint_as_float(x0[2 * c]) - dv[q]);
+          const float d1 = pr[q + 1] * (__uint_as_float(x0[2 * c + 1]) - dv[q + 1]);
+          dk16[c] = pack_bf16(d0, d1);
+        }
+        tmem_st16(tl + C::DP_COL + 16 * hf, dk16);
+#pragma unroll
+        for (int ch = 0; ch < 4; ++ch) {
+          const int lch = 4 * hf + ch;
+          const uint4 v = make_uint4(dk16[4 * ch], dk16[4 * ch + 1], dk16[4 * ch + 2], dk16[4 * ch + 3]);
+          *reinterpret_cast<uint4*>(rowp + ((lch ^ (r & 7)) * 16)) = v;
         }
       }
       fence_proxy_async_smem();
@@ -410,12 +424,16 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
     tc_fence_before();
   } else if (warp >= 8) {
-    // ------------------------------------------ drain: dQᵀ rows -> global
+    // ------------------------- drain: dQᵀ -> smem staging -> TMA reduce-add
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // d row of dQᵀ, key row of dV
+    const int dt = threadIdx.x - 256;   // 0..127 within the drain warpgroup
     const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
+    float* stg = reinterpret_cast<float*>(smem + C::STG_OFF);
+    if (dt == 0) tma_prefetch_desc(&tmDQ);
     bool ok = true;
-    for (int s = 0; s < n; ++s) {
+    int sub_seq = 0;  // staging uses so far
+    for (int s = 0; s < n && ok; ++s) {
       if (!mbar_wait_warp(BAR(C::B_DQFULL), s & 1, wc, 31)) { ok = false; break; }
       tc_fence_after();
       uint32_t x0[32], x1[32];
@@ -427,14 +445,33 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DQEMPTY));
-      if (r < C::DH) {
-        float* base = p.dqacc + ((size_t)(b * p.Hq + step_head(s)) * p.N + step_q0(s)) * D + dh * C::DH + r;
+      const int q_row = (b * p.Hq + step_head(s)) * p.N + step_q0(s);
 #pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(base + (size_t)c * D, __uint_as_float(x0[c]));
+      for (int sub = 0; sub < 64 / C::STG_ROWS; ++sub) {
+        // the previous reduce must have finished reading the staging tile
+        if (dt == 0) {
+          bulk_wait_read_all();
+          mbar_arrive(BAR(C::B_STGFREE));
+        }
+        if (!mbar_wait_warp(BAR(C::B_STGFREE), sub_seq & 1, wc, 33)) { ok = false; break; }
+        if (r < C::DH) {
 #pragma unroll
-        for (int c = 0; c < 32; ++c) red_add_f32(base + (size_t)(32 + c) * D, __uint_as_float(x1[c]));
+          for (int qq = 0; qq < C::STG_ROWS; ++qq) {
+            const int c = sub * C::STG_ROWS + qq;
+            stg[qq * C::DH + r] = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
+          }
+        }
+        fence_proxy_async_smem();
+        mbar_arrive(BAR(C::B_STGFULL));
+        if (dt == 0) {
+          if (!mbar_wait(BAR(C::B_STGFULL), sub_seq & 1, wc, 34)) { ok = false; break; }
+          tma_reduce_add_2d(&tmDQ, sbase + C::STG_OFF, dh * C::DH, q_row + sub * C::STG_ROWS);
+          bulk_commit_group();
+        }
+        ++sub_seq;
       }
     }
+    if (dt == 0) bulk_wait_all();
     // dV epilogue
     if (ok && mbar_wait_warp(BAR(C::B_ACC), 0, wc, 32)) {
       tc_fence_after();

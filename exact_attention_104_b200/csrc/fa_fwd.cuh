@@ -96,6 +96,20 @@ struct KVOrder {
   }
 };
 
+// Maximum of 128 values: eight independent chains of three-input max, then a
+// small tree (short dependency chains keep the issue slots busy).
+__device__ __forceinline__ float row_max128(const float (&s)[128]) {
+  float acc[8];
+#pragma unroll
+  for (int k = 0; k < 8; ++k) {
+    float a = fmaxf(s[16 * k], s[16 * k + 1]);
+#pragma unroll
+    for (int i = 2; i < 16; i += 2) a = fmax3(a, s[16 * k + i], s[16 * k + i + 1]);
+    acc[k] = a;
+  }
+  return fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7])));
+}
+
 template <int D, bool CAUSAL>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -365,56 +379,56 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int c = 0; c < 128; ++c)
             if (c > row) s[c] = -INFINITY;
         }
-        float mx = s[0];
-#pragma unroll
-        for (int c = 1; c < 128; ++c) mx = fmaxf(mx, s[c]);
+        const float mx = row_max128(s);
         const float m_new = fmaxf(m_ref, mx * sl2);
+        // conditional rescale: keep the stale reference max unless the row max
+        // grew by more than kRescaleTau; O itself is scaled after P is stored
+        float alpha = 1.f;
+        bool warp_rescale = false;
         if (j == 0) {
           m_ref = m_new;
         } else {
           const bool need = m_new > m_ref + kRescaleTau;
-          if (__any_sync(0xffffffffu, need)) {
-            const float alpha = need ? ex2(m_ref - m_new) : 1.f;
-            if (need) m_ref = m_new;
+          warp_rescale = __any_sync(0xffffffffu, need);
+          if (need) {
+            alpha = ex2(m_ref - m_new);
+            m_ref = m_new;
             l *= alpha;
-            // O must hold the previous block's product before it is scaled
-            if (!mbar_wait_warp(BAR(C::B_ODONE + odone_idx(j - 1)), odone_par(j - 1), wc, 6)) { ok = false; break; }
-            tc_fence_after();
-#pragma unroll
-            for (int oc = 0; oc < D / 32; ++oc) {
-              uint32_t ov[32];
-              tmem_ld32(tl + ocol + oc * 32, ov);
-              tmem_ld_wait();
-              reg_fence(ov);
-#pragma unroll
-              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-              tmem_st32(tl + ocol + oc * 32, ov);
-            }
-            tmem_st_wait();
           }
         }
+        // P = 2^(s·scale·log2e − m_ref), rounded to bf16 and written over the
+        // first 64 columns of S, 32 source columns (16 TMEM columns) at a time
         const float neg_m = -m_ref;
-        float rs0 = 0.f, rs1 = 0.f;
-        uint32_t pk0[32], pk1[32];
+        float rs[4] = {0.f, 0.f, 0.f, 0.f};
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float a0 = ex2(fmaf(s[2 * c], sl2, neg_m));
-          const float a1 = ex2(fmaf(s[2 * c + 1], sl2, neg_m));
-          rs0 += a0;
-          rs1 += a1;
-          pk0[c] = pack_bf16(a0, a1);
-        }
+        for (int q4 = 0; q4 < 4; ++q4) {
+          uint32_t pk[16];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) {
-          const float a0 = ex2(fmaf(s[64 + 2 * c], sl2, neg_m));
-          const float a1 = ex2(fmaf(s[64 + 2 * c + 1], sl2, neg_m));
-          rs0 += a0;
-          rs1 += a1;
-          pk1[c] = pack_bf16(a0, a1);
+          for (int c = 0; c < 16; ++c) {
+            const float a0 = ex2(fmaf(s[32 * q4 + 2 * c], sl2, neg_m));
+            const float a1 = ex2(fmaf(s[32 * q4 + 2 * c + 1], sl2, neg_m));
+            rs[(c & 1) * 2 + 0] += a0;
+            rs[(c & 1) * 2 + 1] += a1;
+            pk[c] = pack_bf16(a0, a1);
+          }
+          tmem_st16(tl + scol + 16 * q4, pk);
         }
-        l += rs0 + rs1;
-        tmem_st32(tl + scol + 0, pk0);
-        tmem_st32(tl + scol + 32, pk1);
+        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        if (warp_rescale) {
+          // O must hold the previous block's product before it is scaled
+          if (!mbar_wait_warp(BAR(C::B_ODONE + odone_idx(j - 1)), odone_par(j - 1), wc, 6)) { ok = false; break; }
+          tc_fence_after();
+#pragma unroll
+          for (int oc = 0; oc < D / 32; ++oc) {
+            uint32_t ov[32];
+            tmem_ld32(tl + ocol + oc * 32, ov);
+            tmem_ld_wait();
+            reg_fence(ov);
+#pragma unroll
+            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+            tmem_st32(tl + ocol + oc * 32, ov);
+          }
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
