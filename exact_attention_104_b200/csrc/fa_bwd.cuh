@@ -250,56 +250,57 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         tc_fence_after();
         return r;
       };
+      // Descriptors are built once; each MMA only adds a compile-time offset
+      // (the issuing thread must keep up with 48-cycle MMAs).
+      const uint64_t dK_k = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
+      const uint64_t dV_k = sdesc_sw128(sbase + C::V_OFF, 16, 1024);
+      const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+      const uint64_t dDO_k = sdesc_sw128(sbase + C::DO_OFF, 16, 1024);
+      const uint64_t dQ_mn = sdesc_sw128(sbase + C::Q_OFF + (dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
+      const uint64_t dDO_mn = sdesc_sw128(sbase + C::DO_OFF + (dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
+      const uint64_t dKT_mn = sdesc_sw128(sbase + C::K_OFF + (dh * C::DH / 64) * C::KV_PANEL, C::KV_PANEL, 1024);
+      const uint64_t dDS_mn = sdesc_sw128(sbase + C::DS_OFF, 16384, 1024);
       // Sᵀ / dPᵀ: [128 keys x 64 queries] = (K or V tile) · (Q or dO tile)ᵀ over D
-      auto issue_xt = [&](uint32_t a_off, uint32_t b_off, int dcol) {
+      auto issue_xt = [&](uint64_t da0, uint64_t db0, uint32_t dtm) {
 #pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const int koff = (kk & 3) * 32;
-          const uint64_t da = sdesc_sw128(sbase + a_off + (kk >> 2) * C::KV_PANEL + koff, 16, 1024);
-          const uint64_t db = sdesc_sw128(sbase + b_off + (kk >> 2) * C::Q_PANEL + koff, 16, 1024);
-          mma_ss(tbase + dcol, da, db, C::IDESC_ST, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < D / 16; ++kk)
+          mma_ss(dtm, sdesc_add(da0, (kk >> 2) * C::KV_PANEL + (kk & 3) * 32),
+                 sdesc_add(db0, (kk >> 2) * C::Q_PANEL + (kk & 3) * 32), C::IDESC_ST, kk > 0 ? 1u : 0u);
       };
       // dV or dK [128 keys x DH] += (Pᵀ or dSᵀ in TMEM) · (dO or Q tile)[:, dh half]
-      auto issue_acc = [&](int a_col, uint32_t b_off, int dcol, bool first) {
+      auto issue_acc = [&](uint32_t atm, uint64_t db0, uint32_t dtm, bool first) {
 #pragma unroll
-        for (int kk = 0; kk < C::BR / 16; ++kk) {
-          const uint64_t db =
-              sdesc_sw128(sbase + b_off + (dh * C::DH / 64) * C::Q_PANEL + kk * 2048, C::Q_PANEL, 1024);
-          mma_ts(tbase + dcol, tbase + a_col + kk * 8, db, C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
-        }
+        for (int kk = 0; kk < C::BR / 16; ++kk)
+          mma_ts(dtm, atm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
       };
       // dQᵀ [128 d-rows x 64 queries] = K[:, dh half]ᵀ · dSᵀ over the 128 keys
       auto issue_dq = [&]() {
 #pragma unroll
-        for (int kk = 0; kk < C::BC / 16; ++kk) {
-          const uint64_t da =
-              sdesc_sw128(sbase + C::K_OFF + (dh * C::DH / 64) * C::KV_PANEL + kk * 2048, C::KV_PANEL, 1024);
-          const uint64_t db = sdesc_sw128(sbase + C::DS_OFF + kk * 2048, 16384, 1024);
-          mma_ss(tbase + C::DQ_COL, da, db, C::IDESC_DQ, kk > 0 ? 1u : 0u);
-        }
+        for (int kk = 0; kk < C::BC / 16; ++kk)
+          mma_ss(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
+                 kk > 0 ? 1u : 0u);
       };
-      auto q_off = [&](int s) -> uint32_t { return C::Q_OFF + (s % C::NSTAGE) * C::Q_BYTES; };
-      auto do_off = [&](int s) -> uint32_t { return C::DO_OFF + (s % C::NSTAGE) * C::Q_BYTES; };
-
+      auto stage_bytes = [&](int s) -> uint32_t { return (uint32_t)(s % C::NSTAGE) * C::Q_BYTES; };
+      auto q_off = [&](int s) -> uint64_t { return sdesc_add(dQ_k, stage_bytes(s)); };
+      auto do_off = [&](int s) -> uint64_t { return sdesc_add(dDO_k, stage_bytes(s)); };
       if (ok) {
         for (int k = 0; k < C::LA && k < n && ok; ++k) {
           ok = wait_q(k);
           if (!ok) break;
-          issue_xt(C::K_OFF, q_off(k), C::ST_COL + 64 * (k & 1));
+          issue_xt(dK_k, q_off(k), tbase + C::ST_COL + 64 * (k & 1));
           tc_commit(BAR(C::B_SFULL + (k & 1)));
         }
         if (ok) {
-          issue_xt(C::V_OFF, do_off(0), C::DP_COL);
+          issue_xt(dV_k, do_off(0), tbase + C::DP_COL);
           tc_commit(BAR(C::B_DPFULL));
         }
         for (int s = 0; s < n && ok; ++s) {
           if (!mbar_wait(BAR(C::B_PFULL + (s & 1)), (s >> 1) & 1, wc, 14)) { ok = false; break; }
           tc_fence_after();
-          issue_acc(C::ST_COL + 64 * (s & 1), do_off(s), C::DV_COL, s == 0);
+          issue_acc(tbase + C::ST_COL + 64 * (s & 1), sdesc_add(dDO_mn, stage_bytes(s)), tbase + C::DV_COL, s == 0);
           if (!mbar_wait(BAR(C::B_DSFULL), s & 1, wc, 15)) { ok = false; break; }
           tc_fence_after();
-          issue_acc(C::DP_COL, q_off(s), C::DK_COL, s == 0);
+          issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(s)), tbase + C::DK_COL, s == 0);
           tc_commit(BAR(C::B_QEMPTY + s % C::NSTAGE));
           if (s > 0) {
             if (!mbar_wait(BAR(C::B_DQEMPTY), (s - 1) & 1, wc, 16)) { ok = false; break; }
@@ -310,13 +311,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           // dPᵀ of the next step first: the compute warps are waiting for it
           if (s + 1 < n) {
             if (C::LA == 1 && !wait_q(s + 1)) { ok = false; break; }
-            issue_xt(C::V_OFF, do_off(s + 1), C::DP_COL);
+            issue_xt(dV_k, do_off(s + 1), tbase + C::DP_COL);
             tc_commit(BAR(C::B_DPFULL));
           }
           if (s + C::LA < n) {
             const int s2 = s + C::LA;
             if (C::LA > 1 && !wait_q(s2)) { ok = false; break; }
-            issue_xt(C::K_OFF, q_off(s2), C::ST_COL + 64 * (s2 & 1));
+            issue_xt(dK_k, q_off(s2), tbase + C::ST_COL + 64 * (s2 & 1));
             tc_commit(BAR(C::B_SFULL + (s2 & 1)));
           }
         }

@@ -24,6 +24,22 @@
 namespace fa {
 
 constexpr float kRescaleTau = 8.0f;
+constexpr int kPrefetchUnits = 0;  // K/V tiles prefetched into L2 ahead of their load
+
+// Softmax tuning knobs (all variants compute the same P up to rounding):
+//   FA_POLY_PAIRS  n > 0: the second exponential of every n-th column pair runs
+//                  on the FMA pipes (exp2_poly); 0 keeps every one on the MUFU
+//   FA_SPLIT_P     hand P to the MMA warp in two 64-key halves
+//   FA_PACKED_F32  scale/shift and row sums with packed fp32x2 instructions
+#ifndef FA_POLY_PAIRS
+#define FA_POLY_PAIRS 0
+#endif
+#ifndef FA_SPLIT_P
+#define FA_SPLIT_P 1
+#endif
+#ifndef FA_PACKED_F32
+#define FA_PACKED_F32 1
+#endif
 
 template <int D>
 struct FwdCfg {
@@ -36,7 +52,7 @@ struct FwdCfg {
   static constexpr int PANEL = 128 * 128;        // one 64-column panel of a 128-row tile (bytes)
   static constexpr int Q_BYTES = BM * D * 2;
   static constexpr int SLOT_BYTES = BN * CH * 2;
-  static constexpr int NSLOT = (D == 64) ? 8 : 4;
+  static constexpr int NSLOT = (D == 64) ? 8 : 5;
   static constexpr int Q_OFF = 0;
   static constexpr int KV_OFF = NQ * Q_BYTES;
   static constexpr int BAR_OFF = KV_OFF + NSLOT * SLOT_BYTES;
@@ -45,8 +61,9 @@ struct FwdCfg {
   static constexpr int B_KVFULL = 1;                 // + slot
   static constexpr int B_KVEMPTY = 1 + NSLOT;        // + slot
   static constexpr int B_SFULL = 1 + 2 * NSLOT;      // + {0,1}
-  static constexpr int B_PFULL = B_SFULL + 2;        // + {0,1}
-  static constexpr int B_ODONE = B_PFULL + 2;        // + {0,1}
+  static constexpr int B_PFULL = B_SFULL + 2;        // + {0,1}: P keys 0..63 in TMEM
+  static constexpr int B_PFULL2 = B_PFULL + 2;       // + {0,1}: P keys 64..127 in TMEM
+  static constexpr int B_ODONE = B_PFULL2 + 2;       // + {0,1}
   static constexpr int B_DRAIN = B_ODONE + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
@@ -148,6 +165,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(C::B_SFULL + i), 1);
       mbar_init(BAR(C::B_PFULL + i), 4);
+      mbar_init(BAR(C::B_PFULL2 + i), 4);
       mbar_init(BAR(C::B_ODONE + i), 1);
     }
     mbar_init(BAR(C::B_DRAIN), 1);
@@ -186,11 +204,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           tma_load_2d_hint(sbase + C::Q_OFF + t * C::Q_BYTES + pn * C::PANEL, &tmQ, BAR(C::B_QFULL), pn * 64,
                            q_row_base + (qt0 + t) * C::BM, pol_q);
       }
+      // L2 prefetch of unit u: a K/V tile in shared memory only one step ahead
+      // would still wait for HBM/L2 latency; the prefetch runs kPrefetchUnits ahead
+      auto prefetch_unit = [&](int u) {
+        bool pv;
+        int pj;
+        Ord::decode(u, nmax, pv, pj);
+#pragma unroll
+        for (int pn = 0; pn < D / 64; ++pn) tma_prefetch_l2_2d(pv ? &tmV : &tmK, pn * 64, kv_row_base + pj * C::BN);
+      };
+      for (int u = 0; u < kPrefetchUnits && u < 2 * nmax; ++u) prefetch_unit(u);
       bool ok = true;
       for (int u = 0; u < 2 * nmax && ok; ++u) {
         bool is_v;
         int j;
         Ord::decode(u, nmax, is_v, j);
+        if (u + kPrefetchUnits < 2 * nmax) prefetch_unit(u + kPrefetchUnits);
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const int seq = u * C::NCH + c;
@@ -234,32 +263,36 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         v_ready = j;
         return wait_unit(Ord::unitV(j, nmax));
       };
+      // Descriptors are built once; each MMA only adds a compile-time offset.
+      const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+      const uint64_t dKV_k = sdesc_sw128(sbase + C::KV_OFF, 16, 1024);
+      const uint64_t dKV_mn = sdesc_sw128(sbase + C::KV_OFF, C::PANEL, 1024);
       // S[scol] = Q_t · K_jᵀ   (M=128 queries, N=128 keys, K=D)
       auto issue_s = [&](int t, int j, int scol) {
-        const int uk = Ord::unitK(j, nmax);
+        const int seq0 = Ord::unitK(j, nmax) * C::NCH;
+        const uint64_t da0 = sdesc_add(dQ_k, t * C::Q_BYTES);
+        uint64_t db0[C::NCH];
+#pragma unroll
+        for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((seq0 + c) % C::NSLOT) * C::SLOT_BYTES);
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const int koff = (kk & 3) * 32;
-          const uint64_t da = sdesc_sw128(sbase + C::Q_OFF + t * C::Q_BYTES + (kk >> 2) * C::PANEL + koff, 16, 1024);
           const int col = kk * 16;
-          const int seq = uk * C::NCH + col / C::CH;
-          const int slot = seq % C::NSLOT;
-          const uint64_t db = sdesc_sw128(
-              sbase + C::KV_OFF + slot * C::SLOT_BYTES + ((col % C::CH) / 64) * C::PANEL + koff, 16, 1024);
-          mma_ss(tbase + scol, da, db, C::IDESC_S, kk > 0 ? 1u : 0u);
+          mma_ss(tbase + scol, sdesc_add(da0, (kk >> 2) * C::PANEL + (kk & 3) * 32),
+                 sdesc_add(db0[col / C::CH], ((col % C::CH) / 64) * C::PANEL + (kk & 3) * 32), C::IDESC_S,
+                 kk > 0 ? 1u : 0u);
         }
       };
-      // O_t[:, c*CH..] (+)= P(TMEM at scol) · V_j[:, c*CH..]   (K = 128 keys)
-      auto issue_pv = [&](int j, int scol, int ocol) {
-        const int uv = Ord::unitV(j, nmax);
+      // O_t[:, c*CH..] (+)= P(TMEM at scol) · V_j[:, c*CH..]; half 0 covers keys
+      // 0..63 of the tile, half 1 keys 64..127
+      auto issue_pv = [&](int j, int scol, int ocol, int half) {
+        const int seq0 = Ord::unitV(j, nmax) * C::NCH;
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          const int slot = (uv * C::NCH + c) % C::NSLOT;
+          const uint64_t db0 = sdesc_add(dKV_mn, ((seq0 + c) % C::NSLOT) * C::SLOT_BYTES);
 #pragma unroll
-          for (int kk = 0; kk < C::BN / 16; ++kk) {
-            const uint64_t db = sdesc_sw128(sbase + C::KV_OFF + slot * C::SLOT_BYTES + kk * 2048, C::PANEL, 1024);
-            mma_ts(tbase + ocol + c * C::CH, tbase + scol + kk * 8, db, C::IDESC_PV, (j > 0 || kk > 0) ? 1u : 0u);
-          }
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+            mma_ts(tbase + ocol + c * C::CH, tbase + scol + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_PV,
+                   (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
 
@@ -279,8 +312,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               if (!mbar_wait(BAR(C::B_PFULL + t), j & 1, wc, 4)) { ok = false; break; }
               tc_fence_after();
               if (!need_v(j)) { ok = false; break; }
-              issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D);
+              issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D, 0);
+              if (!mbar_wait(BAR(C::B_PFULL2 + t), j & 1, wc, 10)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D, 1);
               tc_commit(BAR(C::B_ODONE + t));
+              if (t == 1 || j >= n_t[1]) release_unit(Ord::unitV(j, nmax));  // last reader of V(j)
               if (j + 1 < n_t[t]) {
                 if (!need_k(j + 1)) { ok = false; break; }
                 issue_s(t, j + 1, C::S_COL + 128 * t);
@@ -288,7 +325,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
               }
             }
             if (!ok) break;
-            release_unit(Ord::unitV(j, nmax));
             if (j + 1 < nmax) release_unit(Ord::unitK(j + 1, nmax));
           }
         } else {
@@ -312,7 +348,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             if (!mbar_wait(BAR(C::B_PFULL + x), (j >> 1) & 1, wc, 4)) { ok = false; break; }
             tc_fence_after();
             if (!need_v(j)) { ok = false; break; }
-            issue_pv(j, C::S_COL + 128 * x, C::O_COL);
+            issue_pv(j, C::S_COL + 128 * x, C::O_COL, 0);
+            if (!mbar_wait(BAR(C::B_PFULL2 + x), (j >> 1) & 1, wc, 10)) { ok = false; break; }
+            tc_fence_after();
+            issue_pv(j, C::S_COL + 128 * x, C::O_COL, 1);
             tc_commit(BAR(C::B_ODONE + x));
             release_unit(Ord::unitV(j, n));
             if (j + 2 < n) {
@@ -397,42 +436,82 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           }
         }
         // P = 2^(s·scale·log2e − m_ref), rounded to bf16 and written over the
-        // first 64 columns of S, 32 source columns (16 TMEM columns) at a time
+        // first 64 columns of S.  With FA_SPLIT_P, keys 0..63 are handed to the
+        // MMA warp before keys 64..127 are exponentiated, so the first half of
+        // the PV product overlaps the second half of the exponentials.
         const float neg_m = -m_ref;
+        uint64_t rs2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
         float rs[4] = {0.f, 0.f, 0.f, 0.f};
+        auto exp_half = [&](int base, uint32_t (&pk)[32]) {
 #pragma unroll
-        for (int q4 = 0; q4 < 4; ++q4) {
-          uint32_t pk[16];
-#pragma unroll
-          for (int c = 0; c < 16; ++c) {
-            const float a0 = ex2(fmaf(s[32 * q4 + 2 * c], sl2, neg_m));
-            const float a1 = ex2(fmaf(s[32 * q4 + 2 * c + 1], sl2, neg_m));
-            rs[(c & 1) * 2 + 0] += a0;
-            rs[(c & 1) * 2 + 1] += a1;
+          for (int c = 0; c < 32; ++c) {
+            float x0, x1;
+            if (FA_PACKED_F32) {
+              f2_split(f2_fma(f2_make(s[base + 2 * c], s[base + 2 * c + 1]), f2_make(sl2, sl2), f2_make(neg_m, neg_m)),
+                       x0, x1);
+            } else {
+              x0 = fmaf(s[base + 2 * c], sl2, neg_m);
+              x1 = fmaf(s[base + 2 * c + 1], sl2, neg_m);
+            }
+            const float a0 = ex2(x0);
+            const float a1 = (FA_POLY_PAIRS > 0 && c % (FA_POLY_PAIRS > 0 ? FA_POLY_PAIRS : 1) == 0) ? exp2_poly(x1)
+                                                                                                     : ex2(x1);
+            if (FA_PACKED_F32) {
+              rs2[c & 1] = f2_add(rs2[c & 1], f2_make(a0, a1));
+            } else {
+              rs[(c & 1) * 2 + 0] += a0;
+              rs[(c & 1) * 2 + 1] += a1;
+            }
             pk[c] = pack_bf16(a0, a1);
           }
-          tmem_st16(tl + scol + 16 * q4, pk);
-        }
-        l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        if (warp_rescale) {
-          // O must hold the previous block's product before it is scaled
-          if (!mbar_wait_warp(BAR(C::B_ODONE + odone_idx(j - 1)), odone_par(j - 1), wc, 6)) { ok = false; break; }
-          tc_fence_after();
+        };
+        {
+          uint32_t pk[32];
+          exp_half(0, pk);
+          if (warp_rescale) {
+            // O must hold the previous block's product before it is scaled,
+            // and be scaled before this block's first PV half accumulates
+            if (!mbar_wait_warp(BAR(C::B_ODONE + odone_idx(j - 1)), odone_par(j - 1), wc, 6)) { ok = false; break; }
+            tc_fence_after();
 #pragma unroll
-          for (int oc = 0; oc < D / 32; ++oc) {
-            uint32_t ov[32];
-            tmem_ld32(tl + ocol + oc * 32, ov);
-            tmem_ld_wait();
-            reg_fence(ov);
+            for (int oc = 0; oc < D / 32; ++oc) {
+              uint32_t ov[32];
+              tmem_ld32(tl + ocol + oc * 32, ov);
+              tmem_ld_wait();
+              reg_fence(ov);
 #pragma unroll
-            for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
-            tmem_st32(tl + ocol + oc * 32, ov);
+              for (int c = 0; c < 32; ++c) ov[c] = __float_as_uint(__uint_as_float(ov[c]) * alpha);
+              tmem_st32(tl + ocol + oc * 32, ov);
+            }
+          }
+          tmem_st32(tl + scol, pk);
+          if (FA_SPLIT_P) {
+            tmem_st_wait();
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(BAR(C::B_PFULL + x));
           }
         }
-        tmem_st_wait();
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive(BAR(C::B_PFULL + x));
+        {
+          uint32_t pk[32];
+          exp_half(64, pk);
+          tmem_st32(tl + scol + 32, pk);
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) {
+            if (!FA_SPLIT_P) mbar_arrive(BAR(C::B_PFULL + x));
+            mbar_arrive(BAR(C::B_PFULL2 + x));
+          }
+        }
+        if (FA_PACKED_F32) {
+          float a, b2, c2, d2;
+          f2_split(rs2[0], a, b2);
+          f2_split(rs2[1], c2, d2);
+          l += (a + b2) + (c2 + d2);
+        } else {
+          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
+        }
       }
       if (ok) ok = mbar_wait_warp(BAR(C::B_ODONE + odone_idx(n - 1)), odone_par(n - 1), wc, 7);
       if (ok) {

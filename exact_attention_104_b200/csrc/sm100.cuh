@@ -116,6 +116,13 @@ __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap
       : "memory");
 }
 
+// Prefetch one 2-D box of a tensor into L2 (no shared memory, no barrier).
+__device__ __forceinline__ void tma_prefetch_l2_2d(const CUtensorMap* m, int x, int y) {
+  asm volatile("cp.async.bulk.prefetch.tensor.2d.L2.global.tile [%0, {%1, %2}];" ::"l"(reinterpret_cast<uint64_t>(m)),
+               "r"(x), "r"(y)
+               : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_last() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_last.b64 %0, 1.0;" : "=l"(p));
@@ -225,6 +232,10 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo, ui
   return d;
 }
 
+// Descriptor of the same layout `bytes` further on (start-address field only;
+// shared-memory offsets stay far below the field's 256 KB range).
+__device__ __forceinline__ uint64_t sdesc_add(uint64_t d, uint32_t bytes) { return d + (uint64_t)(bytes >> 4); }
+
 // TMEM address: lane in bits 16..31, column in bits 0..15.
 __device__ __forceinline__ uint32_t tmem_addr(uint32_t base, uint32_t lane, uint32_t col) {
   return base + (lane << 16) + col;
@@ -282,6 +293,46 @@ __device__ __forceinline__ float ex2(float x) {
   asm("ex2.approx.ftz.f32 %0, %1;" : "=f"(y) : "f"(x));
   return y;
 }
+// 2^x on the FMA/ALU pipes instead of the MUFU unit, for x <= ~8.
+// Range reduction: n = round(x) by adding and subtracting 1.5·2^23 (the sum
+// keeps n in its low mantissa bits), f = x − n ∈ [−1/2, 1/2].  2^f is the cubic
+// 1 + c1·f + c2·f² + c3·f³ (constant term pinned to 1 so integer x is exact)
+// with c1..c3 fitted to 2^f on [−1/2, 1/2] by iteratively reweighted least
+// squares on the relative error (max relative error 1.0e-4, far below the
+// 2^-9 half-ulp of the bf16 value it feeds).  2^n is applied by
+// adding n to the exponent field; x is clamped at −126 so that the exponent
+// never underflows (inputs of −inf give ~1e-38 instead of 0).
+__device__ __forceinline__ float exp2_poly(float x) {
+  x = fmaxf(x, -126.0f);
+  const float r = __fadd_rn(x, 12582912.0f);
+  const float n = __fadd_rn(r, -12582912.0f);
+  const float f = __fadd_rn(x, -n);
+  float p = fmaf(0.055008918046951294f, f, 0.2422109842300415f);
+  p = fmaf(p, f, 0.693282961845398f);
+  p = fmaf(p, f, 1.0f);
+  return __int_as_float(__float_as_int(p) + (__float_as_int(r) << 23));
+}
+
+// Packed fp32x2 arithmetic (two lanes per instruction).
+__device__ __forceinline__ uint64_t f2_make(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_split(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t f2_fma(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t r;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(r) : "l"(a), "l"(b), "l"(c));
+  return r;
+}
+__device__ __forceinline__ uint64_t f2_add(uint64_t a, uint64_t b) {
+  uint64_t r;
+  asm("add.rn.f32x2 %0, %1, %2;" : "=l"(r) : "l"(a), "l"(b));
+  return r;
+}
+
 // max(a, b, c) in one instruction (three-input form of max.f32).
 __device__ __forceinline__ float fmax3(float a, float b, float c) {
   float r;
