@@ -50,6 +50,10 @@ def lib() -> ctypes.CDLL:
     L.fa_set_wait_cap.restype = i
     L.fa_profile_next.argtypes = [vp, vp]
     L.fa_profile_next.restype = i
+    L.fa_selftest_wait_timeout.argtypes = [ctypes.c_longlong, vp]
+    L.fa_selftest_wait_timeout.restype = i
+    L.fa_selftest_exp2.argtypes = [vp, vp, ctypes.c_longlong, i, vp]
+    L.fa_selftest_exp2.restype = i
     L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.fa_bwd_noalloc.restype = i
     _lib = L
@@ -101,6 +105,14 @@ def fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, wor
     return lib().fa_bwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk), _ptr(dv),
                         B, Hq, Hkv, N, d, int(bool(causal)), float(scale), _ptr(workspace),
                         int(workspace_bytes), _stream_handle(stream))
+
+
+def fa_selftest_wait_timeout(cap_cycles: int, stream=None) -> int:
+    return lib().fa_selftest_wait_timeout(int(cap_cycles), _stream_handle(stream))
+
+
+def fa_selftest_exp2(x, y, use_poly: bool, stream=None) -> int:
+    return lib().fa_selftest_exp2(_ptr(x), _ptr(y), int(x.numel()), int(bool(use_poly)), _stream_handle(stream))
 
 
 FA_NOALLOC_SCRATCH_BYTES = 64 * 1024 * 1024

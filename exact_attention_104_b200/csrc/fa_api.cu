@@ -224,6 +224,26 @@ fa_status noalloc_scratch(void** out) {
 
 }  // namespace
 
+namespace fa {
+// One thread waits on a barrier nothing arrives on; the bounded wait gives up.
+__global__ void selftest_wait_kernel(long long cap, int* err) {
+  __shared__ uint64_t bar;
+  __shared__ int abort_flag;
+  if (threadIdx.x == 0) {
+    mbar_init(smem_u32(&bar), 1);
+    abort_flag = 0;
+    fence_mbar_init();
+    const WaitCtx wc{&abort_flag, err, cap};
+    mbar_wait(smem_u32(&bar), 0, wc, 99);
+  }
+}
+__global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restrict__ y, long long n, int poly) {
+  const long long stride = (long long)gridDim.x * blockDim.x;
+  for (long long i = (long long)blockIdx.x * blockDim.x + threadIdx.x; i < n; i += stride)
+    y[i] = poly ? exp2_poly(x[i]) : ex2(x[i]);
+}
+}  // namespace fa
+
 extern "C" {
 
 const char* fa_status_string(fa_status s) {
@@ -242,6 +262,29 @@ fa_status fa_profile_next(void* start_event, void* stop_event) {
   t_prof_start = static_cast<cudaEvent_t>(start_event);
   t_prof_stop = static_cast<cudaEvent_t>(stop_event);
   return FA_OK;
+}
+
+fa_status fa_selftest_wait_timeout(long long cap_cycles, void* stream) {
+  if (cap_cycles < 1 || cap_cycles > (1LL << 31)) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  fa::selftest_wait_kernel<<<1, 32, 0, static_cast<cudaStream_t>(stream)>>>(cap_cycles, di->err);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status fa_selftest_exp2(const float* x, float* y, long long n, int use_poly, void* stream) {
+  if (n < 0) return FA_ERR_INVALID_ARG;
+  if (n == 0) return FA_OK;
+  if (!x || !y || !aligned16(x) || !aligned16(y)) return FA_ERR_INVALID_ARG;
+  if (overlap(span(x, (size_t)n * 4), span(y, (size_t)n * 4))) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  fa_status st = current_device(&di);
+  if (st != FA_OK) return st;
+  long long blocks = (n + 255) / 256;
+  if (blocks > (long long)di->sms * 8) blocks = (long long)di->sms * 8;
+  fa::selftest_exp2_kernel<<<(unsigned)blocks, 256, 0, static_cast<cudaStream_t>(stream)>>>(x, y, n, use_poly);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 fa_status fa_set_wait_cap(long long cycles) {

@@ -242,11 +242,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(BAR(C::B_KVFULL), 0, wc, 12);
+    // (the whole warp runs this role; one elected lane issues each instruction)
+    {
+      bool ok = mbar_wait_warp(BAR(C::B_KVFULL), 0, wc, 12);
       tc_fence_after();
       auto wait_q = [&](int s) -> bool {
-        const bool r = mbar_wait(BAR(C::B_QFULL + s % C::NSTAGE), (s / C::NSTAGE) & 1, wc, 13);
+        const bool r = mbar_wait_warp(BAR(C::B_QFULL + s % C::NSTAGE), (s / C::NSTAGE) & 1, wc, 13);
         tc_fence_after();
         return r;
       };
@@ -264,20 +265,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       auto issue_xt = [&](uint64_t da0, uint64_t db0, uint32_t dtm) {
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk)
-          mma_ss(dtm, sdesc_add(da0, (kk >> 2) * C::KV_PANEL + (kk & 3) * 32),
+          mma_ss_w(dtm, sdesc_add(da0, (kk >> 2) * C::KV_PANEL + (kk & 3) * 32),
                  sdesc_add(db0, (kk >> 2) * C::Q_PANEL + (kk & 3) * 32), C::IDESC_ST, kk > 0 ? 1u : 0u);
       };
       // dV or dK [128 keys x DH] += (Pᵀ or dSᵀ in TMEM) · (dO or Q tile)[:, dh half]
       auto issue_acc = [&](uint32_t atm, uint64_t db0, uint32_t dtm, bool first) {
 #pragma unroll
         for (int kk = 0; kk < C::BR / 16; ++kk)
-          mma_ts(dtm, atm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
+          mma_ts_w(dtm, atm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
       };
       // dQᵀ [128 d-rows x 64 queries] = K[:, dh half]ᵀ · dSᵀ over the 128 keys
       auto issue_dq = [&]() {
 #pragma unroll
         for (int kk = 0; kk < C::BC / 16; ++kk)
-          mma_ss(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
+          mma_ss_w(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
                  kk > 0 ? 1u : 0u);
       };
       auto stage_bytes = [&](int s) -> uint32_t { return (uint32_t)(s % C::NSTAGE) * C::Q_BYTES; };
@@ -288,43 +289,43 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           ok = wait_q(k);
           if (!ok) break;
           issue_xt(dK_k, q_off(k), tbase + C::ST_COL + 64 * (k & 1));
-          tc_commit(BAR(C::B_SFULL + (k & 1)));
+          tc_commit_w(BAR(C::B_SFULL + (k & 1)));
         }
         if (ok) {
           issue_xt(dV_k, do_off(0), tbase + C::DP_COL);
-          tc_commit(BAR(C::B_DPFULL));
+          tc_commit_w(BAR(C::B_DPFULL));
         }
         for (int s = 0; s < n && ok; ++s) {
-          if (!mbar_wait(BAR(C::B_PFULL + (s & 1)), (s >> 1) & 1, wc, 14)) { ok = false; break; }
+          if (!mbar_wait_warp(BAR(C::B_PFULL + (s & 1)), (s >> 1) & 1, wc, 14)) { ok = false; break; }
           tc_fence_after();
           issue_acc(tbase + C::ST_COL + 64 * (s & 1), sdesc_add(dDO_mn, stage_bytes(s)), tbase + C::DV_COL, s == 0);
-          if (!mbar_wait(BAR(C::B_DSFULL), s & 1, wc, 15)) { ok = false; break; }
+          if (!mbar_wait_warp(BAR(C::B_DSFULL), s & 1, wc, 15)) { ok = false; break; }
           tc_fence_after();
           issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(s)), tbase + C::DK_COL, s == 0);
-          tc_commit(BAR(C::B_QEMPTY + s % C::NSTAGE));
+          tc_commit_w(BAR(C::B_QEMPTY + s % C::NSTAGE));
           if (s > 0) {
-            if (!mbar_wait(BAR(C::B_DQEMPTY), (s - 1) & 1, wc, 16)) { ok = false; break; }
+            if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (s - 1) & 1, wc, 16)) { ok = false; break; }
             tc_fence_after();
           }
           issue_dq();
-          tc_commit(BAR(C::B_DQFULL));
+          tc_commit_w(BAR(C::B_DQFULL));
           // dPᵀ of the next step first: the compute warps are waiting for it
           if (s + 1 < n) {
             if (C::LA == 1 && !wait_q(s + 1)) { ok = false; break; }
             issue_xt(dV_k, do_off(s + 1), tbase + C::DP_COL);
-            tc_commit(BAR(C::B_DPFULL));
+            tc_commit_w(BAR(C::B_DPFULL));
           }
           if (s + C::LA < n) {
             const int s2 = s + C::LA;
             if (C::LA > 1 && !wait_q(s2)) { ok = false; break; }
             issue_xt(dK_k, q_off(s2), tbase + C::ST_COL + 64 * (s2 & 1));
-            tc_commit(BAR(C::B_SFULL + (s2 & 1)));
+            tc_commit_w(BAR(C::B_SFULL + (s2 & 1)));
           }
         }
-        if (ok) tc_commit(BAR(C::B_ACC));
+        if (ok) tc_commit_w(BAR(C::B_ACC));
       }
-      tc_commit(BAR(C::B_DRAIN));
-      mbar_wait(BAR(C::B_DRAIN), 0, wc, 17);
+      tc_commit_w(BAR(C::B_DRAIN));
+      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 17);
     }
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------- compute: Pᵀ and dSᵀ rows

@@ -236,22 +236,23 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     }
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
-    if (lane == 0) {
-      bool ok = mbar_wait(BAR(C::B_QFULL), 0, wc, 2);
+    // (the whole warp runs this role; one elected lane issues each instruction)
+    {
+      bool ok = mbar_wait_warp(BAR(C::B_QFULL), 0, wc, 2);
       tc_fence_after();
       int k_ready = -1, v_ready = -1;
       auto wait_unit = [&](int u) -> bool {
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const int seq = u * C::NCH + c;
-          if (!mbar_wait(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 3)) return false;
+          if (!mbar_wait_warp(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 3)) return false;
         }
         tc_fence_after();
         return true;
       };
       auto release_unit = [&](int u) {
 #pragma unroll
-        for (int c = 0; c < C::NCH; ++c) tc_commit(BAR(C::B_KVEMPTY + (u * C::NCH + c) % C::NSLOT));
+        for (int c = 0; c < C::NCH; ++c) tc_commit_w(BAR(C::B_KVEMPTY + (u * C::NCH + c) % C::NSLOT));
       };
       auto need_k = [&](int j) -> bool {
         if (j <= k_ready) return true;
@@ -277,7 +278,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int col = kk * 16;
-          mma_ss(tbase + scol, sdesc_add(da0, (kk >> 2) * C::PANEL + (kk & 3) * 32),
+          mma_ss_w(tbase + scol, sdesc_add(da0, (kk >> 2) * C::PANEL + (kk & 3) * 32),
                  sdesc_add(db0[col / C::CH], ((col % C::CH) / 64) * C::PANEL + (kk & 3) * 32), C::IDESC_S,
                  kk > 0 ? 1u : 0u);
         }
@@ -291,7 +292,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           const uint64_t db0 = sdesc_add(dKV_mn, ((seq0 + c) % C::NSLOT) * C::SLOT_BYTES);
 #pragma unroll
           for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-            mma_ts(tbase + ocol + c * C::CH, tbase + scol + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_PV,
+            mma_ts_w(tbase + ocol + c * C::CH, tbase + scol + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_PV,
                    (j > 0 || kk > 0) ? 1u : 0u);
         }
       };
@@ -303,25 +304,25 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             ok = need_k(0);
             if (!ok) break;
             issue_s(t, 0, C::S_COL + 128 * t);
-            tc_commit(BAR(C::B_SFULL + t));
+            tc_commit_w(BAR(C::B_SFULL + t));
           }
           if (ok) release_unit(Ord::unitK(0, nmax));
           for (int j = 0; j < nmax && ok; ++j) {
             for (int t = 0; t < 2; ++t) {
               if (j >= n_t[t]) continue;
-              if (!mbar_wait(BAR(C::B_PFULL + t), j & 1, wc, 4)) { ok = false; break; }
+              if (!mbar_wait_warp(BAR(C::B_PFULL + t), j & 1, wc, 4)) { ok = false; break; }
               tc_fence_after();
               if (!need_v(j)) { ok = false; break; }
               issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D, 0);
-              if (!mbar_wait(BAR(C::B_PFULL2 + t), j & 1, wc, 10)) { ok = false; break; }
+              if (!mbar_wait_warp(BAR(C::B_PFULL2 + t), j & 1, wc, 10)) { ok = false; break; }
               tc_fence_after();
               issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D, 1);
-              tc_commit(BAR(C::B_ODONE + t));
+              tc_commit_w(BAR(C::B_ODONE + t));
               if (t == 1 || j >= n_t[1]) release_unit(Ord::unitV(j, nmax));  // last reader of V(j)
               if (j + 1 < n_t[t]) {
                 if (!need_k(j + 1)) { ok = false; break; }
                 issue_s(t, j + 1, C::S_COL + 128 * t);
-                tc_commit(BAR(C::B_SFULL + t));
+                tc_commit_w(BAR(C::B_SFULL + t));
               }
             }
             if (!ok) break;
@@ -332,40 +333,40 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           ok = need_k(0);
           if (ok) {
             issue_s(0, 0, C::S_COL);
-            tc_commit(BAR(C::B_SFULL + 0));
+            tc_commit_w(BAR(C::B_SFULL + 0));
             release_unit(Ord::unitK(0, n));
           }
           if (ok && n > 1) {
             ok = need_k(1);
             if (ok) {
               issue_s(0, 1, C::S_COL + 128);
-              tc_commit(BAR(C::B_SFULL + 1));
+              tc_commit_w(BAR(C::B_SFULL + 1));
               release_unit(Ord::unitK(1, n));
             }
           }
           for (int j = 0; j < n && ok; ++j) {
             const int x = j & 1;
-            if (!mbar_wait(BAR(C::B_PFULL + x), (j >> 1) & 1, wc, 4)) { ok = false; break; }
+            if (!mbar_wait_warp(BAR(C::B_PFULL + x), (j >> 1) & 1, wc, 4)) { ok = false; break; }
             tc_fence_after();
             if (!need_v(j)) { ok = false; break; }
             issue_pv(j, C::S_COL + 128 * x, C::O_COL, 0);
-            if (!mbar_wait(BAR(C::B_PFULL2 + x), (j >> 1) & 1, wc, 10)) { ok = false; break; }
+            if (!mbar_wait_warp(BAR(C::B_PFULL2 + x), (j >> 1) & 1, wc, 10)) { ok = false; break; }
             tc_fence_after();
             issue_pv(j, C::S_COL + 128 * x, C::O_COL, 1);
-            tc_commit(BAR(C::B_ODONE + x));
+            tc_commit_w(BAR(C::B_ODONE + x));
             release_unit(Ord::unitV(j, n));
             if (j + 2 < n) {
               if (!need_k(j + 2)) { ok = false; break; }
               issue_s(0, j + 2, C::S_COL + 128 * x);
-              tc_commit(BAR(C::B_SFULL + x));
+              tc_commit_w(BAR(C::B_SFULL + x));
               release_unit(Ord::unitK(j + 2, n));
             }
           }
         }
       }
       // no MMA may still be running when TMEM is released
-      tc_commit(BAR(C::B_DRAIN));
-      mbar_wait(BAR(C::B_DRAIN), 0, wc, 8);
+      tc_commit_w(BAR(C::B_DRAIN));
+      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 8);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax

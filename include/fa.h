@@ -103,6 +103,21 @@ fa_status fa_set_wait_cap(long long cycles);
  * NULL for both cancels a pending request. */
 fa_status fa_profile_next(void* start_event, void* stop_event);
 
+/* Self-test of the failure path: launches one tiny kernel whose single
+ * thread waits, through the same bounded mbarrier wait the attention kernels
+ * use, on an on-chip barrier that nothing ever arrives on.  After
+ * `cap_cycles` SM cycles (must be in [1, 2^31]) the wait gives up, records
+ * FA_ERR_TIMEOUT in the device error word and the kernel returns normally;
+ * fa_device_status() then reports FA_ERR_TIMEOUT once.  Nothing faults or
+ * hangs, and the context stays usable. */
+fa_status fa_selftest_wait_timeout(long long cap_cycles, void* stream);
+
+/* Self-test of the device exponentials: y[i] = 2^x[i] for n floats (device
+ * pointers, 16-byte aligned), computed with the MUFU instruction
+ * (use_poly = 0) or with the FMA-pipe polynomial the softmax can use
+ * (use_poly = 1). */
+fa_status fa_selftest_exp2(const float* x, float* y, long long n, int use_poly, void* stream);
+
 /* Size in bytes of the fixed device scratch array used by fa_bwd_noalloc. */
 #define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 

@@ -67,8 +67,9 @@ def compare_sampled(w: Workload, g, units, n_rows=48, seed=0, bwd=True):
         kh, vh = f64(g["k"][b, g_kv]), f64(g["v"][b, g_kv])
         heads = list(range(g_kv * w.G, (g_kv + 1) * w.G))
         # always include the first and last rows of the sequence and of a tile
-        rows = np.unique(np.concatenate([[0, 127, 128, N - 1], rng.choice(N, n_rows, replace=False)]))
-        krows = np.unique(np.concatenate([[0, 127, N - 128, N - 1], rng.choice(N, n_rows, replace=False)]))
+        fixed = np.array([r for r in (0, 127, 128, N - 128, N - 1) if 0 <= r < N])
+        rows = np.unique(np.concatenate([fixed, rng.choice(N, min(n_rows, N), replace=False)]))
+        krows = np.unique(np.concatenate([fixed, rng.choice(N, min(n_rows, N), replace=False)]))
         qh_all = np.stack([f64(g["q"][b, h]) for h in heads])
         doh_all = np.stack([f64(g["do"][b, h]) for h in heads])
         for i, h in enumerate(heads):
