@@ -162,6 +162,13 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
+  if (C::REG_SPLIT) {
+    // the register split is sized for exactly LAUNCH_REGS per thread at launch;
+    // any other allocation could make setmaxnreg.inc wait forever
+    cudaFuncAttributes fattr;
+    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) return FA_ERR_CUDA;
+    if (fattr.numRegs != C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
+  }
   dim3 grid((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);

@@ -75,6 +75,14 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, CH, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
+  // Register split with two softmax warpgroups: the launch gives every thread
+  // LAUNCH_REGS; the control warpgroup gives registers back, the softmax
+  // warpgroups take them (128·CTRL_REGS + 256·SOFTMAX_REGS = 384·LAUNCH_REGS).
+  static constexpr int LAUNCH_REGS = 168;
+  static constexpr int CTRL_REGS = 80;
+  static constexpr int SOFTMAX_REGS = 208;
+  static constexpr bool REG_SPLIT = (NQ == 2);
+  static_assert(!REG_SPLIT || 128 * CTRL_REGS + 256 * SOFTMAX_REGS <= THREADS * LAUNCH_REGS, "register split");
 };
 
 struct FwdParams {
@@ -184,6 +192,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -237,6 +246,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // (the whole warp runs this role; one elected lane issues each instruction)
+    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     {
       bool ok = mbar_wait_warp(BAR(C::B_QFULL), 0, wc, 2);
       tc_fence_after();
@@ -368,8 +378,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tc_commit_w(BAR(C::B_DRAIN));
       mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 8);
     }
-  } else if (warp >= 4) {
+  } else if (warp < 4) {
+    // idle warps of the control warpgroup: hand their registers to the softmax
+    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
+  } else {
     // ------------------------------------------------------------- softmax
+    if (C::REG_SPLIT) setmaxnreg_inc<C::SOFTMAX_REGS>();
     const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
