@@ -163,11 +163,11 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
   if (C::REG_SPLIT) {
-    // the register split is sized for exactly LAUNCH_REGS per thread at launch;
-    // any other allocation could make setmaxnreg.inc wait forever
+    // the register split is sized for at least LAUNCH_REGS per thread at
+    // launch; fewer could make setmaxnreg.inc wait forever
     cudaFuncAttributes fattr;
     if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) return FA_ERR_CUDA;
-    if (fattr.numRegs != C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
+    if (fattr.numRegs < C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
   }
   dim3 grid((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
   ProfileScope prof(stream);
@@ -180,6 +180,12 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
   using C = fa::BwdCfg<D>;
   auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  if (C::REG_SPLIT) {
+    // the register split is sized for at least LAUNCH_REGS per thread at launch
+    cudaFuncAttributes fattr;
+    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) return FA_ERR_CUDA;
+    if (fattr.numRegs < C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
+  }
   CUtensorMap tdq;
   if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.N, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)

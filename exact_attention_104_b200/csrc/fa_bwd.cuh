@@ -81,6 +81,14 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, BR, true, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(DQ_COL + 64 <= TMEM_COLS, "TMEM budget");
+  // Register split between the warpgroups (control, compute, drain), sized for
+  // a launch of at least LAUNCH_REGS registers per thread.
+  static constexpr int LAUNCH_REGS = 160;
+  static constexpr int CTRL_REGS = 104;
+  static constexpr int COMPUTE_REGS = 208;
+  static constexpr int DRAIN_REGS = 168;
+  static constexpr bool REG_SPLIT = (D <= 128);  // d = 256 needs more than 104 in the MMA warp
+  static_assert(128 * (CTRL_REGS + COMPUTE_REGS + DRAIN_REGS) <= THREADS * LAUNCH_REGS, "register split");
 };
 
 // ------------------------------------------------------------ preprocess
@@ -213,6 +221,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
+    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -243,6 +252,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // (the whole warp runs this role; one elected lane issues each instruction)
+    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     {
       bool ok = mbar_wait_warp(BAR(C::B_KVFULL), 0, wc, 12);
       tc_fence_after();
@@ -327,8 +337,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_commit_w(BAR(C::B_DRAIN));
       mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 17);
     }
+  } else if (warp < 4) {
+    // idle warps of the control warpgroup
+    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
   } else if (warp >= 4 && warp < 8) {
     // ------------------------------------------- compute: Pᵀ and dSᵀ rows
+    if (C::REG_SPLIT) setmaxnreg_inc<C::COMPUTE_REGS>();
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row within the tile
     const int key = jt * C::BC + r;
@@ -427,6 +441,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     tc_fence_before();
   } else if (warp >= 8) {
     // ------------------------- drain: dQᵀ -> smem staging -> TMA reduce-add
+    if (C::REG_SPLIT) setmaxnreg_inc<C::DRAIN_REGS>();
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // d row of dQᵀ, key row of dV
     const int dt = threadIdx.x - 256;   // 0..127 within the drain warpgroup

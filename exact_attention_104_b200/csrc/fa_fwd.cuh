@@ -75,9 +75,9 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, CH, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
-  // Register split with two softmax warpgroups: the launch gives every thread
-  // LAUNCH_REGS; the control warpgroup gives registers back, the softmax
-  // warpgroups take them (128·CTRL_REGS + 256·SOFTMAX_REGS = 384·LAUNCH_REGS).
+  // Register split with two softmax warpgroups, sized for a launch of at least
+  // LAUNCH_REGS per thread: the control warpgroup gives registers back, the
+  // softmax warpgroups take them.
   static constexpr int LAUNCH_REGS = 168;
   static constexpr int CTRL_REGS = 80;
   static constexpr int SOFTMAX_REGS = 208;
