@@ -155,6 +155,21 @@ fa_status check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* e
 
 size_t round256(size_t x) { return (x + 255) & ~size_t(255); }
 
+// The per-warpgroup register split (setmaxnreg) of a kernel is only valid for
+// a launch allocation inside [C::MIN_LAUNCH_REGS, C::MAX_LAUNCH_REGS]: below
+// the minimum an increase would wait forever, outside the window an
+// increase/decrease would go the wrong way.  Checked before every launch.
+template <class C, class Kern>
+bool reg_split_fits(Kern kern) {
+  cudaFuncAttributes fattr;
+  if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  const int r = (fattr.numRegs + 7) & ~7;  // allocation granularity
+  return r >= C::MIN_LAUNCH_REGS && r <= C::MAX_LAUNCH_REGS;
+}
+
 template <int D, bool CAUSAL>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
                      int B, int Hq, cudaStream_t stream) {
@@ -163,11 +178,7 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
   if (C::REG_SPLIT) {
-    // the register split is sized for at least LAUNCH_REGS per thread at
-    // launch; fewer could make setmaxnreg.inc wait forever
-    cudaFuncAttributes fattr;
-    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) return FA_ERR_CUDA;
-    if (fattr.numRegs < C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
+    if (!reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
   }
   dim3 grid((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
   ProfileScope prof(stream);
@@ -180,12 +191,7 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
                           const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
   using C = fa::BwdCfg<D>;
   auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
-  if (C::REG_SPLIT) {
-    // the register split is sized for at least LAUNCH_REGS per thread at launch
-    cudaFuncAttributes fattr;
-    if (cudaFuncGetAttributes(&fattr, kern) != cudaSuccess) return FA_ERR_CUDA;
-    if (fattr.numRegs < C::LAUNCH_REGS) return FA_ERR_UNSUPPORTED;
-  }
+  if (C::REG_SPLIT && !reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
   CUtensorMap tdq;
   if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.N, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)

@@ -81,14 +81,16 @@ struct BwdCfg {
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, BR, true, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(DQ_COL + 64 <= TMEM_COLS, "TMEM budget");
-  // Register split between the warpgroups (control, compute, drain), sized for
-  // a launch of at least LAUNCH_REGS registers per thread.
-  static constexpr int LAUNCH_REGS = 160;
+  // Register split between the warpgroups (control: setmaxnreg.dec; compute
+  // and drain: setmaxnreg.inc).  Valid for a launch allocation R with
+  // CTRL_REGS <= R <= min(COMPUTE_REGS, DRAIN_REGS) and
+  // 128·(CTRL_REGS + COMPUTE_REGS + DRAIN_REGS) <= 384·R; checked on the host.
   static constexpr int CTRL_REGS = 104;
   static constexpr int COMPUTE_REGS = 208;
   static constexpr int DRAIN_REGS = 168;
   static constexpr bool REG_SPLIT = (D <= 128);  // d = 256 needs more than 104 in the MMA warp
-  static_assert(128 * (CTRL_REGS + COMPUTE_REGS + DRAIN_REGS) <= THREADS * LAUNCH_REGS, "register split");
+  static constexpr int MIN_LAUNCH_REGS = (128 * (CTRL_REGS + COMPUTE_REGS + DRAIN_REGS) + THREADS - 1) / THREADS;
+  static constexpr int MAX_LAUNCH_REGS = COMPUTE_REGS < DRAIN_REGS ? COMPUTE_REGS : DRAIN_REGS;
 };
 
 // ------------------------------------------------------------ preprocess

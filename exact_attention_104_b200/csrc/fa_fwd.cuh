@@ -75,14 +75,16 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, CH, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
-  // Register split with two softmax warpgroups, sized for a launch of at least
-  // LAUNCH_REGS per thread: the control warpgroup gives registers back, the
-  // softmax warpgroups take them.
-  static constexpr int LAUNCH_REGS = 168;
+  // Register split with two softmax warpgroups: the control warpgroup gives
+  // registers back (setmaxnreg.dec), the softmax warpgroups take them
+  // (setmaxnreg.inc).  Valid for a launch allocation R with
+  // CTRL_REGS <= R <= SOFTMAX_REGS and 128·CTRL_REGS + 256·SOFTMAX_REGS <= 384·R;
+  // the host checks R against [MIN_LAUNCH_REGS, MAX_LAUNCH_REGS] before launch.
   static constexpr int CTRL_REGS = 80;
   static constexpr int SOFTMAX_REGS = 208;
   static constexpr bool REG_SPLIT = (NQ == 2);
-  static_assert(!REG_SPLIT || 128 * CTRL_REGS + 256 * SOFTMAX_REGS <= THREADS * LAUNCH_REGS, "register split");
+  static constexpr int MIN_LAUNCH_REGS = (128 * CTRL_REGS + 256 * SOFTMAX_REGS + THREADS - 1) / THREADS;
+  static constexpr int MAX_LAUNCH_REGS = SOFTMAX_REGS;
 };
 
 struct FwdParams {
