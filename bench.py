@@ -190,6 +190,11 @@ def run_reference(args, w, rank, world):
 # ------------------------------------------------------------------- ours
 L2_BYTES = 126 * 2**20
 
+# dram__bytes_read.sum + dram__bytes_write.sum of one fa_bwd_kernel launch, from one ncu
+# capture of the current kernel (profiles/fa_kernels_d128_train_ncu_full.md).  Must be reset
+# to None whenever fa_bwd_kernel changes.
+MEASURED_TRAFFIC = {"train_b8_h16_n2048_d128": 631.2e6}
+
 
 def _l2_note(*tensors) -> str:
     nbytes = sum(t.numel() * t.element_size() for t in tensors)
@@ -343,7 +348,7 @@ def run_ours(args, w, rank, world, local_rank):
         "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
         "flops_per_launch": bwd_main_flops,
         "ms_per_launch": ms_bwd_kernel,
-        "traffic": args.traffic_bytes if args.traffic_bytes else None,
+        "traffic": args.traffic_bytes if args.traffic_bytes else MEASURED_TRAFFIC.get(w.name),
     }
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
