@@ -10,6 +10,7 @@
 #include "fa.h"
 #include "fa_bwd.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_persistent.cuh"
 
 // Device error word: kernels that abandon a bounded wait record it here.
 __device__ int g_fa_err = 0;
@@ -186,6 +187,41 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// Two query tiles per item (d = 64, 128): one persistent CTA per SM walks the
+// item list.  d = 256: one CTA per 128-row query tile.
+#ifndef FA_FWD_PERSISTENT
+#define FA_FWD_PERSISTENT 1
+#endif
+
+template <int D, bool CAUSAL>
+fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                                const fa::FwdParams& fp, int B, int Hq, int sms, cudaStream_t stream) {
+  using C = fa::FwdPCfg<D>;
+  auto kern = fa::fa_fwd_persistent_kernel<D, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  if (!reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
+  fa::FwdPParams p;
+  p.o = fp.o;
+  p.lse = fp.lse;
+  p.N = fp.N;
+  p.Hq = fp.Hq;
+  p.G = fp.G;
+  p.n_qtiles = fp.n_qtiles;
+  p.n_units = (fp.n_qtiles + 1) / 2;
+  p.BH = B * Hq;
+  const long long items = (long long)p.n_units * p.BH;
+  if (items >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  p.n_items = (int)items;
+  p.scale_log2 = fp.scale_log2;
+  p.wait_cap = fp.wait_cap;
+  p.err = fp.err;
+  const int grid = p.n_items < sms ? p.n_items : sms;
+  ProfileScope prof(stream);
+  kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D, bool CAUSAL>
 fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
@@ -355,8 +391,17 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.err = di->err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   switch (d) {
+#if FA_FWD_PERSISTENT
+    case 64:
+      return causal ? launch_fwd_persistent<64, true>(tq, tk, tv, p, B, Hq, di->sms, s)
+                    : launch_fwd_persistent<64, false>(tq, tk, tv, p, B, Hq, di->sms, s);
+    case 128:
+      return causal ? launch_fwd_persistent<128, true>(tq, tk, tv, p, B, Hq, di->sms, s)
+                    : launch_fwd_persistent<128, false>(tq, tk, tv, p, B, Hq, di->sms, s);
+#else
     case 64: return causal ? launch_fwd<64, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<64, false>(tq, tk, tv, p, B, Hq, s);
     case 128: return causal ? launch_fwd<128, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<128, false>(tq, tk, tv, p, B, Hq, s);
+#endif
     case 256: return causal ? launch_fwd<256, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<256, false>(tq, tk, tv, p, B, Hq, s);
   }
   return FA_ERR_UNSUPPORTED;
