@@ -6,6 +6,7 @@
 #include <cmath>
 #include <cstdint>
 #include <mutex>
+#include <type_traits>
 
 #include "fa.h"
 #include "fa_bwd.cuh"
@@ -136,6 +137,9 @@ Range span(const void* p, size_t bytes) {
 }
 bool overlap(Range a, Range b) { return a.lo < b.hi && b.lo < a.hi; }
 
+// N rounded up to a whole number of 128-row tiles.
+long long pad128(long long n) { return (n + 127) / 128 * 128; }
+
 // Size checks shared by both passes.  Returns FA_OK, or the status to report;
 // sets *empty for a problem with nothing to compute.
 fa_status check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* empty) {
@@ -148,9 +152,8 @@ fa_status check_sizes(int B, int Hq, int Hkv, int N, int d, float scale, bool* e
     *empty = true;
     return FA_OK;
   }
-  if (N % 128 != 0) return FA_ERR_UNSUPPORTED;
   if (B > 65535 || Hq > 65535 || Hkv > 65535) return FA_ERR_UNSUPPORTED;
-  if ((long long)B * Hq * N >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * pad128(N) >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
   return FA_OK;
 }
 
@@ -171,11 +174,11 @@ bool reg_split_fits(Kern kern) {
   return r >= C::MIN_LAUNCH_REGS && r <= C::MAX_LAUNCH_REGS;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool TAIL>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
                      int B, int Hq, cudaStream_t stream) {
   using C = fa::FwdCfg<D>;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, TAIL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
   if (C::REG_SPLIT) {
@@ -193,11 +196,11 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 #define FA_FWD_PERSISTENT 1
 #endif
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool TAIL>
 fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const fa::FwdParams& fp, int B, int Hq, int sms, cudaStream_t stream) {
   using C = fa::FwdPCfg<D>;
-  auto kern = fa::fa_fwd_persistent_kernel<D, CAUSAL>;
+  auto kern = fa::fa_fwd_persistent_kernel<D, CAUSAL, TAIL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
   if (!reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
@@ -222,17 +225,17 @@ fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, co
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-template <int D, bool CAUSAL>
+template <int D, bool CAUSAL, bool TAIL>
 fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                           const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
   using C = fa::BwdCfg<D>;
-  auto kern = fa::fa_bwd_kernel<D, CAUSAL>;
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL, TAIL>;
   if (C::REG_SPLIT && !reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
   CUtensorMap tdq;
-  if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.N, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
+  if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.Np, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
-  dim3 grid((p.N / C::BC) * C::NDH, Hkv, B);
+  dim3 grid(((p.N + C::BC - 1) / C::BC) * C::NDH, Hkv, B);
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -240,17 +243,17 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 
 template <int D>
 fa_status launch_bwd_pre(const void* o, const void* dout, const float* lse, float* dvec, float* lse2, float* dqacc,
-                         long long rows, int sms, cudaStream_t stream) {
-  const long long dq_vec4 = rows * D / 4;
-  long long want = rows * (D / 8);
+                         int N, int Np, long long rows_p, int sms, cudaStream_t stream) {
+  const long long dq_vec4 = rows_p * D / 4;
+  long long want = rows_p * (D / 8);
   if (dq_vec4 > want) want = dq_vec4;
   long long blocks = (want + 255) / 256;
   const long long cap = (long long)sms * 8;
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   fa::fa_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc, rows,
-      dq_vec4);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc, N, Np,
+      rows_p, dq_vec4);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -351,8 +354,8 @@ fa_status fa_set_wait_cap(long long cycles) {
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   bool empty = false;
   if (check_sizes(B, Hq, Hkv, N, d, 1.f, &empty) != FA_OK) return 0;
-  const size_t rows = (size_t)B * Hq * N;
-  return 2 * round256(rows * 4) + round256(rows * (size_t)d * 4);
+  const size_t rows_p = (size_t)B * Hq * pad128(N);  // per-head stride N rounded up to 128
+  return 2 * round256(rows_p * 4) + round256(rows_p * (size_t)d * 4);
 }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
@@ -385,24 +388,31 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
-  p.n_qtiles = N / 128;
+  p.n_qtiles = (N + 127) / 128;
   p.scale_log2 = scale * fa::kLog2e;
   p.wait_cap = g_wait_cap;
   p.err = di->err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tail = (N % 128) != 0;
+  // one kernel instance per (d, causal, ragged tail)
+  auto dispatch = [&](auto dtag) -> fa_status {
+    constexpr int D = decltype(dtag)::value;
+    constexpr bool kPersistent = FA_FWD_PERSISTENT && D <= 128;
+    if constexpr (kPersistent) {
+      if (causal) return tail ? launch_fwd_persistent<D, true, true>(tq, tk, tv, p, B, Hq, di->sms, s)
+                              : launch_fwd_persistent<D, true, false>(tq, tk, tv, p, B, Hq, di->sms, s);
+      return tail ? launch_fwd_persistent<D, false, true>(tq, tk, tv, p, B, Hq, di->sms, s)
+                  : launch_fwd_persistent<D, false, false>(tq, tk, tv, p, B, Hq, di->sms, s);
+    } else {
+      if (causal) return tail ? launch_fwd<D, true, true>(tq, tk, tv, p, B, Hq, s)
+                              : launch_fwd<D, true, false>(tq, tk, tv, p, B, Hq, s);
+      return tail ? launch_fwd<D, false, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<D, false, false>(tq, tk, tv, p, B, Hq, s);
+    }
+  };
   switch (d) {
-#if FA_FWD_PERSISTENT
-    case 64:
-      return causal ? launch_fwd_persistent<64, true>(tq, tk, tv, p, B, Hq, di->sms, s)
-                    : launch_fwd_persistent<64, false>(tq, tk, tv, p, B, Hq, di->sms, s);
-    case 128:
-      return causal ? launch_fwd_persistent<128, true>(tq, tk, tv, p, B, Hq, di->sms, s)
-                    : launch_fwd_persistent<128, false>(tq, tk, tv, p, B, Hq, di->sms, s);
-#else
-    case 64: return causal ? launch_fwd<64, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<64, false>(tq, tk, tv, p, B, Hq, s);
-    case 128: return causal ? launch_fwd<128, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<128, false>(tq, tk, tv, p, B, Hq, s);
-#endif
-    case 256: return causal ? launch_fwd<256, true>(tq, tk, tv, p, B, Hq, s) : launch_fwd<256, false>(tq, tk, tv, p, B, Hq, s);
+    case 64: return dispatch(std::integral_constant<int, 64>{});
+    case 128: return dispatch(std::integral_constant<int, 128>{});
+    case 256: return dispatch(std::integral_constant<int, 256>{});
   }
   return FA_ERR_UNSUPPORTED;
 }
@@ -435,16 +445,19 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   st = current_device(&di);
   if (st != FA_OK) return st;
 
+  // workspace: D, lse2 (B·Hq·Np fp32 each) and the dQ accumulator (B·Hq·Np·d fp32)
+  const int Np = (int)pad128(N);
+  const size_t rows_p = (size_t)B * Hq * Np;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dvec = reinterpret_cast<float*>(ws);
-  float* lse2 = reinterpret_cast<float*>(ws + round256(rows * 4));
-  float* dqacc = reinterpret_cast<float*>(ws + 2 * round256(rows * 4));
+  float* lse2 = reinterpret_cast<float*>(ws + round256(rows_p * 4));
+  float* dqacc = reinterpret_cast<float*>(ws + 2 * round256(rows_p * 4));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   switch (d) {
-    case 64: st = launch_bwd_pre<64>(o, dout, lse, dvec, lse2, dqacc, (long long)rows, di->sms, s); break;
-    case 128: st = launch_bwd_pre<128>(o, dout, lse, dvec, lse2, dqacc, (long long)rows, di->sms, s); break;
-    default: st = launch_bwd_pre<256>(o, dout, lse, dvec, lse2, dqacc, (long long)rows, di->sms, s); break;
+    case 64: st = launch_bwd_pre<64>(o, dout, lse, dvec, lse2, dqacc, N, Np, (long long)rows_p, di->sms, s); break;
+    case 128: st = launch_bwd_pre<128>(o, dout, lse, dvec, lse2, dqacc, N, Np, (long long)rows_p, di->sms, s); break;
+    default: st = launch_bwd_pre<256>(o, dout, lse, dvec, lse2, dqacc, N, Np, (long long)rows_p, di->sms, s); break;
   }
   if (st != FA_OK) return st;
 
@@ -460,6 +473,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.dk = static_cast<__nv_bfloat16*>(dk);
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.N = N;
+  p.Np = Np;
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;
@@ -467,17 +481,29 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.scale_log2 = scale * fa::kLog2e;
   p.wait_cap = g_wait_cap;
   p.err = di->err;
+  const bool tail = (N % 128) != 0;
+  auto main_kernel = [&](auto dtag) -> fa_status {
+    constexpr int D = decltype(dtag)::value;
+    if (causal) return tail ? launch_bwd_main<D, true, true>(tq, tk, tv, tdo, p, B, Hkv, s)
+                            : launch_bwd_main<D, true, false>(tq, tk, tv, tdo, p, B, Hkv, s);
+    return tail ? launch_bwd_main<D, false, true>(tq, tk, tv, tdo, p, B, Hkv, s)
+                : launch_bwd_main<D, false, false>(tq, tk, tv, tdo, p, B, Hkv, s);
+  };
   switch (d) {
-    case 64: st = causal ? launch_bwd_main<64, true>(tq, tk, tv, tdo, p, B, Hkv, s) : launch_bwd_main<64, false>(tq, tk, tv, tdo, p, B, Hkv, s); break;
-    case 128: st = causal ? launch_bwd_main<128, true>(tq, tk, tv, tdo, p, B, Hkv, s) : launch_bwd_main<128, false>(tq, tk, tv, tdo, p, B, Hkv, s); break;
-    default: st = causal ? launch_bwd_main<256, true>(tq, tk, tv, tdo, p, B, Hkv, s) : launch_bwd_main<256, false>(tq, tk, tv, tdo, p, B, Hkv, s); break;
+    case 64: st = main_kernel(std::integral_constant<int, 64>{}); break;
+    case 128: st = main_kernel(std::integral_constant<int, 128>{}); break;
+    default: st = main_kernel(std::integral_constant<int, 256>{}); break;
   }
   if (st != FA_OK) return st;
 
-  const long long n_vec4 = (long long)rows * d / 4;
-  long long blocks = (n_vec4 + 255) / 256;
-  if (blocks > (long long)di->sms * 8) blocks = (long long)di->sms * 8;
-  fa::fa_dq_convert_kernel<<<(unsigned)blocks, 256, 0, s>>>(dqacc, static_cast<__nv_bfloat16*>(dq), scale, n_vec4);
+  long long blocks = ((long long)rows + 7) / 8;  // 8 warps (rows) per block
+  if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+  __nv_bfloat16* dq16 = static_cast<__nv_bfloat16*>(dq);
+  switch (d) {
+    case 64: fa::fa_dq_convert_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(dqacc, dq16, scale, rows, N, Np); break;
+    case 128: fa::fa_dq_convert_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(dqacc, dq16, scale, rows, N, Np); break;
+    default: fa::fa_dq_convert_kernel<256><<<(unsigned)blocks, 256, 0, s>>>(dqacc, dq16, scale, rows, N, Np); break;
+  }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 

@@ -94,14 +94,20 @@ struct BwdCfg {
 };
 
 // ------------------------------------------------------------ preprocess
-// One group of D/8 threads per row: D_i = Σ_c dO_ic·O_ic in fp32, and
-// lse2_i = LSE_i·log2e.  Also zeroes the fp32 dQ accumulator.
+// The per-row workspace arrays (D, lse2 and the fp32 dQ accumulator) use a
+// per-head row stride Np = N rounded up to 128, so every 64-row step starts on
+// a 256-byte boundary and rows N..Np-1 of a head are padding that no other
+// head shares.
+//
+// One group of D/8 threads per padded row: D_i = Σ_c dO_ic·O_ic in fp32 and
+// lse2_i = LSE_i·log2e for i < N, zero for the padding rows.  Also zeroes
+// the fp32 dQ accumulator.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          const float* __restrict__ lse, float* __restrict__ dvec,
                                                          float* __restrict__ lse2, float* __restrict__ dqacc,
-                                                         long long rows, long long dq_vec4) {
+                                                         int N, int Np, long long rows_p, long long dq_vec4) {
   constexpr int TPR = D / 8;
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
@@ -112,10 +118,14 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
   const long long groups = nthreads / TPR;
   const long long gid = tid / TPR;
   const int sub = (int)(tid % TPR);
-  for (long long r0 = 0; r0 < rows; r0 += groups) {
-    const long long r = r0 + gid;
+  for (long long r0 = 0; r0 < rows_p; r0 += groups) {
+    const long long rp = r0 + gid;             // padded row (< 2^31, checked on the host)
+    const unsigned head = (unsigned)rp / (unsigned)Np;
+    const int i = (int)((unsigned)rp - head * (unsigned)Np);  // row within the head
+    const bool real = rp < rows_p && gid < groups && i < N;
+    const long long r = (long long)head * N + i;  // row of O, dO, LSE
     float acc = 0.f;
-    if (r < rows && gid < groups) {
+    if (real) {
       const uint4 ov = *reinterpret_cast<const uint4*>(o + r * D + sub * 8);
       const uint4 dv = *reinterpret_cast<const uint4*>(dout + r * D + sub * 8);
       const __nv_bfloat162* o2 = reinterpret_cast<const __nv_bfloat162*>(&ov);
@@ -130,24 +140,36 @@ __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __
     }
 #pragma unroll
     for (int off = TPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-    if (r < rows && gid < groups && sub == 0) {
-      dvec[r] = acc;
-      lse2[r] = lse[r] * kLog2e;
+    if (rp < rows_p && gid < groups && sub == 0) {
+      dvec[rp] = acc;
+      lse2[rp] = real ? lse[r] * kLog2e : 0.f;
     }
   }
 }
 
+// dQ = bf16(s · accumulator), from the padded accumulator rows to the dense
+// [B, Hq, N, d] output: one warp per row, lane = group of 4 columns.
+template <int D>
 __global__ void __launch_bounds__(256) fa_dq_convert_kernel(const float* __restrict__ dqacc,
                                                             __nv_bfloat16* __restrict__ dq, float scale,
-                                                            long long n_vec4) {
-  const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
-  const long long nthreads = (long long)gridDim.x * blockDim.x;
-  for (long long i = tid; i < n_vec4; i += nthreads) {
-    const float4 a = reinterpret_cast<const float4*>(dqacc)[i];
-    uint2 w;
-    w.x = pack_bf16(a.x * scale, a.y * scale);
-    w.y = pack_bf16(a.z * scale, a.w * scale);
-    reinterpret_cast<uint2*>(dq)[i] = w;
+                                                            long long rows, int N, int Np) {
+  constexpr int V4 = D / 4;
+  const long long warp0 = ((long long)blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  const long long nwarps = ((long long)gridDim.x * blockDim.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  for (long long r = warp0; r < rows; r += nwarps) {
+    const unsigned head = (unsigned)r / (unsigned)N;  // r < 2^31 (checked on the host)
+    const long long rp = r + (long long)head * (Np - N);
+    const float4* src = reinterpret_cast<const float4*>(dqacc) + rp * V4;
+    uint2* dst = reinterpret_cast<uint2*>(dq) + r * V4;
+#pragma unroll
+    for (int c = lane; c < V4; c += 32) {
+      const float4 a = src[c];
+      uint2 w;
+      w.x = pack_bf16(a.x * scale, a.y * scale);
+      w.y = pack_bf16(a.z * scale, a.w * scale);
+      dst[c] = w;
+    }
   }
 }
 
@@ -157,13 +179,15 @@ struct BwdParams {
   float* dqacc;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  int N, Hq, Hkv, G;
+  int N, Np, Hq, Hkv, G;  // Np: per-head row stride of lse2, dvec and dqacc
   float scale, scale_log2;
   long long wait_cap;
   int* err;
 };
 
-template <int D, bool CAUSAL>
+// TAIL: N is not a multiple of 128 (keys and queries past N get P = 0, rows past
+// N are not stored).
+template <int D, bool CAUSAL, bool TAIL>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
@@ -182,7 +206,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const int dh = blockIdx.x % C::NDH;  // output column half
   const int hkv = blockIdx.y;
   const int b = blockIdx.z;
-  const int nqt = p.N / C::BR;
+  const int nqt = (p.N + C::BR - 1) / C::BR;
   const int i_start = CAUSAL ? (jt * C::BC) / C::BR : 0;
   const int per_head = nqt - i_start;
   const int n = p.G * per_head;  // steps
@@ -240,6 +264,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int st = s % C::NSTAGE;
         if (!mbar_wait(BAR(C::B_QEMPTY + st), ((s / C::NSTAGE) & 1) ^ 1, wc, 11)) break;
         const int q_row = (b * p.Hq + step_head(s)) * p.N + step_q0(s);
+        const int q_row_p = (b * p.Hq + step_head(s)) * p.Np + step_q0(s);
         const uint32_t bar = BAR(C::B_QFULL + st);
         mbar_expect_tx(bar, 2 * C::Q_BYTES + 512);
 #pragma unroll
@@ -247,8 +272,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tma_load_2d(sbase + C::Q_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmQ, bar, pn * 64, q_row);
           tma_load_2d(sbase + C::DO_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmDO, bar, pn * 64, q_row);
         }
-        bulk_load(sbase + C::LS_OFF + st * 512, p.lse2 + q_row, 256, bar);
-        bulk_load(sbase + C::LS_OFF + st * 512 + 256, p.dvec + q_row, 256, bar);
+        bulk_load(sbase + C::LS_OFF + st * 512, p.lse2 + q_row_p, 256, bar);
+        bulk_load(sbase + C::LS_OFF + st * 512 + 256, p.dvec + q_row_p, 256, bar);
       }
     }
   } else if (warp == 1) {
@@ -378,6 +403,12 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int c = 0; c < 64; ++c)
           if (key > q0 + c) pr[c] = 0.f;
       }
+      // ragged N: keys and queries past the end of the sequence contribute nothing
+      if (TAIL && (key >= p.N || q0 + C::BR > p.N)) {
+#pragma unroll
+        for (int c = 0; c < 64; ++c)
+          if (key >= p.N || q0 + c >= p.N) pr[c] = 0.f;
+      }
       uint32_t pk[32];
 #pragma unroll
       for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
@@ -422,6 +453,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       if (lane == 0) mbar_arrive(BAR(C::B_DSFULL));
     }
     // dK epilogue (scaled by s)
+    // (tcgen05.ld is warp-collective: every lane loads, only rows < N are stored)
     if (ok && mbar_wait_warp(BAR(C::B_ACC), 0, wc, 25)) {
       tc_fence_after();
       __nv_bfloat16* dst = p.dk + ((size_t)(b * p.Hkv + hkv) * p.N + key) * D + dh * C::DH;
@@ -436,8 +468,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int c = 0; c < 16; ++c)
           w[c] = pack_bf16(__uint_as_float(v[2 * c]) * p.scale, __uint_as_float(v[2 * c + 1]) * p.scale);
         uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
+        if (!TAIL || key < p.N) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        }
       }
     }
     tc_fence_before();
@@ -464,7 +498,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tc_fence_before();
       __syncwarp();
       if (lane == 0) mbar_arrive(BAR(C::B_DQEMPTY));
-      const int q_row = (b * p.Hq + step_head(s)) * p.N + step_q0(s);
+      const int q_row = (b * p.Hq + step_head(s)) * p.Np + step_q0(s);  // padded accumulator row
 #pragma unroll
       for (int sub = 0; sub < 64 / C::STG_ROWS; ++sub) {
         // the previous reduce must have finished reading the staging tile
@@ -505,8 +539,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) w[c] = pack_bf16(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
         uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
+        if (!TAIL || jt * C::BC + r < p.N) {
 #pragma unroll
-        for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+        }
       }
     }
     tc_fence_before();

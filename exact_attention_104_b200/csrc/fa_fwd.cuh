@@ -137,7 +137,8 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
   return fmaxf(fmax3(acc[0], acc[1], acc[2]), fmax3(acc[3], acc[4], fmax3(acc[5], acc[6], acc[7])));
 }
 
-template <int D, bool CAUSAL>
+// TAIL: N is not a multiple of 128 (keys past N masked, rows past N not stored).
+template <int D, bool CAUSAL, bool TAIL>
 __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
@@ -435,6 +436,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int c = 0; c < 128; ++c)
             if (c > row) s[c] = -INFINITY;
         }
+        // ragged N: keys past the end of the sequence (the causal mask already
+        // excludes them for every row < N)
+        if (TAIL && !CAUSAL && (j + 1) * C::BN > p.N) {
+          const int lim = p.N - j * C::BN;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) s[c] = -INFINITY;
+        }
         const float mx = row_max128(s);
         const float m_new = fmaxf(m_ref, mx * sl2);
         // conditional rescale: keep the stale reference max unless the row max
@@ -546,12 +555,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int c = 0; c < 16; ++c)
             w[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
+          if (!TAIL || q_row < p.N) {  // rows past a ragged end are computed, not stored
 #pragma unroll
-          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+            for (int c = 0; c < 4; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
+          }
         }
         float lg;
         asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-        p.lse[(size_t)(b * p.Hq + h) * p.N + q_row] = (m_ref + lg) * kLn2;
+        if (!TAIL || q_row < p.N) p.lse[(size_t)(b * p.Hq + h) * p.N + q_row] = (m_ref + lg) * kLn2;
       }
       tc_fence_before();
     }

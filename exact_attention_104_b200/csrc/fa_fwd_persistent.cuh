@@ -63,6 +63,11 @@ struct FwdPCfg {
   static constexpr bool REG_SPLIT = true;
   static constexpr int MIN_LAUNCH_REGS = (128 * CTRL_REGS + 256 * SOFTMAX_REGS + THREADS - 1) / THREADS;
   static constexpr int MAX_LAUNCH_REGS = SOFTMAX_REGS;
+  // Exponentials moved from the MUFU to the FMA pipes (exp2_poly): the second
+  // one of every kPolyPairs-th column pair, 1/8 of them at d = 64, where the
+  // MUFU rather than the tensor pipe bounds a tile (+3 % measured); none at
+  // d = 128, where every fraction tried (1/8, 1/4, 1/2) was slower.
+  static constexpr int kPolyPairs = (D == 64) ? 4 : 0;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL + 2 * D <= TMEM_COLS, "TMEM budget");
 };
@@ -119,7 +124,8 @@ __device__ __forceinline__ int fwd_item_index(int k, int c, int G) {
   return k * G + ((CAUSAL && (k & 1)) ? (G - 1 - c) : c);
 }
 
-template <int D, bool CAUSAL>
+// TAIL: N is not a multiple of 128 (keys past N masked, rows past N not stored).
+template <int D, bool CAUSAL, bool TAIL>
 __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
     fa_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const FwdPParams p) {
@@ -371,10 +377,19 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
           s[64 + c] = __uint_as_float(r2[c]);
           s[96 + c] = __uint_as_float(r3[c]);
         }
-        if (CAUSAL && w.kv_block(w.first(t) + j) == qt) {
+        const int kb = w.kv_block(w.first(t) + j);
+        if (CAUSAL && kb == qt) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > row) s[c] = -INFINITY;
+        }
+        // ragged N: keys past the end of the sequence (the causal mask already
+        // excludes them for every row < N)
+        if (TAIL && !CAUSAL && (kb + 1) * C::BN > p.N) {
+          const int lim = p.N - kb * C::BN;
+#pragma unroll
+          for (int c = 0; c < 128; ++c)
+            if (c >= lim) s[c] = -INFINITY;
         }
         const float mx = row_max128(s);
         const float m_new = fmaxf(m_ref, mx * sl2);
@@ -401,7 +416,9 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
             f2_split(f2_fma(f2_make(s[base + 2 * c], s[base + 2 * c + 1]), f2_make(sl2, sl2), f2_make(neg_m, neg_m)),
                      x0, x1);
             const float a0 = ex2(x0);
-            const float a1 = ex2(x1);
+            // every kPolyPairs-th pair's second exponential on the FMA pipes
+            const float a1 = (C::kPolyPairs > 0 && c % (C::kPolyPairs > 0 ? C::kPolyPairs : 1) == 0) ? exp2_poly(x1)
+                                                                                                   : ex2(x1);
             rs2[c & 1] = f2_add(rs2[c & 1], f2_make(a0, a1));
             pk[c] = pack_bf16(a0, a1);
           }
@@ -465,12 +482,14 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         for (int c = 0; c < 16; ++c)
           wv[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
         uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
+        if (!TAIL || q_row < p.N) {  // rows past a ragged end are computed, not stored
 #pragma unroll
-        for (int c = 0; c < 4; ++c) dst[c] = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+          for (int c = 0; c < 4; ++c) dst[c] = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
+        }
       }
       float lg;
       asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-      p.lse[(size_t)(w.b * p.Hq + w.h) * p.N + q_row] = (m_ref + lg) * kLn2;
+      if (!TAIL || q_row < p.N) p.lse[(size_t)(w.b * p.Hq + w.h) * p.N + q_row] = (m_ref + lg) * kLn2;
       done += n;
     }
     tc_fence_before();

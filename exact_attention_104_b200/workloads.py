@@ -59,6 +59,14 @@ WORKLOADS = {
     "long_b1_h16_n16384_d128_causal": Workload("long_b1_h16_n16384_d128_causal", 1, 16, 16, 16384, 128, True, 1.0, 1002),
     "gqa_b4_hq32_hkv8_n4096_d128_causal": Workload("gqa_b4_hq32_hkv8_n4096_d128_causal", 4, 32, 8, 4096, 128, True, 1.0, 1003),
     "wide_b2_h8_n8192_d256_bigqk": Workload("wide_b2_h8_n8192_d256_bigqk", 2, 8, 8, 8192, 256, False, 3.0, 1004),
+    # head dimension 64: one exponential per 64 multiply-adds instead of 128,
+    # the regime where the exponentials rather than the tensor cores bound
+    # the forward pass
+    "train_b8_h16_n2048_d64": Workload("train_b8_h16_n2048_d64", 8, 16, 16, 2048, 64, False, 1.0, 1005),
+    # N not a multiple of 128: the last query and key tiles of every head are
+    # partial
+    "ragged_b8_h16_n2000_d128_causal": Workload("ragged_b8_h16_n2000_d128_causal", 8, 16, 16, 2000, 128, True, 1.0,
+                                                1006),
 }
 
 BENCH_WORKLOAD = "train_b8_h16_n2048_d128"

@@ -22,6 +22,9 @@
  *   q, o, dout, dq : bf16 [B, Hq,  N, d]
  *   k, v, dk, dv   : bf16 [B, Hkv, N, d]
  *   lse            : fp32 [B, Hq,  N]
+ * N is any positive length.  The kernels work in 128-row tiles; when N is not
+ * a multiple of 128, keys past N are masked out of every row and query rows
+ * past N are neither stored nor given any weight in the gradients.
  *
  * Ownership.  The caller allocates every buffer (device memory) and keeps it
  * alive until the work on `stream` has finished.  The library allocates no
@@ -34,9 +37,9 @@
  *                       multiple of Hkv, non-finite or non-positive scale,
  *                       an output overlapping an input or another output,
  *                       workspace too small;
- *   FA_ERR_UNSUPPORTED  d not in {64, 128, 256}, N not a multiple of 128,
- *                       sizes beyond the index limits (B, Hq ≤ 65535,
- *                       B·Hq·N < 2^31), or no sm_100 device;
+ *   FA_ERR_UNSUPPORTED  d not in {64, 128, 256}, sizes beyond the index
+ *                       limits (B, Hq ≤ 65535, B·Hq·Np < 2^31 with Np = N
+ *                       rounded up to 128), or no sm_100 device;
  *   FA_ERR_CUDA         a CUDA launch or attribute call failed;
  *   FA_ERR_TIMEOUT      (fa_device_status only) a kernel gave up a bounded
  *                       wait and returned early; its outputs are invalid.
@@ -67,9 +70,11 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                  void* stream);
 
-/* Bytes of device workspace fa_bwd needs: two fp32 [B,Hq,N] row vectors
- * (D = rowsum(dO∘O) and LSE·log2 e) and an fp32 [B,Hq,N,d] dQ accumulator,
- * each rounded up to 256 bytes.  Returns 0 for invalid sizes. */
+/* Bytes of device workspace fa_bwd needs: two fp32 [B,Hq,Np] row vectors
+ * (D = rowsum(dO∘O) and LSE·log2 e) and an fp32 [B,Hq,Np,d] dQ accumulator,
+ * each rounded up to 256 bytes, where Np = N rounded up to a multiple of 128
+ * (per-head padding rows keep every tile aligned and private to its head).
+ * Returns 0 for invalid sizes. */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
 /* Backward pass: given q, k, v, the forward outputs o and lse, and the output
@@ -135,8 +140,9 @@ fa_status fa_selftest_exp2(const float* x, float* y, long long n, int use_poly, 
  * exits.  Nothing is allocated or freed per call.
  *
  * Limit: the problem's fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) must not
- * exceed FA_NOALLOC_SCRATCH_BYTES (for d = 128 that is B·Hq·N ≤ 129,055
- * query rows); larger problems return FA_ERR_UNSUPPORTED and enqueue nothing.
+ * exceed FA_NOALLOC_SCRATCH_BYTES (for d = 128 that is B·Hq·Np ≤ 129,055
+ * padded query rows); larger problems return FA_ERR_UNSUPPORTED and enqueue
+ * nothing.
  *
  * Set-up: the first call on each device, with that device current, looks up
  * the array's device address (cudaGetSymbolAddress).  Make that first call

@@ -66,8 +66,10 @@ def compare_sampled(w: Workload, g, units, n_rows=48, seed=0, bwd=True):
     for (b, g_kv) in units:
         kh, vh = f64(g["k"][b, g_kv]), f64(g["v"][b, g_kv])
         heads = list(range(g_kv * w.G, (g_kv + 1) * w.G))
-        # always include the first and last rows of the sequence and of a tile
-        fixed = np.array([r for r in (0, 127, 128, N - 128, N - 1) if 0 <= r < N])
+        # always include the first and last rows of the sequence and of a tile,
+        # and the first row of the last (possibly partial) tile
+        last_tile = (N - 1) // 128 * 128
+        fixed = np.array(sorted({r for r in (0, 127, 128, N - 128, last_tile - 1, last_tile, N - 1) if 0 <= r < N}))
         rows = np.unique(np.concatenate([fixed, rng.choice(N, min(n_rows, N), replace=False)]))
         krows = np.unique(np.concatenate([fixed, rng.choice(N, min(n_rows, N), replace=False)]))
         qh_all = np.stack([f64(g["q"][b, h]) for h in heads])

@@ -45,11 +45,15 @@ def test_status_strings(lib):
 
 
 def test_workspace_bytes_formula(lib):
-    # two fp32 row vectors and an fp32 [B,Hq,N,d] accumulator, each 256-rounded
+    # two fp32 row vectors and an fp32 [B,Hq,Np,d] accumulator, each 256-rounded,
+    # with Np = N rounded up to a multiple of 128 (per-head padding rows)
     B, Hq, Hkv, N, d = 8, 16, 16, 2048, 128
     rows = B * Hq * N
     assert binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) == 2 * rows * 4 + rows * d * 4
     assert binding.fa_bwd_workspace_bytes(1, 1, 1, 128, 64) == 2 * 512 + 128 * 64 * 4
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 100, 64) == 2 * 512 + 128 * 64 * 4
+    assert binding.fa_bwd_workspace_bytes(2, 3, 1, 129, 256) == 2 * 1536 * 4 + 1536 * 256 * 4
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 1, 128) == 2 * 512 + 128 * 128 * 4
     assert binding.fa_bwd_workspace_bytes(1, 3, 2, 128, 64) == 0      # Hq % Hkv != 0
     assert binding.fa_bwd_workspace_bytes(1, 2, 2, 128, 96) == 0      # unsupported d
 
@@ -77,9 +81,9 @@ def _fwd(lib, **kw):
     (dict(scale=float("inf")), binding.FA_ERR_INVALID_ARG),
     (dict(d=96), binding.FA_ERR_UNSUPPORTED),
     (dict(d=0), binding.FA_ERR_INVALID_ARG),
-    (dict(N=200), binding.FA_ERR_UNSUPPORTED),                   # ragged tail
     (dict(B=70000), binding.FA_ERR_UNSUPPORTED),
     (dict(B=1024, Hq=1024, Hkv=1024, N=4096), binding.FA_ERR_UNSUPPORTED),
+    (dict(B=1024, Hq=1024, Hkv=1024, N=1921), binding.FA_ERR_UNSUPPORTED),  # B·Hq·pad128(N) = 2^31
     (dict(o=FAKE), binding.FA_ERR_INVALID_ARG),                  # output aliases q
     (dict(lse=FAKE * 4 + 64), binding.FA_ERR_INVALID_ARG),       # lse overlaps o
     (dict(B=0, q=0, k=0, v=0, o=0, lse=0), binding.FA_OK),       # empty problem: nothing to do
@@ -107,7 +111,7 @@ def _bwd(lib, **kw):
     (dict(ws=FAKE * 9), binding.FA_ERR_INVALID_ARG),             # workspace aliases dv
     (dict(Hq=4, Hkv=3), binding.FA_ERR_INVALID_ARG),
     (dict(d=32), binding.FA_ERR_UNSUPPORTED),
-    (dict(N=130), binding.FA_ERR_UNSUPPORTED),
+    (dict(B=1024, Hq=1024, Hkv=1024, N=2047), binding.FA_ERR_UNSUPPORTED),  # padded rows reach 2^31
     (dict(B=0), binding.FA_OK),
 ])
 def test_bwd_argument_validation(lib, kw, expect):

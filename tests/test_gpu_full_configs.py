@@ -1,5 +1,6 @@
 """GPU parity at the full sizes of the five reference workloads (C2 in both
-masking modes), in the launch configuration bench.py times.  The oracle
+masking modes), plus the d = 64 and ragged-length workloads, in the launch
+configuration bench.py times.  The oracle
 computes sampled outputs one head at a time: O and LSE for sampled query rows,
 dQ for the same rows and dK, dV for sampled key rows (every query row
 contributes to those, so the oracle computes the full probability columns)."""
@@ -19,6 +20,8 @@ UNITS = {
     "long_b1_h16_n16384_d128_causal": [(0, 9)],
     "gqa_b4_hq32_hkv8_n4096_d128_causal": [(3, 7)],
     "wide_b2_h8_n8192_d256_bigqk": [(1, 5)],
+    "train_b8_h16_n2048_d64": [(2, 11)],
+    "ragged_b8_h16_n2000_d128_causal": [(0, 0), (7, 15)],
 }
 
 

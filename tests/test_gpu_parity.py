@@ -45,6 +45,30 @@ def test_small_shapes_fwd_bwd(w):
     assert_within_tolerance(err)
 
 
+# ragged lengths: N not a multiple of 128 (last query and key tiles partly
+# outside the sequence), down to a single row
+RAGGED = []
+for d in (64, 128, 256):
+    for causal in (False, True):
+        for (B, Hq, Hkv, N) in ((1, 2, 2, 1), (1, 2, 2, 77), (2, 2, 1, 129), (1, 4, 2, 200), (1, 2, 2, 383)):
+            RAGGED.append(Workload(f"r_d{d}_{'c' if causal else 'nc'}_{B}_{Hq}_{Hkv}_{N}", B, Hq, Hkv, N, d, causal,
+                                   1.0, 11 + d + N))
+
+
+@pytest.mark.parametrize("w", RAGGED, ids=lambda w: w.name)
+def test_ragged_lengths_fwd_bwd(w):
+    g = run_gpu(w)
+    err = compare_full(w, g)
+    if w.N == 1:
+        # one key: P = 1, so D = dP and dS = P∘(dP − D) is exactly 0, as are dQ
+        # and dK; a relative error against an all-zero reference is undefined,
+        # so the kernel's rounding residue of dP − D is bounded absolutely
+        for name in ("dq", "dk"):
+            assert float(f64(g[name]).__abs__().max()) <= 1e-3, (name, err)
+        err = dict(err, dq=0.0, dk=0.0)
+    assert_within_tolerance(err)
+
+
 @pytest.mark.parametrize("d", [64, 128, 256])
 @pytest.mark.parametrize("causal", [False, True])
 def test_large_logits(d, causal):
@@ -96,10 +120,6 @@ def test_zero_queries_give_uniform_attention(causal):
 
 
 def test_unsupported_and_invalid_are_reported():
-    q = torch.zeros(1, 2, 200, 64, dtype=torch.bfloat16, device="cuda")
-    with pytest.raises(FAError) as e:
-        attention_forward(q, q.clone(), q.clone())
-    assert e.value.status == binding.FA_ERR_UNSUPPORTED
     q = torch.zeros(1, 2, 128, 96, dtype=torch.bfloat16, device="cuda")
     with pytest.raises(FAError) as e:
         attention_forward(q, q.clone(), q.clone())
