@@ -235,7 +235,9 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
   if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.Np, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
-  dim3 grid(((p.N + C::BC - 1) / C::BC) * C::NDH, Hkv, B);
+  const long long units = (long long)((p.N + C::BC - 1) / C::BC) * C::NDH * Hkv * B;
+  if (units >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  const dim3 grid((unsigned)units);
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -474,6 +476,19 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.dv = static_cast<__nv_bfloat16*>(dv);
   p.N = N;
   p.Np = Np;
+  p.B = B;
+  {
+    // Causal: key tiles in bands, heaviest band first (see fa_bwd_kernel).  More
+    // bands shorten the tail of heavy CTAs dispatched last; fewer keep the
+    // concurrently running CTAs on fewer heads (Q/dO reuse in L2).  The band
+    // count is a rule fitted to measurements (same box, fa_bwd call time):
+    // 128 (b, kv head) units per key tile: 4 bands +3.2 % over head-major;
+    // 32 units: 2 bands +4 %; 16 units (N = 16384): head-major best, 4 bands −4 %.
+    const int n_kt = (N + 127) / 128;
+    const int units = (d == 256 ? 2 : 1) * Hkv * B;
+    const int bands = !causal ? 1 : (units >= 64 ? 4 : (units > 16 ? 2 : 1));
+    p.jt_band = (n_kt + bands - 1) / bands;
+  }
   p.Hq = Hq;
   p.Hkv = Hkv;
   p.G = Hq / Hkv;

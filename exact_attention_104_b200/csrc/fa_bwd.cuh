@@ -179,7 +179,8 @@ struct BwdParams {
   float* dqacc;
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
-  int N, Np, Hq, Hkv, G;  // Np: per-head row stride of lse2, dvec and dqacc
+  int N, Np, B, Hq, Hkv, G;  // Np: per-head row stride of lse2, dvec and dqacc
+  int jt_band;               // key tiles per scheduling band (see fa_bwd_kernel)
   float scale, scale_log2;
   long long wait_cap;
   int* err;
@@ -202,10 +203,23 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int jt = blockIdx.x / C::NDH;  // key tile
-  const int dh = blockIdx.x % C::NDH;  // output column half
-  const int hkv = blockIdx.y;
-  const int b = blockIdx.z;
+  // Work unit of this CTA (one 1-D grid).  Key tiles are taken in bands of
+  // p.jt_band, earliest band first; inside a band the units go head by head,
+  // so that the key tiles of one head that run at the same time stream the
+  // same Q/dO tiles through L2.  Causal: earlier key tiles have more query
+  // steps, so heavy bands run first and the last CTAs dispatched are light
+  // (no long tail).  Non-causal: one band (plain head-major order).
+  const int n_kt = (p.N + C::BC - 1) / C::BC;
+  const int U = C::NDH * p.Hkv * p.B;  // units per key tile
+  const int bi = (int)(blockIdx.x / ((unsigned)p.jt_band * U));
+  const int wb = min(p.jt_band, n_kt - bi * p.jt_band);  // key tiles in this band
+  const int rb = (int)(blockIdx.x - (unsigned)bi * p.jt_band * U);
+  const int bh = rb / (wb * C::NDH);
+  const int rem = rb - bh * (wb * C::NDH);
+  const int jt = bi * p.jt_band + rem / C::NDH;  // key tile
+  const int dh = rem % C::NDH;                   // output column half
+  const int hkv = bh % p.Hkv;
+  const int b = bh / p.Hkv;
   const int nqt = (p.N + C::BR - 1) / C::BR;
   const int i_start = CAUSAL ? (jt * C::BC) / C::BR : 0;
   const int per_head = nqt - i_start;
