@@ -181,9 +181,6 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, TAIL>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
-  if (C::REG_SPLIT) {
-    if (!reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
-  }
   dim3 grid((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
@@ -191,11 +188,7 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 }
 
 // Two query tiles per item (d = 64, 128): one persistent CTA per SM walks the
-// item list.  d = 256: one CTA per 128-row query tile.
-#ifndef FA_FWD_PERSISTENT
-#define FA_FWD_PERSISTENT 1
-#endif
-
+// item list.  d = 256: one CTA per 128-row query tile (launch_fwd).
 template <int D, bool CAUSAL, bool TAIL>
 fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const fa::FwdParams& fp, int B, int Hq, int sms, cudaStream_t stream) {
@@ -399,8 +392,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   // one kernel instance per (d, causal, ragged tail)
   auto dispatch = [&](auto dtag) -> fa_status {
     constexpr int D = decltype(dtag)::value;
-    constexpr bool kPersistent = FA_FWD_PERSISTENT && D <= 128;
-    if constexpr (kPersistent) {
+    if constexpr (D <= 128) {
       if (causal) return tail ? launch_fwd_persistent<D, true, true>(tq, tk, tv, p, B, Hq, di->sms, s)
                               : launch_fwd_persistent<D, true, false>(tq, tk, tv, p, B, Hq, di->sms, s);
       return tail ? launch_fwd_persistent<D, false, true>(tq, tk, tv, p, B, Hq, di->sms, s)

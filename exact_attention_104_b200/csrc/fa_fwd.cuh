@@ -8,10 +8,13 @@
 // concept page, "Core idea" (tile into on-chip memory, write only O and a few
 // per-row statistics).
 //
-// One CTA owns NQ query tiles of 128 rows of one (batch, head):
-//   warp 0        TMA producer: Q tiles once, then K/V chunks through a ring
-//   warp 1        MMA issuer (one thread) + TMEM owner
-//   warps 4..     one softmax warpgroup per query tile; thread = query row
+// FwdCfg holds the tile shapes shared with the persistent kernel
+// (fa_fwd_persistent.cuh), which handles d = 64 and 128 with two query tiles
+// per work item.  fa_fwd_kernel below is the d = 256 kernel: one CTA owns one
+// 128-row query tile of one (batch, head):
+//   warp 0        TMA producer: the Q tile once, then K/V chunks through a ring
+//   warp 1        MMA issuer + TMEM owner
+//   warps 4-7     softmax warpgroup; thread = query row
 // S = Q Kᵀ and O += P V both run on tcgen05 with fp32 accumulators in TMEM.
 // P (bf16) is written back over the first half of its S columns and read by
 // the PV MMA directly from TMEM.  The O rescale is conditional: a row keeps a
@@ -24,22 +27,6 @@
 namespace fa {
 
 constexpr float kRescaleTau = 8.0f;
-constexpr int kPrefetchUnits = 0;  // K/V tiles prefetched into L2 ahead of their load
-
-// Softmax tuning knobs (all variants compute the same P up to rounding):
-//   FA_POLY_PAIRS  n > 0: the second exponential of every n-th column pair runs
-//                  on the FMA pipes (exp2_poly); 0 keeps every one on the MUFU
-//   FA_SPLIT_P     hand P to the MMA warp in two 64-key halves
-//   FA_PACKED_F32  scale/shift and row sums with packed fp32x2 instructions
-#ifndef FA_POLY_PAIRS
-#define FA_POLY_PAIRS 0
-#endif
-#ifndef FA_SPLIT_P
-#define FA_SPLIT_P 1
-#endif
-#ifndef FA_PACKED_F32
-#define FA_PACKED_F32 1
-#endif
 
 template <int D>
 struct FwdCfg {
@@ -75,16 +62,6 @@ struct FwdCfg {
   static constexpr uint32_t IDESC_PV = idesc_bf16_f32(128, CH, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL + NQ * D <= TMEM_COLS, "TMEM budget");
-  // Register split with two softmax warpgroups: the control warpgroup gives
-  // registers back (setmaxnreg.dec), the softmax warpgroups take them
-  // (setmaxnreg.inc).  Valid for a launch allocation R with
-  // CTRL_REGS <= R <= SOFTMAX_REGS and 128·CTRL_REGS + 256·SOFTMAX_REGS <= 384·R;
-  // the host checks R against [MIN_LAUNCH_REGS, MAX_LAUNCH_REGS] before launch.
-  static constexpr int CTRL_REGS = 80;
-  static constexpr int SOFTMAX_REGS = 208;
-  static constexpr bool REG_SPLIT = (NQ == 2);
-  static constexpr int MIN_LAUNCH_REGS = (128 * CTRL_REGS + 256 * SOFTMAX_REGS + THREADS - 1) / THREADS;
-  static constexpr int MAX_LAUNCH_REGS = SOFTMAX_REGS;
 };
 
 struct FwdParams {
@@ -96,26 +73,14 @@ struct FwdParams {
   int* err;
 };
 
-// Load-order of K/V tiles ("units"; each unit is NCH chunks).  With two query
-// tiles the MMA warp first uses K(j) then V(j); with one query tile it keeps
-// two S tiles in flight and first uses K(0), K(1), V(0), K(2), V(1), ...
-template <int NQ>
+// Load order of the K/V tiles ("units"; each unit is NCH chunks) of the
+// one-tile kernel: it keeps two S tiles in flight, so the MMA warp first uses
+// K(0), K(1), V(0), K(2), V(1), ..., K(n-1), V(n-2), V(n-1).
 struct KVOrder {
-  __device__ static int unitK(int j, int n) {
-    if (NQ == 2) return 2 * j;
-    return j == 0 ? 0 : 2 * j - 1;
-  }
-  __device__ static int unitV(int j, int n) {
-    if (NQ == 2) return 2 * j + 1;
-    return (j == n - 1) ? 2 * n - 1 : 2 * j + 2;
-  }
+  __device__ static int unitK(int j, int n) { return j == 0 ? 0 : 2 * j - 1; }
+  __device__ static int unitV(int j, int n) { return (j == n - 1) ? 2 * n - 1 : 2 * j + 2; }
   // inverse: unit u -> (is_v, j)
   __device__ static void decode(int u, int n, bool& is_v, int& j) {
-    if (NQ == 2) {
-      is_v = (u & 1);
-      j = u >> 1;
-      return;
-    }
     if (u == 0) { is_v = false; j = 0; }
     else if (u == 2 * n - 1) { is_v = true; j = n - 1; }
     else if (u & 1) { is_v = false; j = (u + 1) >> 1; }
@@ -143,7 +108,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D>;
-  using Ord = KVOrder<C::NQ>;
+  using Ord = KVOrder;
+  static_assert(C::NQ == 1, "one query tile per CTA (d = 64 and 128 use fa_fwd_persistent_kernel)");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -157,15 +123,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   const int b = blockIdx.z;
   const int hkv = h / p.G;
   // causal: heaviest query tiles first so the tail of the grid is short
-  const int unit = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
-  const int qt0 = unit * C::NQ;
-  int n_t[2] = {0, 0};
-#pragma unroll
-  for (int t = 0; t < C::NQ; ++t) {
-    const int qt = qt0 + t;
-    n_t[t] = (qt < p.n_qtiles) ? (CAUSAL ? qt + 1 : p.n_qtiles) : 0;
-  }
-  const int nmax = n_t[0] > n_t[1] ? n_t[0] : n_t[1];
+  const int qt = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+  const int n = CAUSAL ? qt + 1 : p.n_qtiles;  // K/V tiles this query tile sees
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_QFULL), 1);
@@ -195,7 +154,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
-    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
       tma_prefetch_desc(&tmK);
@@ -204,34 +162,16 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const uint64_t pol_q = policy_evict_first();
       const int q_row_base = (b * p.Hq + h) * p.N;
       const int kv_row_base = (b * p.Hkv + hkv) * p.N;
-      int nvalid = 0;
+      mbar_expect_tx(BAR(C::B_QFULL), C::Q_BYTES);
 #pragma unroll
-      for (int t = 0; t < C::NQ; ++t) nvalid += (n_t[t] > 0);
-      mbar_expect_tx(BAR(C::B_QFULL), nvalid * C::Q_BYTES);
-#pragma unroll
-      for (int t = 0; t < C::NQ; ++t) {
-        if (n_t[t] == 0) continue;
-#pragma unroll
-        for (int pn = 0; pn < D / 64; ++pn)
-          tma_load_2d_hint(sbase + C::Q_OFF + t * C::Q_BYTES + pn * C::PANEL, &tmQ, BAR(C::B_QFULL), pn * 64,
-                           q_row_base + (qt0 + t) * C::BM, pol_q);
-      }
-      // L2 prefetch of unit u: a K/V tile in shared memory only one step ahead
-      // would still wait for HBM/L2 latency; the prefetch runs kPrefetchUnits ahead
-      auto prefetch_unit = [&](int u) {
-        bool pv;
-        int pj;
-        Ord::decode(u, nmax, pv, pj);
-#pragma unroll
-        for (int pn = 0; pn < D / 64; ++pn) tma_prefetch_l2_2d(pv ? &tmV : &tmK, pn * 64, kv_row_base + pj * C::BN);
-      };
-      for (int u = 0; u < kPrefetchUnits && u < 2 * nmax; ++u) prefetch_unit(u);
+      for (int pn = 0; pn < D / 64; ++pn)
+        tma_load_2d_hint(sbase + C::Q_OFF + pn * C::PANEL, &tmQ, BAR(C::B_QFULL), pn * 64, q_row_base + qt * C::BM,
+                         pol_q);
       bool ok = true;
-      for (int u = 0; u < 2 * nmax && ok; ++u) {
+      for (int u = 0; u < 2 * n && ok; ++u) {
         bool is_v;
         int j;
-        Ord::decode(u, nmax, is_v, j);
-        if (u + kPrefetchUnits < 2 * nmax) prefetch_unit(u + kPrefetchUnits);
+        Ord::decode(u, n, is_v, j);
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const int seq = u * C::NCH + c;
@@ -249,7 +189,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
   } else if (warp == 1) {
     // ---------------------------------------------------------- MMA issuer
     // (the whole warp runs this role; one elected lane issues each instruction)
-    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     {
       bool ok = mbar_wait_warp(BAR(C::B_QFULL), 0, wc, 2);
       tc_fence_after();
@@ -270,21 +209,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       auto need_k = [&](int j) -> bool {
         if (j <= k_ready) return true;
         k_ready = j;
-        return wait_unit(Ord::unitK(j, nmax));
+        return wait_unit(Ord::unitK(j, n));
       };
       auto need_v = [&](int j) -> bool {
         if (j <= v_ready) return true;
         v_ready = j;
-        return wait_unit(Ord::unitV(j, nmax));
+        return wait_unit(Ord::unitV(j, n));
       };
       // Descriptors are built once; each MMA only adds a compile-time offset.
       const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
       const uint64_t dKV_k = sdesc_sw128(sbase + C::KV_OFF, 16, 1024);
       const uint64_t dKV_mn = sdesc_sw128(sbase + C::KV_OFF, C::PANEL, 1024);
-      // S[scol] = Q_t · K_jᵀ   (M=128 queries, N=128 keys, K=D)
-      auto issue_s = [&](int t, int j, int scol) {
-        const int seq0 = Ord::unitK(j, nmax) * C::NCH;
-        const uint64_t da0 = sdesc_add(dQ_k, t * C::Q_BYTES);
+      // S[scol] = Q · K_jᵀ   (M=128 queries, N=128 keys, K=D)
+      auto issue_s = [&](int j, int scol) {
+        const int seq0 = Ord::unitK(j, n) * C::NCH;
+        const uint64_t da0 = dQ_k;
         uint64_t db0[C::NCH];
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((seq0 + c) % C::NSLOT) * C::SLOT_BYTES);
@@ -296,10 +235,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
                  kk > 0 ? 1u : 0u);
         }
       };
-      // O_t[:, c*CH..] (+)= P(TMEM at scol) · V_j[:, c*CH..]; half 0 covers keys
+      // O[:, c*CH..] (+)= P(TMEM at scol) · V_j[:, c*CH..]; half 0 covers keys
       // 0..63 of the tile, half 1 keys 64..127
       auto issue_pv = [&](int j, int scol, int ocol, int half) {
-        const int seq0 = Ord::unitV(j, nmax) * C::NCH;
+        const int seq0 = Ord::unitV(j, n) * C::NCH;
 #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const uint64_t db0 = sdesc_add(dKV_mn, ((seq0 + c) % C::NSLOT) * C::SLOT_BYTES);
@@ -311,48 +250,18 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       };
 
       if (ok) {
-        if (C::NQ == 2) {
-          for (int t = 0; t < 2 && ok; ++t) {
-            if (n_t[t] == 0) continue;
-            ok = need_k(0);
-            if (!ok) break;
-            issue_s(t, 0, C::S_COL + 128 * t);
-            tc_commit_w(BAR(C::B_SFULL + t));
-          }
-          if (ok) release_unit(Ord::unitK(0, nmax));
-          for (int j = 0; j < nmax && ok; ++j) {
-            for (int t = 0; t < 2; ++t) {
-              if (j >= n_t[t]) continue;
-              if (!mbar_wait_warp(BAR(C::B_PFULL + t), j & 1, wc, 4)) { ok = false; break; }
-              tc_fence_after();
-              if (!need_v(j)) { ok = false; break; }
-              issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D, 0);
-              if (!mbar_wait_warp(BAR(C::B_PFULL2 + t), j & 1, wc, 10)) { ok = false; break; }
-              tc_fence_after();
-              issue_pv(j, C::S_COL + 128 * t, C::O_COL + t * D, 1);
-              tc_commit_w(BAR(C::B_ODONE + t));
-              if (t == 1 || j >= n_t[1]) release_unit(Ord::unitV(j, nmax));  // last reader of V(j)
-              if (j + 1 < n_t[t]) {
-                if (!need_k(j + 1)) { ok = false; break; }
-                issue_s(t, j + 1, C::S_COL + 128 * t);
-                tc_commit_w(BAR(C::B_SFULL + t));
-              }
-            }
-            if (!ok) break;
-            if (j + 1 < nmax) release_unit(Ord::unitK(j + 1, nmax));
-          }
-        } else {
-          const int n = n_t[0];
+        {
+          // two S tiles in flight: S(j+2) is issued as soon as PV(j) has read P(j)
           ok = need_k(0);
           if (ok) {
-            issue_s(0, 0, C::S_COL);
+            issue_s(0, C::S_COL);
             tc_commit_w(BAR(C::B_SFULL + 0));
             release_unit(Ord::unitK(0, n));
           }
           if (ok && n > 1) {
             ok = need_k(1);
             if (ok) {
-              issue_s(0, 1, C::S_COL + 128);
+              issue_s(1, C::S_COL + 128);
               tc_commit_w(BAR(C::B_SFULL + 1));
               release_unit(Ord::unitK(1, n));
             }
@@ -370,7 +279,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             release_unit(Ord::unitV(j, n));
             if (j + 2 < n) {
               if (!need_k(j + 2)) { ok = false; break; }
-              issue_s(0, j + 2, C::S_COL + 128 * x);
+              issue_s(j + 2, C::S_COL + 128 * x);
               tc_commit_w(BAR(C::B_SFULL + x));
               release_unit(Ord::unitK(j + 2, n));
             }
@@ -381,35 +290,26 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tc_commit_w(BAR(C::B_DRAIN));
       mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 8);
     }
-  } else if (warp < 4) {
-    // idle warps of the control warpgroup: hand their registers to the softmax
-    if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
-  } else {
+  } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax
-    if (C::REG_SPLIT) setmaxnreg_inc<C::SOFTMAX_REGS>();
-    const int t = (warp - 4) >> 2;
     const int quarter = warp & 3;
     const int row = quarter * 32 + lane;
-    const int n = n_t[t];
-    if (n > 0) {
-      const int qt = qt0 + t;
+    {
       const int q_row = qt * C::BM + row;
       const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
       const float sl2 = p.scale_log2;
-      const int ocol = C::O_COL + t * D;
+      const int ocol = C::O_COL;
       float m_ref = -INFINITY;
       float l = 0.f;
       bool ok = true;
-      // Completion of PV(j) is signalled on o_done[t] (two query tiles: PV(t, j+1)
-      // cannot start before this warpgroup has seen S(t, j+1), which follows
-      // PV(t, j)) or on o_done[j & 1] (one query tile: S(j+1) is issued before
-      // PV(j), so one barrier could run two phases ahead of a waiter and make
-      // its parity test ambiguous).
-      auto odone_idx = [&](int jj) { return C::NQ == 2 ? t : (jj & 1); };
-      auto odone_par = [&](int jj) -> uint32_t { return C::NQ == 2 ? (jj & 1) : ((jj >> 1) & 1); };
+      // Completion of PV(j) is signalled on o_done[j & 1]: S(j+1) is issued
+      // before PV(j), so a single barrier could run two phases ahead of a
+      // waiter and make its parity test ambiguous.
+      auto odone_idx = [&](int jj) { return jj & 1; };
+      auto odone_par = [&](int jj) -> uint32_t { return (jj >> 1) & 1; };
       for (int j = 0; j < n; ++j) {
-        const int x = (C::NQ == 2) ? t : (j & 1);
-        const uint32_t par = (C::NQ == 2) ? (j & 1) : ((j >> 1) & 1);
+        const int x = j & 1;  // S buffer of K/V tile j
+        const uint32_t par = (j >> 1) & 1;
         const int scol = C::S_COL + 128 * x;
         if (!mbar_wait_warp(BAR(C::B_SFULL + x), par, wc, 5)) { ok = false; break; }
         tc_fence_after();
@@ -462,32 +362,21 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           }
         }
         // P = 2^(s·scale·log2e − m_ref), rounded to bf16 and written over the
-        // first 64 columns of S.  With FA_SPLIT_P, keys 0..63 are handed to the
-        // MMA warp before keys 64..127 are exponentiated, so the first half of
-        // the PV product overlaps the second half of the exponentials.
+        // first 64 columns of S.  Keys 0..63 are handed to the MMA warp before
+        // keys 64..127 are exponentiated, so the first half of the PV product
+        // overlaps the second half of the exponentials.  Scale/shift and row
+        // sums use packed fp32x2 instructions.
         const float neg_m = -m_ref;
         uint64_t rs2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
-        float rs[4] = {0.f, 0.f, 0.f, 0.f};
         auto exp_half = [&](int base, uint32_t (&pk)[32]) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
             float x0, x1;
-            if (FA_PACKED_F32) {
-              f2_split(f2_fma(f2_make(s[base + 2 * c], s[base + 2 * c + 1]), f2_make(sl2, sl2), f2_make(neg_m, neg_m)),
-                       x0, x1);
-            } else {
-              x0 = fmaf(s[base + 2 * c], sl2, neg_m);
-              x1 = fmaf(s[base + 2 * c + 1], sl2, neg_m);
-            }
+            f2_split(f2_fma(f2_make(s[base + 2 * c], s[base + 2 * c + 1]), f2_make(sl2, sl2), f2_make(neg_m, neg_m)),
+                     x0, x1);
             const float a0 = ex2(x0);
-            const float a1 = (FA_POLY_PAIRS > 0 && c % (FA_POLY_PAIRS > 0 ? FA_POLY_PAIRS : 1) == 0) ? exp2_poly(x1)
-                                                                                                     : ex2(x1);
-            if (FA_PACKED_F32) {
-              rs2[c & 1] = f2_add(rs2[c & 1], f2_make(a0, a1));
-            } else {
-              rs[(c & 1) * 2 + 0] += a0;
-              rs[(c & 1) * 2 + 1] += a1;
-            }
+            const float a1 = ex2(x1);
+            rs2[c & 1] = f2_add(rs2[c & 1], f2_make(a0, a1));
             pk[c] = pack_bf16(a0, a1);
           }
         };
@@ -511,12 +400,10 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             }
           }
           tmem_st32(tl + scol, pk);
-          if (FA_SPLIT_P) {
-            tmem_st_wait();
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(BAR(C::B_PFULL + x));
-          }
+          tmem_st_wait();
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(C::B_PFULL + x));
         }
         {
           uint32_t pk[32];
@@ -525,19 +412,12 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
-          if (lane == 0) {
-            if (!FA_SPLIT_P) mbar_arrive(BAR(C::B_PFULL + x));
-            mbar_arrive(BAR(C::B_PFULL2 + x));
-          }
+          if (lane == 0) mbar_arrive(BAR(C::B_PFULL2 + x));
         }
-        if (FA_PACKED_F32) {
-          float a, b2, c2, d2;
-          f2_split(rs2[0], a, b2);
-          f2_split(rs2[1], c2, d2);
-          l += (a + b2) + (c2 + d2);
-        } else {
-          l += (rs[0] + rs[1]) + (rs[2] + rs[3]);
-        }
+        float a, b2, c2, d2;
+        f2_split(rs2[0], a, b2);
+        f2_split(rs2[1], c2, d2);
+        l += (a + b2) + (c2 + d2);
       }
       if (ok) ok = mbar_wait_warp(BAR(C::B_ODONE + odone_idx(n - 1)), odone_par(n - 1), wc, 7);
       if (ok) {
