@@ -58,6 +58,7 @@ __all__ = [
     "attention_backward",
     "head_forward_rows",
     "head_backward_sampled",
+    "attention_forward_suffix",
     "attention_flops",
 ]
 
@@ -293,6 +294,45 @@ def head_backward_sampled(q_heads, kh, vh, do_heads, scale, causal, q_rows, k_ro
             dv_rows += p_cols.T @ doh[rows]
             dk_rows += scale * (ds_cols.T @ qh[rows])
     return dq_rows, dk_rows, dv_rows
+
+
+# ---------------------------------------------------------------------------
+# Fewer queries than keys: the queries are the last positions of the sequence
+# ---------------------------------------------------------------------------
+
+def attention_forward_suffix(q, k, v, scale, causal=False):
+    """Attention of Nq queries against Nk keys when the queries are the last Nq
+    positions of an Nk-long sequence (decoding against cached keys and values).
+
+    The pages define the causal mask for equal lengths only (key j is visible
+    to the query at position i iff j <= i).  Reading used here: query row r
+    sits at position Nk - Nq + r, so key j is masked iff j > Nk - Nq + r; then
+    these rows are exactly the last Nq rows of the square computation over the
+    whole sequence.  Without the mask every query sees all Nk keys.
+
+    q: [B, Hq, Nq, d]; k, v: [B, Hkv, Nk, d] (Nq <= Nk when causal).  Returns
+    O [B, Hq, Nq, d] and LSE [B, Hq, Nq] (natural log), float64."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    G = Hq // Hkv
+    pos = (Nk - Nq) + np.arange(Nq)  # sequence position of each query row
+    o = np.zeros_like(q)
+    lse = np.zeros((B, Hq, Nq))
+    for b in range(B):
+        for h in range(Hq):
+            g = h // G
+            s = scale * (q[b, h] @ k[b, g].T)
+            if causal:
+                s = np.where(np.arange(Nk)[None, :] > pos[:, None], -np.inf, s)
+            m = s.max(axis=1, keepdims=True)
+            e = np.exp(s - m)
+            l = e.sum(axis=1, keepdims=True)
+            o[b, h] = (e / l) @ v[b, g]
+            lse[b, h] = (m + np.log(l))[:, 0]
+    return o, lse
 
 
 def attention_flops(B, Hq, N, d, causal):

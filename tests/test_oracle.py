@@ -296,6 +296,91 @@ def test_flop_count():
 
 
 # ---------------------------------------------------------------------------
+# Fewer queries than keys (decoding): attention_forward_suffix
+# ---------------------------------------------------------------------------
+
+def _suffix_check(fn, causal, Nq, Hq, Hkv, seed):
+    """The last Nq rows of the square computation over the whole sequence."""
+    rng = np.random.default_rng(seed)
+    B, N, d = 2, 13, 5
+    q = rng.standard_normal((B, Hq, N, d))
+    k = rng.standard_normal((B, Hkv, N, d))
+    v = rng.standard_normal((B, Hkv, N, d))
+    o_sq, lse_sq = oracle.attention_forward(q, k, v, 0.6, causal)
+    o, lse = fn(q[:, :, N - Nq:], k, v, 0.6, causal)
+    np.testing.assert_allclose(o, o_sq[:, :, N - Nq:], rtol=0, atol=1e-12)
+    np.testing.assert_allclose(lse, lse_sq[:, :, N - Nq:], rtol=0, atol=1e-12)
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("Nq", [1, 4, 13])
+@pytest.mark.parametrize("Hq,Hkv", [(2, 2), (4, 1)])
+def test_suffix_equals_last_rows_of_square_attention(causal, Nq, Hq, Hkv):
+    _suffix_check(oracle.attention_forward_suffix, causal, Nq, Hq, Hkv, 5 + Nq)
+
+
+def test_suffix_alignment_mistake_is_caught():
+    # a top-left aligned mask (query row r sees keys 0..r) must fail the pin
+    def top_left(q, k, v, scale, causal=False):
+        q = np.asarray(q, np.float64)
+        B, Hq, Nq, d = q.shape
+        Hkv, Nk = k.shape[1], k.shape[2]
+        o = np.zeros_like(q)
+        lse = np.zeros((B, Hq, Nq))
+        for b in range(B):
+            for h in range(Hq):
+                g = h // (Hq // Hkv)
+                sc = scale * (q[b, h] @ k[b, g].T)
+                if causal:
+                    sc = np.where(np.arange(Nk)[None, :] > np.arange(Nq)[:, None], -np.inf, sc)
+                m = sc.max(axis=1, keepdims=True)
+                e = np.exp(sc - m)
+                o[b, h] = e / e.sum(axis=1, keepdims=True) @ v[b, g]
+                lse[b, h] = (m + np.log(e.sum(axis=1, keepdims=True)))[:, 0]
+        return o, lse
+
+    with pytest.raises(AssertionError):
+        _suffix_check(top_left, True, 4, 2, 2, 9)
+
+
+def test_suffix_matches_brute_force_loops():
+    # every visible key enumerated with scalar exp and explicit sums
+    rng = np.random.default_rng(17)
+    Nq, Nk, d = 3, 7, 4
+    q = rng.standard_normal((1, 1, Nq, d))
+    k = rng.standard_normal((1, 1, Nk, d))
+    v = rng.standard_normal((1, 1, Nk, d))
+    for causal in (False, True):
+        o, lse = oracle.attention_forward_suffix(q, k, v, 0.5, causal)
+        for r in range(Nq):
+            last = (Nk - Nq + r) if causal else Nk - 1
+            sc = [0.5 * sum(q[0, 0, r, c] * k[0, 0, j, c] for c in range(d)) for j in range(last + 1)]
+            mx = max(sc)
+            w = [math.exp(x - mx) for x in sc]
+            tot = sum(w)
+            for c in range(d):
+                ref = sum(w[j] * v[0, 0, j, c] for j in range(last + 1)) / tot
+                assert abs(o[0, 0, r, c] - ref) < 1e-12
+            assert abs(lse[0, 0, r] - (mx + math.log(tot))) < 1e-12
+
+
+def test_suffix_closed_forms():
+    # Q = 0: O is the mean of the visible values, LSE = ln(number visible);
+    # V = 1: O = 1 whatever the scores
+    rng = np.random.default_rng(3)
+    Nq, Nk, d = 4, 10, 3
+    v = rng.standard_normal((1, 2, Nk, d))
+    k = rng.standard_normal((1, 2, Nk, d))
+    o, lse = oracle.attention_forward_suffix(np.zeros((1, 2, Nq, d)), k, v, 1.0, True)
+    for r in range(Nq):
+        n_vis = Nk - Nq + r + 1
+        np.testing.assert_allclose(o[0, :, r], v[0, :, :n_vis].mean(axis=1), atol=1e-12)
+        np.testing.assert_allclose(lse[0, :, r], math.log(n_vis), atol=1e-12)
+    o1, _ = oracle.attention_forward_suffix(rng.standard_normal((1, 2, Nq, d)), k, np.ones_like(v), 0.7, True)
+    np.testing.assert_allclose(o1, 1.0, atol=1e-12)
+
+
+# ---------------------------------------------------------------------------
 # Planted mistakes: each must be caught by one of the pins above
 # ---------------------------------------------------------------------------
 
