@@ -187,6 +187,181 @@ def run_reference(args, w, rank, world):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- decode
+def decode_oracle_sample(w, seconds: float, max_batches: int | None = None):
+    """Time the fp64 oracle's suffix attention on whole batch entries (all
+    heads of one b) of a decode workload.  Returns (TFLOPS, batches, seconds)."""
+    import oracle
+    from exact_attention_104_b200.workloads import make_decode_inputs
+
+    key = (w.name, w.seed)
+    if key not in _CPU_INPUTS:
+        _CPU_INPUTS.clear()
+        _CPU_INPUTS[key] = make_decode_inputs(w, "cpu")
+    q, k, v = _CPU_INPUTS[key]
+    done, t_total = 0, 0.0
+    while True:
+        b = done % w.B
+        sl = lambda t: t[b:b + 1].double().numpy()  # noqa: E731
+        t0 = time.perf_counter()
+        oracle.attention_forward_suffix(sl(q), sl(k), sl(v), w.scale, w.causal)
+        t_total += time.perf_counter() - t0
+        done += 1
+        if t_total >= seconds or (max_batches is not None and done >= max_batches):
+            break
+    return w.fwd_flops() / w.B * done / t_total / 1e12, done, t_total
+
+
+def run_decode(args, w, rank, world, local_rank):
+    """One step = one fa_fwd_decode call over the whole decode workload (all
+    batch entries and heads), K and V resident in HBM.  Reported in the same
+    TFLOPS metric; the roofline is HBM bandwidth, since every step must read
+    the whole K/V cache once."""
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_104_b200 import binding
+    from exact_attention_104_b200.workloads import make_decode_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    stream = torch.cuda.current_stream()
+    q, k, v = make_decode_inputs(w, dev, seed=w.seed + 7919 * rank)
+    o = torch.empty_like(q)
+    lse = torch.empty(w.B, w.Hq, w.Nq, dtype=torch.float32, device=dev)
+    ws_bytes = binding.fa_decode_workspace_bytes(w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d)
+    ws = torch.empty(max(ws_bytes, 256), dtype=torch.uint8, device=dev)
+
+    def step(prof=None):
+        if prof is not None:
+            binding.fa_profile_next(*prof)
+        st = binding.fa_fwd_decode(q, k, v, o, lse, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, w.scale, ws,
+                                   ws_bytes, stream)
+        if st:
+            raise binding.FAError(st, "fa_fwd_decode")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    def max_over_ranks(x: float) -> float:
+        if world == 1:
+            return x
+        t = torch.tensor([x], dtype=torch.float64, device=dev)
+        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        return float(t.item())
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if binding.fa_device_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    k_ev = [(ev(), ev()) for _ in range(K)]
+    start, stop = ev(), ev()
+    for e in [x for pair in k_ev for x in pair] + [start, stop]:
+        e.record(stream)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        start.record(stream)
+        for i in range(K):
+            step(k_ev[i])
+        stop.record(stream)
+        barrier()
+    clocks = clk.summary()
+    if binding.fa_device_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    ms_step = max_over_ranks(start.elapsed_time(stop)) / K
+    ms_split = max_over_ranks(sum(a.elapsed_time(b) for a, b in k_ev) / K)
+    F = w.fwd_flops()
+    value = F * world / (ms_step * 1e-3) / 1e12
+    peaks = _peaks()
+    gbs = w.hbm_bytes() / (ms_split * 1e-3) / 1e9
+
+    e2e = None
+    if not args.no_e2e:
+        # a decoding step's own data is its query rows and its outputs; the K/V
+        # cache stays on the device between steps
+        hq = q.cpu().pin_memory()
+        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
+        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+
+        def e2e_step():
+            q.copy_(hq, non_blocking=True)
+            step()
+            ho.copy_(o, non_blocking=True)
+            hl.copy_(lse, non_blocking=True)
+
+        e2e_step()
+        ke = max(3, min(K, 50))
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        ms_e2e = max_over_ranks(a.elapsed_time(b)) / ke
+        e2e = {"value": F * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": hq.numel() * hq.element_size(),
+               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
+               "steps": ke}
+
+    cpu = None
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        tflops, nb, secs = decode_oracle_sample(w, args.cpu_seconds)
+        cpu = {"value": tflops, "unit": "TFLOPS", "cores": _blas_threads(), "kind": "oracle",
+               "sample": f"{nb} batch entries (all heads) of {w.describe()}, fp64, {secs:.1f} s"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "causal": w.causal, "global_batch": w.B * world, "parallelism": f"dp{world}",
+                   "l2": f"K/V {2 * w.B * w.Hkv * w.Nk * w.d * 2 / 2**20:.0f} MiB per step (> 126 MiB L2: no flush "
+                         "needed)" if 4 * w.B * w.Hkv * w.Nk * w.d > 126 * 2**20 else "K/V fit in L2"},
+        "roofline": {"kernel": "fa_decode_split_kernel", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+                     "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
+                     "peak_source": peaks["source"] + " HBM copy (MEASURED_PEAKS.json)",
+                     "bytes_per_launch": w.hbm_bytes(), "ms_per_launch": ms_split, "traffic": None},
+        "ms": {"split_kernel": ms_split, "call": ms_step},
+        "cpu_baseline": cpu,
+        "e2e": e2e,
+        "gpu_launches": 2 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
+def run_decode_reference(args, w, rank):
+    """The reference arm for a decode workload: the fp64 oracle on one batch
+    entry (all heads) per step.  Rank 0 only."""
+    if rank != 0:
+        return
+    for _ in range(args.warmup):
+        decode_oracle_sample(w, 0.0, max_batches=1)
+    total = 0.0
+    for _ in range(args.steps):
+        total += decode_oracle_sample(w, 0.0, max_batches=1)[2]
+    value = w.fwd_flops() / w.B * args.steps / total / 1e12
+    line = {
+        "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
+        "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
+        "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+        "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "Nq": w.Nq, "Nk": w.Nk, "d": w.d,
+                   "causal": w.causal},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": _blas_threads(), "kind": "oracle",
+                         "sample": f"one batch entry (all heads) of {w.describe()} per step, fp64"},
+        "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+    print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------- e2e
 def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ranks, K):
     """The step through the public C ABI with its data on the host: every step
@@ -452,17 +627,19 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    from exact_attention_104_b200.workloads import BENCH_WORKLOAD, WORKLOADS
+    from exact_attention_104_b200.workloads import BENCH_WORKLOAD, DECODE_WORKLOADS, WORKLOADS
 
-    names = list(WORKLOADS) if args.workload == "all" else [args.workload or BENCH_WORKLOAD]
-    w = WORKLOADS[names[0]]
+    names = list(WORKLOADS) + list(DECODE_WORKLOADS) if args.workload == "all" else [args.workload or BENCH_WORKLOAD]
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
 
     if args.impl == "reference":
         for name in names:
-            run_reference(args, WORKLOADS[name], rank, world)
+            if name in DECODE_WORKLOADS:
+                run_decode_reference(args, DECODE_WORKLOADS[name], rank)
+            else:
+                run_reference(args, WORKLOADS[name], rank, world)
         return
 
     if world > 1:
@@ -476,7 +653,10 @@ def main():
                                 device_id=torch.device("cuda", local_rank))
     try:
         for name in names:
-            run_ours(args, WORKLOADS[name], rank, world, local_rank)
+            if name in DECODE_WORKLOADS:
+                run_decode(args, DECODE_WORKLOADS[name], rank, world, local_rank)
+            else:
+                run_ours(args, WORKLOADS[name], rank, world, local_rank)
     finally:
         if world > 1:
             import torch.distributed as dist

@@ -14,6 +14,9 @@ from .binding import (  # noqa: F401
     fa_status_string,
     attention_forward,
     attention_backward,
+    attention_decode,
+    fa_fwd_decode,
+    fa_decode_workspace_bytes,
     lib,
     LIB_PATH,
 )

@@ -56,6 +56,10 @@ def lib() -> ctypes.CDLL:
     L.fa_selftest_exp2.restype = i
     L.fa_bwd_noalloc.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.fa_bwd_noalloc.restype = i
+    L.fa_decode_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    L.fa_decode_workspace_bytes.restype = z
+    L.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, z, vp]
+    L.fa_fwd_decode.restype = i
     _lib = L
     return L
 
@@ -127,6 +131,19 @@ def fa_bwd_noalloc(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, causal, sc
                                 _stream_handle(stream))
 
 
+def fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d) -> int:
+    return lib().fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d)
+
+
+def fa_fwd_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace, workspace_bytes,
+                  stream=None) -> int:
+    """Raw C-ABI call of the decoding forward pass (Nq queries, the last
+    positions of an Nk-long sequence).  Returns the status."""
+    return lib().fa_fwd_decode(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, Nq, Nk, d,
+                               int(bool(causal)), float(scale), _ptr(workspace), int(workspace_bytes),
+                               _stream_handle(stream))
+
+
 def fa_profile_next(start_event=None, stop_event=None) -> int:
     """Ask the next fa_fwd / fa_bwd call on this thread to record the given
     torch.cuda.Event objects around its attention kernel."""
@@ -181,3 +198,28 @@ def attention_backward(q, k, v, o, lse, do, causal=False, scale=None, dq=None, d
     _check(fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, workspace,
                   workspace.numel() * workspace.element_size(), stream), "fa_bwd")
     return dq, dk, dv
+
+
+def attention_decode(q, k, v, causal=False, scale=None, out=None, lse=None, workspace=None, stream=None):
+    """O, LSE of Nq queries q [B,Hq,Nq,d] against cached k, v [B,Hkv,Nk,d]; the
+    queries are the last Nq positions of the sequence (see fa_fwd_decode)."""
+    if q.dim() != 4 or k.dim() != 4 or v.dim() != 4 or k.shape != v.shape:
+        raise FAError(FA_ERR_INVALID_ARG, "attention_decode: q, k, v must be [B,H,N,d] with k.shape == v.shape")
+    B, Hq, Nq, d = q.shape
+    Hkv, Nk = k.shape[1], k.shape[2]
+    if k.shape[0] != B or k.shape[3] != d:
+        raise FAError(FA_ERR_INVALID_ARG, "attention_decode: batch or head dimension mismatch")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise FAError(FA_ERR_INVALID_ARG, "attention_decode: inputs must be contiguous bf16 CUDA tensors")
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(B, Hq, Nq, dtype=torch.float32, device=q.device)
+    need = fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(fa_fwd_decode(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace,
+                         workspace.numel() * workspace.element_size(), stream), "fa_fwd_decode")
+    return out, lse

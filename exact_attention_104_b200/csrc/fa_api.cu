@@ -3,6 +3,7 @@
 #include <cuda.h>
 #include <cuda_runtime.h>
 
+#include <algorithm>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -10,6 +11,7 @@
 
 #include "fa.h"
 #include "fa_bwd.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd_persistent.cuh"
 
@@ -297,6 +299,81 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restr
 }
 }  // namespace fa
 
+// ------------------------------------------------------------------ decode
+// Split plan of a decode call: row groups of RMAX (4, 8 or 16) query rows,
+// and enough key splits for about kDecodeCtas CTAs in all (a pure function of
+// the sizes, so that fa_decode_workspace_bytes needs no device).
+constexpr int kDecodeCtas = 1024;
+constexpr int kDecodeMaxSplit = 256;
+struct DecodePlan {
+  int rmax = 4, n_rg = 1, n_split = 1, tiles_per_split = 1;
+  size_t part_o_bytes = 0, part_ml_bytes = 0;
+};
+
+fa_status decode_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scale, int causal, bool* empty) {
+  *empty = false;
+  if (B < 0 || Nq < 0 || Nk < 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (B == 0 || Nq == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  if (Nk == 0) return FA_ERR_INVALID_ARG;              // a query with no key at all
+  if (causal && Nq > Nk) return FA_ERR_INVALID_ARG;   // queries before the first key
+  if (Nq > 256) return FA_ERR_UNSUPPORTED;            // decoding sizes; use fa_fwd for long query blocks
+  if (B > 65535 || Hq > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)B * Hq * Nq >= (1LL << 31) || (long long)B * Hkv * Nk >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  DecodePlan pl;
+  const long long R = (long long)(Hq / Hkv) * Nq;
+  pl.rmax = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
+  pl.n_rg = (int)((R + pl.rmax - 1) / pl.rmax);
+  const long long units = (long long)B * Hkv * pl.n_rg;
+  const int n_tiles = (Nk + 63) / 64;
+  long long want = (kDecodeCtas + units - 1) / units;
+  if (want < 1) want = 1;
+  int n_split = (int)std::min<long long>({want, (long long)n_tiles, (long long)kDecodeMaxSplit});
+  pl.tiles_per_split = (n_tiles + n_split - 1) / n_split;
+  pl.n_split = (n_tiles + pl.tiles_per_split - 1) / pl.tiles_per_split;
+  const size_t rows = (size_t)pl.n_split * units * pl.rmax;
+  pl.part_o_bytes = round256(rows * d * 4);
+  pl.part_ml_bytes = round256(rows * 2 * 4);
+  return pl;
+}
+
+template <int D, int RMAX, bool CAUSAL>
+fa_status launch_decode_split(const fa::DecodeParams& p, unsigned units, cudaStream_t s) {
+  using C = fa::DecCfg<D, RMAX>;
+  auto kern = fa::fa_decode_split_kernel<D, RMAX, CAUSAL>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  ProfileScope prof(s);
+  kern<<<dim3((unsigned)p.n_split, units), C::THREADS, C::SMEM_BYTES, s>>>(p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D>
+fa_status launch_decode(const fa::DecodeParams& p, int rmax, bool causal, unsigned units, cudaStream_t s) {
+  fa_status st;
+  switch (rmax) {
+    case 4: st = causal ? launch_decode_split<D, 4, true>(p, units, s) : launch_decode_split<D, 4, false>(p, units, s); break;
+    case 8: st = causal ? launch_decode_split<D, 8, true>(p, units, s) : launch_decode_split<D, 8, false>(p, units, s); break;
+    default: st = causal ? launch_decode_split<D, 16, true>(p, units, s) : launch_decode_split<D, 16, false>(p, units, s); break;
+  }
+  if (st != FA_OK) return st;
+  switch (rmax) {
+    case 4: fa::fa_decode_combine_kernel<D, 4><<<units, 256, 0, s>>>(p); break;
+    case 8: fa::fa_decode_combine_kernel<D, 8><<<units, 256, 0, s>>>(p); break;
+    default: fa::fa_decode_combine_kernel<D, 16><<<units, 256, 0, s>>>(p); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 extern "C" {
 
 const char* fa_status_string(fa_status s) {
@@ -544,6 +621,69 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (st != FA_OK) return st;
   return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, scratch,
                 (size_t)FA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
+  bool empty = false;
+  if (decode_sizes(B, Hq, Hkv, Nq, Nk, d, 1.f, 0, &empty) != FA_OK || empty) return 0;
+  const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d);
+  return pl.part_o_bytes + pl.part_ml_bytes;
+}
+
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                        int Nq, int Nk, int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream) {
+  bool empty = false;
+  fa_status st = decode_sizes(B, Hq, Hkv, Nq, Nk, d, scale, causal, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, (const void*)o, (const void*)lse})
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_decode_workspace_bytes(B, Hq, Hkv, Nq, Nk, d);
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * Nq * d * 2, kvbytes = (size_t)B * Hkv * Nk * d * 2;
+  const Range ins[3] = {span(q, qbytes), span(k, kvbytes), span(v, kvbytes)};
+  const Range outs[3] = {span(o, qbytes), span(lse, (size_t)B * Hq * Nq * 4), span(workspace, need)};
+  for (int i = 0; i < 3; ++i) {
+    for (int j = 0; j < 3; ++j)
+      if (overlap(outs[i], ins[j])) return FA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], outs[j])) return FA_ERR_INVALID_ARG;
+  }
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+
+  const DecodePlan pl = decode_plan(B, Hq, Hkv, Nq, Nk, d);
+  fa::DecodeParams p;
+  p.q = static_cast<const __nv_bfloat16*>(q);
+  p.k = static_cast<const __nv_bfloat16*>(k);
+  p.v = static_cast<const __nv_bfloat16*>(v);
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.part_o = static_cast<float*>(workspace);
+  p.part_ml = reinterpret_cast<float*>(static_cast<uint8_t*>(workspace) + pl.part_o_bytes);
+  p.B = B;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.R = p.G * Nq;
+  p.n_rg = pl.n_rg;
+  p.n_split = pl.n_split;
+  p.tiles_per_split = pl.tiles_per_split;
+  p.scale_log2 = scale * fa::kLog2e;
+  const long long n_units = (long long)B * Hkv * pl.n_rg;
+  if (n_units > 65535) return FA_ERR_UNSUPPORTED;  // grid.y of the split kernel
+  const unsigned units = (unsigned)n_units;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  switch (d) {
+    case 64: return launch_decode<64>(p, pl.rmax, causal != 0, units, s);
+    case 128: return launch_decode<128>(p, pl.rmax, causal != 0, units, s);
+    default: return launch_decode<256>(p, pl.rmax, causal != 0, units, s);
+  }
 }
 
 }  // extern "C"

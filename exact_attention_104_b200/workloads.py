@@ -72,6 +72,66 @@ WORKLOADS = {
 BENCH_WORKLOAD = "train_b8_h16_n2048_d128"
 
 
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Nq query rows per head (the last Nq positions of the sequence) against
+    Nk cached keys and values."""
+    name: str
+    B: int
+    Hq: int
+    Hkv: int
+    Nq: int
+    Nk: int
+    d: int
+    causal: bool
+    seed: int
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    def visible_pairs(self) -> int:
+        """(query, key) pairs per head that the mask leaves visible."""
+        if not self.causal:
+            return self.Nq * self.Nk
+        return sum(self.Nk - self.Nq + i + 1 for i in range(self.Nq))
+
+    def fwd_flops(self) -> float:
+        """4·d FLOPs per visible (query, key) pair and query head."""
+        return 4.0 * self.B * self.Hq * self.d * self.visible_pairs()
+
+    def hbm_bytes(self) -> int:
+        """Bytes one call must move: K and V once, Q in, O and LSE out."""
+        kv = 2 * self.B * self.Hkv * self.Nk * self.d * 2
+        qo = 2 * self.B * self.Hq * self.Nq * self.d * 2
+        return kv + qo + self.B * self.Hq * self.Nq * 4
+
+    def describe(self) -> str:
+        return (f"B={self.B} Hq={self.Hq} Hkv={self.Hkv} Nq={self.Nq} Nk={self.Nk} d={self.d} "
+                f"{'causal' if self.causal else 'non-causal'}")
+
+
+DECODE_WORKLOADS = {
+    # one decoding step of a batch of 8 sequences with a 32k-token cache, GQA 4:1
+    "decode_b8_hq32_hkv8_nk32768_d128": DecodeWorkload("decode_b8_hq32_hkv8_nk32768_d128", 8, 32, 8, 1, 32768, 128,
+                                                      True, 1007),
+}
+
+
+def make_decode_inputs(w: DecodeWorkload, device="cpu", seed: int | None = None):
+    """Draw (q, k, v) as bf16 tensors [B,Hq,Nq,d], [B,Hkv,Nk,d], [B,Hkv,Nk,d]
+    (standard normals, in that order) from the workload's seed."""
+    g = torch.Generator("cpu").manual_seed(w.seed if seed is None else seed)
+    q = torch.randn(w.B, w.Hq, w.Nq, w.d, generator=g, dtype=torch.float32)
+    k = torch.randn(w.B, w.Hkv, w.Nk, w.d, generator=g, dtype=torch.float32)
+    v = torch.randn(w.B, w.Hkv, w.Nk, w.d, generator=g, dtype=torch.float32)
+    return tuple(t.to(torch.bfloat16).to(device) for t in (q, k, v))
+
+
 def make_inputs(w: Workload, device="cpu", seed: int | None = None):
     """Draw (q, k, v, do) as bf16 tensors with shapes [B,Hq,N,d], [B,Hkv,N,d],
     [B,Hkv,N,d], [B,Hq,N,d] from the workload's seed, then move them to

@@ -123,6 +123,28 @@ fa_status fa_selftest_wait_timeout(long long cap_cycles, void* stream);
  * (use_poly = 1). */
 fa_status fa_selftest_exp2(const float* x, float* y, long long n, int use_poly, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Decoding: Nq query rows per head against Nk cached keys and values.
+ *
+ * The queries are the last Nq positions of an Nk-long sequence: query row i
+ * sits at position Nk - Nq + i, and with `causal` != 0 it sees keys
+ * 0 .. Nk - Nq + i (so its result is row Nk - Nq + i of fa_fwd over the whole
+ * sequence).  Same per-row online softmax as fa_fwd ("深度学习进阶（三十一）
+ * FlashAttention：IO 感知的精确注意力" §2.2); the key axis is split over
+ * CTAs and the partial results are merged with their running maxima and
+ * normalisers, since with few query rows the pass is bound by reading K, V.
+ *
+ * Layouts: q, o bf16 [B, Hq, Nq, d]; k, v bf16 [B, Hkv, Nk, d]; lse fp32
+ * [B, Hq, Nq] (natural log).  `workspace` (device, 256-byte aligned, at least
+ * fa_decode_workspace_bytes) holds the per-split partial results.
+ * Errors as for fa_fwd, plus FA_ERR_INVALID_ARG for Nk == 0 with Nq > 0 and
+ * for causal with Nq > Nk, and FA_ERR_UNSUPPORTED for Nq > 256 (use fa_fwd).
+ * Two kernels are enqueued on `stream`; B == 0 or Nq == 0 is a no-op. */
+size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d);
+fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, float* lse,
+                        int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
+                        void* workspace, size_t workspace_bytes, void* stream);
+
 /* Size in bytes of the fixed device scratch array used by fa_bwd_noalloc. */
 #define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 

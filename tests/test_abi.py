@@ -122,3 +122,44 @@ def test_wait_cap_setter(lib):
     assert lib.fa_set_wait_cap(-1) == binding.FA_ERR_INVALID_ARG
     assert lib.fa_set_wait_cap(1 << 28) == binding.FA_OK
     assert lib.fa_set_wait_cap(0) == binding.FA_OK
+
+
+def test_decode_workspace_bytes(lib):
+    # per-split partial O (fp32, d per row) and (m, l) for every row group of
+    # 4, 8 or 16 query rows; grows with the key count until the split count caps
+    ws = binding.fa_decode_workspace_bytes
+    assert ws(8, 32, 8, 1, 32768, 128) > 0
+    assert ws(8, 32, 8, 1, 64, 128) <= ws(8, 32, 8, 1, 4096, 128)
+    assert ws(1, 4, 1, 1, 100, 64) % 256 == 0
+    assert ws(1, 3, 2, 1, 100, 64) == 0       # Hq % Hkv != 0
+    assert ws(1, 2, 2, 1, 100, 96) == 0       # unsupported d
+    assert ws(1, 2, 2, 1, 0, 64) == 0         # queries with no key
+    assert ws(0, 2, 2, 1, 100, 64) == 0       # empty problem needs nothing
+
+
+def _dec(lib, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5, B=1, Hq=4, Hkv=2, Nq=1, Nk=300, d=128,
+             causal=1, scale=0.088, ws=FAKE * 6, wsb=1 << 20)
+    a.update(kw)
+    return binding.fa_fwd_decode(a["q"], a["k"], a["v"], a["o"], a["lse"], a["B"], a["Hq"], a["Hkv"], a["Nq"],
+                                 a["Nk"], a["d"], a["causal"], a["scale"], a["ws"], a["wsb"], 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), binding.FA_ERR_INVALID_ARG),
+    (dict(ws=0), binding.FA_ERR_INVALID_ARG),
+    (dict(k=FAKE * 2 + 8), binding.FA_ERR_INVALID_ARG),          # misaligned
+    (dict(ws=FAKE * 6 + 16), binding.FA_ERR_INVALID_ARG),        # workspace not 256-aligned
+    (dict(wsb=100), binding.FA_ERR_INVALID_ARG),                 # workspace too small
+    (dict(o=FAKE), binding.FA_ERR_INVALID_ARG),                  # output aliases q
+    (dict(Hq=3), binding.FA_ERR_INVALID_ARG),                    # Hq % Hkv
+    (dict(Nk=0), binding.FA_ERR_INVALID_ARG),                    # queries with no key
+    (dict(Nq=301), binding.FA_ERR_INVALID_ARG),                  # causal queries before the first key
+    (dict(Nq=300, causal=0), binding.FA_ERR_UNSUPPORTED),        # long query blocks belong to fa_fwd
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(scale=-1.0), binding.FA_ERR_INVALID_ARG),
+    (dict(B=0), binding.FA_OK),                                  # empty problem: nothing to do
+    (dict(Nq=0), binding.FA_OK),
+])
+def test_decode_argument_validation(lib, kw, expect):
+    assert _dec(lib, **kw) == expect

@@ -1,0 +1,71 @@
+"""GPU parity of the decoding forward pass (fa_fwd_decode, through the C ABI)
+against the fp64 oracle's suffix attention: Nq queries that are the last Nq
+positions of an Nk-long sequence.  Tolerances are the forward's (O max-abs
+2e-2, mean-abs 2e-3; LSE 1e-3)."""
+
+import numpy as np
+import pytest
+import torch
+
+import oracle
+from exact_attention_104_b200 import attention_decode, binding, lib
+from exact_attention_104_b200.workloads import DECODE_WORKLOADS, DecodeWorkload, make_decode_inputs
+
+from _parity import LSE_MAX_ABS, O_MAX_ABS, O_MEAN_ABS, f64
+
+pytestmark = pytest.mark.gpu
+
+
+@pytest.fixture(scope="module", autouse=True)
+def _short_waits():
+    lib().fa_set_wait_cap(1 << 28)
+    yield
+    lib().fa_set_wait_cap(0)
+
+
+def _check(w):
+    q, k, v = make_decode_inputs(w, "cuda")
+    o, lse = attention_decode(q, k, v, causal=w.causal, scale=w.scale)
+    torch.cuda.synchronize()
+    assert binding.fa_device_status() == binding.FA_OK
+    o_ref, lse_ref = oracle.attention_forward_suffix(f64(q), f64(k), f64(v), w.scale, w.causal)
+    err_o = np.abs(f64(o) - o_ref)
+    err_l = np.abs(f64(lse) - lse_ref)
+    msg = f"{w.name}: O max {err_o.max():.3e} mean {err_o.mean():.3e} LSE max {err_l.max():.3e}"
+    assert err_o.max() <= O_MAX_ABS and err_o.mean() <= O_MEAN_ABS and err_l.max() <= LSE_MAX_ABS, msg
+
+
+# (B, Hq, Hkv, Nq, Nk, d, causal): single key; GQA groups of 4 and 8 rows;
+# Nk ragged against the 64-key tiles; Nq = Nk (a whole square problem);
+# G·Nq = 128 rows (eight row groups); d = 64, 128, 256
+CASES = [
+    (1, 1, 1, 1, 1, 128, True),
+    (1, 4, 1, 1, 100, 128, True),
+    (2, 8, 2, 3, 1000, 64, True),
+    (1, 8, 1, 16, 4097, 128, False),
+    (1, 2, 2, 16, 16, 256, True),
+    (2, 32, 8, 1, 5000, 128, True),
+    (1, 4, 4, 5, 64, 256, False),
+    (1, 16, 2, 2, 3333, 128, True),
+    (1, 2, 1, 7, 129, 64, False),
+]
+
+
+@pytest.mark.parametrize("case", CASES, ids=lambda c: "b{}_hq{}_hkv{}_nq{}_nk{}_d{}_{}".format(*c[:6], "c" if c[6] else "nc"))
+def test_decode_matches_oracle(case):
+    B, Hq, Hkv, Nq, Nk, d, causal = case
+    _check(DecodeWorkload("dec", B, Hq, Hkv, Nq, Nk, d, causal, 300 + Nk + Nq))
+
+
+@pytest.mark.parametrize("name", list(DECODE_WORKLOADS))
+def test_decode_bench_workload_matches_oracle(name):
+    _check(DECODE_WORKLOADS[name])
+
+
+def test_decode_is_deterministic():
+    w = DecodeWorkload("det", 2, 8, 2, 2, 2000, 128, True, 91)
+    q, k, v = make_decode_inputs(w, "cuda")
+    a = attention_decode(q, k, v, causal=True)
+    b = attention_decode(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])

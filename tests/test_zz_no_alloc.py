@@ -32,6 +32,7 @@ def _workspace_bwd(w, q, k, v, o, lse, do):
     Workload("na_d128_gqa_causal", 2, 4, 2, 512, 128, True, 1.0, 61),
     Workload("na_d64", 1, 2, 2, 384, 64, False, 1.0, 62),
     Workload("na_d256", 1, 2, 1, 256, 256, False, 1.0, 63),
+    Workload("na_d128_ragged_causal", 1, 2, 2, 300, 128, True, 1.0, 65),
 ], ids=lambda w: w.name)
 def test_noalloc_backward_matches_workspace_backward_on_two_calls(w):
     assert binding.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d) <= binding.FA_NOALLOC_SCRATCH_BYTES
