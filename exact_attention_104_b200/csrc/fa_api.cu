@@ -220,9 +220,15 @@ fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, co
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// d = 64, 128: one persistent CTA per SM walks the key-tile units; d = 256:
+// one CTA per unit (its one query/dO stage leaves nothing to overlap).
+#ifndef FA_BWD_PERSISTENT
+#define FA_BWD_PERSISTENT 1
+#endif
+
 template <int D, bool CAUSAL, bool TAIL>
 fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tdo, const fa::BwdParams& p, int B, int Hkv, cudaStream_t stream) {
+                          const CUtensorMap& tdo, fa::BwdParams p, int B, int Hkv, int sms, cudaStream_t stream) {
   using C = fa::BwdCfg<D>;
   auto kern = fa::fa_bwd_kernel<D, CAUSAL, TAIL>;
   if (C::REG_SPLIT && !reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
@@ -232,7 +238,9 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
     return FA_ERR_CUDA;
   const long long units = (long long)((p.N + C::BC - 1) / C::BC) * C::NDH * Hkv * B;
   if (units >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
-  const dim3 grid((unsigned)units);
+  p.n_units = (int)units;
+  const bool persistent = FA_BWD_PERSISTENT && D <= 128;
+  const dim3 grid((unsigned)(persistent && units > sms ? sms : units));
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -240,7 +248,7 @@ fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CU
 
 template <int D>
 fa_status launch_bwd_pre(const void* o, const void* dout, const float* lse, float* dvec, float* lse2, float* dqacc,
-                         int N, int Np, long long rows_p, int sms, cudaStream_t stream) {
+                         int* unit_counter, int N, int Np, long long rows_p, int sms, cudaStream_t stream) {
   const long long dq_vec4 = rows_p * D / 4;
   long long want = rows_p * (D / 8);
   if (dq_vec4 > want) want = dq_vec4;
@@ -249,8 +257,8 @@ fa_status launch_bwd_pre(const void* o, const void* dout, const float* lse, floa
   if (blocks > cap) blocks = cap;
   if (blocks < 1) blocks = 1;
   fa::fa_bwd_pre_kernel<D><<<(unsigned)blocks, 256, 0, stream>>>(
-      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc, N, Np,
-      rows_p, dq_vec4);
+      static_cast<const __nv_bfloat16*>(o), static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc,
+      unit_counter, N, Np, rows_p, dq_vec4);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -427,7 +435,7 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d) {
   bool empty = false;
   if (check_sizes(B, Hq, Hkv, N, d, 1.f, &empty) != FA_OK) return 0;
   const size_t rows_p = (size_t)B * Hq * pad128(N);  // per-head stride N rounded up to 128
-  return 2 * round256(rows_p * 4) + round256(rows_p * (size_t)d * 4);
+  return 2 * round256(rows_p * 4) + round256(rows_p * (size_t)d * 4) + 256;  // + the unit counter
 }
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv, int N,
@@ -516,19 +524,21 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   st = current_device(&di);
   if (st != FA_OK) return st;
 
-  // workspace: D, lse2 (B·Hq·Np fp32 each) and the dQ accumulator (B·Hq·Np·d fp32)
+  // workspace: D, lse2 (B·Hq·Np fp32 each), the dQ accumulator (B·Hq·Np·d fp32)
+  // and the main kernel's unit counter
   const int Np = (int)pad128(N);
   const size_t rows_p = (size_t)B * Hq * Np;
   uint8_t* ws = static_cast<uint8_t*>(workspace);
   float* dvec = reinterpret_cast<float*>(ws);
   float* lse2 = reinterpret_cast<float*>(ws + round256(rows_p * 4));
   float* dqacc = reinterpret_cast<float*>(ws + 2 * round256(rows_p * 4));
+  int* unit_counter = reinterpret_cast<int*>(ws + 2 * round256(rows_p * 4) + round256(rows_p * (size_t)d * 4));
   cudaStream_t s = static_cast<cudaStream_t>(stream);
 
   switch (d) {
-    case 64: st = launch_bwd_pre<64>(o, dout, lse, dvec, lse2, dqacc, N, Np, (long long)rows_p, di->sms, s); break;
-    case 128: st = launch_bwd_pre<128>(o, dout, lse, dvec, lse2, dqacc, N, Np, (long long)rows_p, di->sms, s); break;
-    default: st = launch_bwd_pre<256>(o, dout, lse, dvec, lse2, dqacc, N, Np, (long long)rows_p, di->sms, s); break;
+    case 64: st = launch_bwd_pre<64>(o, dout, lse, dvec, lse2, dqacc, unit_counter, N, Np, (long long)rows_p, di->sms, s); break;
+    case 128: st = launch_bwd_pre<128>(o, dout, lse, dvec, lse2, dqacc, unit_counter, N, Np, (long long)rows_p, di->sms, s); break;
+    default: st = launch_bwd_pre<256>(o, dout, lse, dvec, lse2, dqacc, unit_counter, N, Np, (long long)rows_p, di->sms, s); break;
   }
   if (st != FA_OK) return st;
 
@@ -546,6 +556,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.N = N;
   p.Np = Np;
   p.B = B;
+  p.unit_counter = unit_counter;
   {
     // Causal: key tiles in bands, heaviest band first (see fa_bwd_kernel).  More
     // bands shorten the tail of heavy CTAs dispatched last; fewer keep the
@@ -568,10 +579,10 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   const bool tail = (N % 128) != 0;
   auto main_kernel = [&](auto dtag) -> fa_status {
     constexpr int D = decltype(dtag)::value;
-    if (causal) return tail ? launch_bwd_main<D, true, true>(tq, tk, tv, tdo, p, B, Hkv, s)
-                            : launch_bwd_main<D, true, false>(tq, tk, tv, tdo, p, B, Hkv, s);
-    return tail ? launch_bwd_main<D, false, true>(tq, tk, tv, tdo, p, B, Hkv, s)
-                : launch_bwd_main<D, false, false>(tq, tk, tv, tdo, p, B, Hkv, s);
+    if (causal) return tail ? launch_bwd_main<D, true, true>(tq, tk, tv, tdo, p, B, Hkv, di->sms, s)
+                            : launch_bwd_main<D, true, false>(tq, tk, tv, tdo, p, B, Hkv, di->sms, s);
+    return tail ? launch_bwd_main<D, false, true>(tq, tk, tv, tdo, p, B, Hkv, di->sms, s)
+                : launch_bwd_main<D, false, false>(tq, tk, tv, tdo, p, B, Hkv, di->sms, s);
   };
   switch (d) {
     case 64: st = main_kernel(std::integral_constant<int, 64>{}); break;

@@ -65,11 +65,17 @@ struct BwdCfg {
   static constexpr int B_DQEMPTY = B_DQFULL + 1;
   static constexpr int B_STGFREE = B_DQEMPTY + 1;  // staging may be overwritten
   static constexpr int B_STGFULL = B_STGFREE + 1;  // staging written by all drain threads
-  static constexpr int B_ACC = B_STGFULL + 1;
-  static constexpr int B_DRAIN = B_ACC + 1;
+  static constexpr int B_ACC = B_STGFULL + 1;     // a unit's dK, dV accumulated
+  static constexpr int B_KVEMPTY = B_ACC + 1;     // a unit's last product has read K, V
+  static constexpr int B_DKFREE = B_KVEMPTY + 1;  // dK read out of TMEM (next unit may overwrite)
+  static constexpr int B_DVFREE = B_DKFREE + 1;   // dV read out of TMEM
+  static constexpr int B_UNITFULL = B_DVFREE + 1;   // + {0,1}: next unit index published
+  static constexpr int B_UNITEMPTY = B_UNITFULL + 2; // + {0,1}: read by all nine consumer warps
+  static constexpr int B_DRAIN = B_UNITEMPTY + 2;
   static constexpr int NBAR = B_DRAIN + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
-  static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
+  static constexpr int UNIT_OFF = MISC_OFF + 16;   // two unit-index slots
+  static constexpr int SMEM_BYTES = UNIT_OFF + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int DK_COL = 0;
   static constexpr int DV_COL = DH;
@@ -101,16 +107,18 @@ struct BwdCfg {
 //
 // One group of D/8 threads per padded row: D_i = Σ_c dO_ic·O_ic in fp32 and
 // lse2_i = LSE_i·log2e for i < N, zero for the padding rows.  Also zeroes
-// the fp32 dQ accumulator.
+// the fp32 dQ accumulator and the main kernel's unit counter.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_pre_kernel(const __nv_bfloat16* __restrict__ o,
                                                          const __nv_bfloat16* __restrict__ dout,
                                                          const float* __restrict__ lse, float* __restrict__ dvec,
                                                          float* __restrict__ lse2, float* __restrict__ dqacc,
-                                                         int N, int Np, long long rows_p, long long dq_vec4) {
+                                                         int* __restrict__ unit_counter, int N, int Np,
+                                                         long long rows_p, long long dq_vec4) {
   constexpr int TPR = D / 8;
   const long long tid = (long long)blockIdx.x * blockDim.x + threadIdx.x;
   const long long nthreads = (long long)gridDim.x * blockDim.x;
+  if (tid == 0) *unit_counter = 0;
   // zero the accumulator
   float4* acc4 = reinterpret_cast<float4*>(dqacc);
   for (long long i = tid; i < dq_vec4; i += nthreads) acc4[i] = make_float4(0.f, 0.f, 0.f, 0.f);
@@ -180,14 +188,61 @@ struct BwdParams {
   __nv_bfloat16* dk;
   __nv_bfloat16* dv;
   int N, Np, B, Hq, Hkv, G;  // Np: per-head row stride of lse2, dvec and dqacc
-  int jt_band;               // key tiles per scheduling band (see fa_bwd_kernel)
+  int jt_band;               // key tiles per scheduling band (see bwd_unit)
+  int n_units;               // key-tile units (x output-column halves at d = 256)
+  int* unit_counter;         // next unclaimed unit (zeroed by fa_bwd_pre_kernel)
   float scale, scale_log2;
   long long wait_cap;
   int* err;
 };
 
+// One unit of backward work: a 128-key tile (and, at d = 256, one half of the
+// output columns) of one (batch, kv head), streamed against the 64-row query
+// tiles of every query head of its GQA group (causal: only those at or after
+// the diagonal).  Units are numbered so that key tiles come in bands of
+// p.jt_band, earliest band first, head by head inside a band: CTAs running at
+// the same time share Q/dO tiles in L2, and with a causal mask the heavy bands
+// (early key tiles, more query steps) run first.
+struct BwdUnit {
+  int jt, dh, hkv, b, i_start, per_head, n;
+};
+
+template <int D, bool CAUSAL>
+__device__ __forceinline__ BwdUnit bwd_unit(int idx, const BwdParams& p) {
+  using C = BwdCfg<D>;
+  const int n_kt = (p.N + C::BC - 1) / C::BC;
+  const int U = C::NDH * p.Hkv * p.B;  // units per key tile
+  const int bi = idx / (p.jt_band * U);
+  const int wb = min(p.jt_band, n_kt - bi * p.jt_band);  // key tiles in this band
+  const int rb = idx - bi * p.jt_band * U;
+  const int bh = rb / (wb * C::NDH);
+  const int rem = rb - bh * (wb * C::NDH);
+  BwdUnit u;
+  u.jt = bi * p.jt_band + rem / C::NDH;
+  u.dh = rem % C::NDH;
+  u.hkv = bh % p.Hkv;
+  u.b = bh / p.Hkv;
+  const int nqt = (p.N + C::BR - 1) / C::BR;
+  u.i_start = CAUSAL ? (u.jt * C::BC) / C::BR : 0;
+  u.per_head = nqt - u.i_start;
+  u.n = p.G * u.per_head;  // query steps
+  return u;
+}
+
 // TAIL: N is not a multiple of 128 (keys and queries past N get P = 0, rows past
 // N are not stored).
+//
+// A CTA claims units one at a time from a global counter (the producer thread
+// takes the next index with an atomic add and hands it to the other roles
+// through a two-slot ring in shared memory), so the heaviest units spread over
+// the SMs as the hardware block scheduler would spread CTAs; with fewer CTAs
+// than units the kernel is persistent.  All step-level barriers
+// count steps across units (g = steps of earlier units + s), so consecutive
+// units form one pipeline; across a unit boundary K and V are reloaded once
+// the unit's last product has read them (b_kvempty), and the next unit's first
+// dV / dK products wait until the previous unit's accumulators have been read
+// out of TMEM (b_dvfree / b_dkfree), so its epilogue overlaps the next unit's
+// first loads and products.
 template <int D, bool CAUSAL, bool TAIL>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
@@ -203,27 +258,6 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  // Work unit of this CTA (one 1-D grid).  Key tiles are taken in bands of
-  // p.jt_band, earliest band first; inside a band the units go head by head,
-  // so that the key tiles of one head that run at the same time stream the
-  // same Q/dO tiles through L2.  Causal: earlier key tiles have more query
-  // steps, so heavy bands run first and the last CTAs dispatched are light
-  // (no long tail).  Non-causal: one band (plain head-major order).
-  const int n_kt = (p.N + C::BC - 1) / C::BC;
-  const int U = C::NDH * p.Hkv * p.B;  // units per key tile
-  const int bi = (int)(blockIdx.x / ((unsigned)p.jt_band * U));
-  const int wb = min(p.jt_band, n_kt - bi * p.jt_band);  // key tiles in this band
-  const int rb = (int)(blockIdx.x - (unsigned)bi * p.jt_band * U);
-  const int bh = rb / (wb * C::NDH);
-  const int rem = rb - bh * (wb * C::NDH);
-  const int jt = bi * p.jt_band + rem / C::NDH;  // key tile
-  const int dh = rem % C::NDH;                   // output column half
-  const int hkv = bh % p.Hkv;
-  const int b = bh / p.Hkv;
-  const int nqt = (p.N + C::BR - 1) / C::BR;
-  const int i_start = CAUSAL ? (jt * C::BC) / C::BR : 0;
-  const int per_head = nqt - i_start;
-  const int n = p.G * per_head;  // steps
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_KVFULL), 1);
@@ -242,6 +276,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(BAR(C::B_STGFREE), 1);
     mbar_init(BAR(C::B_STGFULL), 128);
     mbar_init(BAR(C::B_ACC), 1);
+    mbar_init(BAR(C::B_KVEMPTY), 1);
+    mbar_init(BAR(C::B_DKFREE), 4);
+    mbar_init(BAR(C::B_DVFREE), 4);
+    for (int i = 0; i < 2; ++i) {
+      mbar_init(BAR(C::B_UNITFULL + i), 1);
+      mbar_init(BAR(C::B_UNITEMPTY + i), 9);  // MMA warp, four compute warps, four drain warps
+    }
     mbar_init(BAR(C::B_DRAIN), 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -256,8 +297,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   const uint32_t tbase = *tmem_holder;
   const WaitCtx wc{abort_flag, p.err, p.wait_cap};
 
-  auto step_head = [&](int s) { return hkv * p.G + s / per_head; };
-  auto step_q0 = [&](int s) { return (i_start + s % per_head) * C::BR; };
+  auto step_head = [&](const BwdUnit& u, int s) { return u.hkv * p.G + s / u.per_head; };
+  auto step_q0 = [&](const BwdUnit& u, int s) { return (u.i_start + s % u.per_head) * C::BR; };
+  // unit-index ring: slot uc & 1 holds the index of this CTA's uc-th unit
+  volatile int* unit_slot = reinterpret_cast<volatile int*>(smem + C::UNIT_OFF);
+  // consumer side (whole warp): the index of unit uc, or -1 on a failed wait
+  auto next_unit = [&](int uc) -> int {
+    if (!mbar_wait_warp(BAR(C::B_UNITFULL + (uc & 1)), (uc >> 1) & 1, wc, 26)) return -1;
+    const int idx = unit_slot[uc & 1];
+    __syncwarp();
+    if (lane == 0) mbar_arrive(BAR(C::B_UNITEMPTY + (uc & 1)));
+    return idx;
+  };
 
   if (warp == 0) {
     // ------------------------------------------------------------ producer
@@ -267,27 +318,50 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&tmK);
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
-      const int kv_row = (b * p.Hkv + hkv) * p.N + jt * C::BC;
-      mbar_expect_tx(BAR(C::B_KVFULL), 2 * C::KV_BYTES);
+      int gs = 0;  // steps loaded before this unit
+      bool ok = true;
+      for (int uc = 0; ok; ++uc) {
+        // claim the next unit and publish its index (an index past the end
+        // tells every role to stop)
+        const int idx = atomicAdd(p.unit_counter, 1);
+        if (uc >= 2 && !mbar_wait(BAR(C::B_UNITEMPTY + (uc & 1)), ((uc >> 1) - 1) & 1, wc, 27)) break;
+        unit_slot[uc & 1] = idx;
+        mbar_arrive(BAR(C::B_UNITFULL + (uc & 1)));
+        if (idx >= p.n_units) break;
+        const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+        // Q, dO, lse2, D of step s of this unit into its stage
+        auto load_q = [&](int s) -> bool {
+          const int g = gs + s;
+          const int st = g % C::NSTAGE;
+          if (!mbar_wait(BAR(C::B_QEMPTY + st), ((g / C::NSTAGE) & 1) ^ 1, wc, 11)) return false;
+          const int q_row = (u.b * p.Hq + step_head(u, s)) * p.N + step_q0(u, s);
+          const int q_row_p = (u.b * p.Hq + step_head(u, s)) * p.Np + step_q0(u, s);
+          const uint32_t bar = BAR(C::B_QFULL + st);
+          mbar_expect_tx(bar, 2 * C::Q_BYTES + 512);
 #pragma unroll
-      for (int pn = 0; pn < D / 64; ++pn) {
-        tma_load_2d(sbase + C::K_OFF + pn * C::KV_PANEL, &tmK, BAR(C::B_KVFULL), pn * 64, kv_row);
-        tma_load_2d(sbase + C::V_OFF + pn * C::KV_PANEL, &tmV, BAR(C::B_KVFULL), pn * 64, kv_row);
-      }
-      for (int s = 0; s < n; ++s) {
-        const int st = s % C::NSTAGE;
-        if (!mbar_wait(BAR(C::B_QEMPTY + st), ((s / C::NSTAGE) & 1) ^ 1, wc, 11)) break;
-        const int q_row = (b * p.Hq + step_head(s)) * p.N + step_q0(s);
-        const int q_row_p = (b * p.Hq + step_head(s)) * p.Np + step_q0(s);
-        const uint32_t bar = BAR(C::B_QFULL + st);
-        mbar_expect_tx(bar, 2 * C::Q_BYTES + 512);
+          for (int pn = 0; pn < D / 64; ++pn) {
+            tma_load_2d(sbase + C::Q_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmQ, bar, pn * 64, q_row);
+            tma_load_2d(sbase + C::DO_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmDO, bar, pn * 64, q_row);
+          }
+          bulk_load(sbase + C::LS_OFF + st * 512, p.lse2 + q_row_p, 256, bar);
+          bulk_load(sbase + C::LS_OFF + st * 512 + 256, p.dvec + q_row_p, 256, bar);
+          return true;
+        };
+        // the first steps' tiles only need free stages: load them before K, V,
+        // which wait for the previous unit's last product
+        const int pre = u.n < C::NSTAGE ? u.n : C::NSTAGE;
+        for (int s = 0; s < pre && ok; ++s) ok = load_q(s);
+        if (!ok) break;
+        if (uc > 0 && !mbar_wait(BAR(C::B_KVEMPTY), (uc - 1) & 1, wc, 18)) break;
+        const int kv_row = (u.b * p.Hkv + u.hkv) * p.N + u.jt * C::BC;
+        mbar_expect_tx(BAR(C::B_KVFULL), 2 * C::KV_BYTES);
 #pragma unroll
         for (int pn = 0; pn < D / 64; ++pn) {
-          tma_load_2d(sbase + C::Q_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmQ, bar, pn * 64, q_row);
-          tma_load_2d(sbase + C::DO_OFF + st * C::Q_BYTES + pn * C::Q_PANEL, &tmDO, bar, pn * 64, q_row);
+          tma_load_2d(sbase + C::K_OFF + pn * C::KV_PANEL, &tmK, BAR(C::B_KVFULL), pn * 64, kv_row);
+          tma_load_2d(sbase + C::V_OFF + pn * C::KV_PANEL, &tmV, BAR(C::B_KVFULL), pn * 64, kv_row);
         }
-        bulk_load(sbase + C::LS_OFF + st * 512, p.lse2 + q_row_p, 256, bar);
-        bulk_load(sbase + C::LS_OFF + st * 512 + 256, p.dvec + q_row_p, 256, bar);
+        for (int s = pre; s < u.n && ok; ++s) ok = load_q(s);
+        gs += u.n;
       }
     }
   } else if (warp == 1) {
@@ -295,22 +369,18 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     // (the whole warp runs this role; one elected lane issues each instruction)
     if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
     {
-      bool ok = mbar_wait_warp(BAR(C::B_KVFULL), 0, wc, 12);
-      tc_fence_after();
-      auto wait_q = [&](int s) -> bool {
-        const bool r = mbar_wait_warp(BAR(C::B_QFULL + s % C::NSTAGE), (s / C::NSTAGE) & 1, wc, 13);
+      bool ok = true;
+      auto wait_q = [&](int g) -> bool {
+        const bool r = mbar_wait_warp(BAR(C::B_QFULL + g % C::NSTAGE), (g / C::NSTAGE) & 1, wc, 13);
         tc_fence_after();
         return r;
       };
-      // Descriptors are built once; each MMA only adds a compile-time offset
-      // (the issuing thread must keep up with 48-cycle MMAs).
+      // Descriptors are built once per unit; each MMA only adds a compile-time
+      // offset (the issuing thread must keep up with 48-cycle MMAs).
       const uint64_t dK_k = sdesc_sw128(sbase + C::K_OFF, 16, 1024);
       const uint64_t dV_k = sdesc_sw128(sbase + C::V_OFF, 16, 1024);
       const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
       const uint64_t dDO_k = sdesc_sw128(sbase + C::DO_OFF, 16, 1024);
-      const uint64_t dQ_mn = sdesc_sw128(sbase + C::Q_OFF + (dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
-      const uint64_t dDO_mn = sdesc_sw128(sbase + C::DO_OFF + (dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
-      const uint64_t dKT_mn = sdesc_sw128(sbase + C::K_OFF + (dh * C::DH / 64) * C::KV_PANEL, C::KV_PANEL, 1024);
       const uint64_t dDS_mn = sdesc_sw128(sbase + C::DS_OFF, 16384, 1024);
       // Sᵀ / dPᵀ: [128 keys x 64 queries] = (K or V tile) · (Q or dO tile)ᵀ over D
       auto issue_xt = [&](uint64_t da0, uint64_t db0, uint32_t dtm) {
@@ -325,55 +395,72 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int kk = 0; kk < C::BR / 16; ++kk)
           mma_ts_w(dtm, atm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
       };
-      // dQᵀ [128 d-rows x 64 queries] = K[:, dh half]ᵀ · dSᵀ over the 128 keys
-      auto issue_dq = [&]() {
+      auto stage_bytes = [&](int g) -> uint32_t { return (uint32_t)(g % C::NSTAGE) * C::Q_BYTES; };
+      auto q_off = [&](int g) -> uint64_t { return sdesc_add(dQ_k, stage_bytes(g)); };
+      auto do_off = [&](int g) -> uint64_t { return sdesc_add(dDO_k, stage_bytes(g)); };
+      int gs = 0;
+      for (int uc = 0; ok; ++uc) {
+        const int idx = next_unit(uc);
+        if (idx < 0) { ok = false; break; }
+        if (idx >= p.n_units) break;
+        const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+        const int n = u.n;
+        const uint64_t dQ_mn = sdesc_sw128(sbase + C::Q_OFF + (u.dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
+        const uint64_t dDO_mn = sdesc_sw128(sbase + C::DO_OFF + (u.dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
+        const uint64_t dKT_mn = sdesc_sw128(sbase + C::K_OFF + (u.dh * C::DH / 64) * C::KV_PANEL, C::KV_PANEL, 1024);
+        // dQᵀ [128 d-rows x 64 queries] = K[:, dh half]ᵀ · dSᵀ over the 128 keys
+        auto issue_dq = [&]() {
 #pragma unroll
-        for (int kk = 0; kk < C::BC / 16; ++kk)
-          mma_ss_w(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
-                 kk > 0 ? 1u : 0u);
-      };
-      auto stage_bytes = [&](int s) -> uint32_t { return (uint32_t)(s % C::NSTAGE) * C::Q_BYTES; };
-      auto q_off = [&](int s) -> uint64_t { return sdesc_add(dQ_k, stage_bytes(s)); };
-      auto do_off = [&](int s) -> uint64_t { return sdesc_add(dDO_k, stage_bytes(s)); };
-      if (ok) {
+          for (int kk = 0; kk < C::BC / 16; ++kk)
+            mma_ss_w(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
+                   kk > 0 ? 1u : 0u);
+        };
+        if (!mbar_wait_warp(BAR(C::B_KVFULL), uc & 1, wc, 12)) { ok = false; break; }
+        tc_fence_after();
         for (int k = 0; k < C::LA && k < n && ok; ++k) {
-          ok = wait_q(k);
+          ok = wait_q(gs + k);
           if (!ok) break;
-          issue_xt(dK_k, q_off(k), tbase + C::ST_COL + 64 * (k & 1));
-          tc_commit_w(BAR(C::B_SFULL + (k & 1)));
+          issue_xt(dK_k, q_off(gs + k), tbase + C::ST_COL + 64 * ((gs + k) & 1));
+          tc_commit_w(BAR(C::B_SFULL + ((gs + k) & 1)));
         }
-        if (ok) {
-          issue_xt(dV_k, do_off(0), tbase + C::DP_COL);
-          tc_commit_w(BAR(C::B_DPFULL));
-        }
+        if (!ok) break;
+        issue_xt(dV_k, do_off(gs), tbase + C::DP_COL);
+        tc_commit_w(BAR(C::B_DPFULL));
         for (int s = 0; s < n && ok; ++s) {
-          if (!mbar_wait_warp(BAR(C::B_PFULL + (s & 1)), (s >> 1) & 1, wc, 14)) { ok = false; break; }
+          const int g = gs + s;
+          if (!mbar_wait_warp(BAR(C::B_PFULL + (g & 1)), (g >> 1) & 1, wc, 14)) { ok = false; break; }
+          // the previous unit's dV must have been read out before it is overwritten
+          if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DVFREE), (uc - 1) & 1, wc, 19)) { ok = false; break; }
           tc_fence_after();
-          issue_acc(tbase + C::ST_COL + 64 * (s & 1), sdesc_add(dDO_mn, stage_bytes(s)), tbase + C::DV_COL, s == 0);
-          if (!mbar_wait_warp(BAR(C::B_DSFULL), s & 1, wc, 15)) { ok = false; break; }
+          issue_acc(tbase + C::ST_COL + 64 * (g & 1), sdesc_add(dDO_mn, stage_bytes(g)), tbase + C::DV_COL, s == 0);
+          if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
+          if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
           tc_fence_after();
-          issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(s)), tbase + C::DK_COL, s == 0);
-          tc_commit_w(BAR(C::B_QEMPTY + s % C::NSTAGE));
-          if (s > 0) {
-            if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (s - 1) & 1, wc, 16)) { ok = false; break; }
+          issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(g)), tbase + C::DK_COL, s == 0);
+          tc_commit_w(BAR(C::B_QEMPTY + g % C::NSTAGE));
+          if (g > 0) {
+            if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
             tc_fence_after();
           }
           issue_dq();
           tc_commit_w(BAR(C::B_DQFULL));
           // dPᵀ of the next step first: the compute warps are waiting for it
           if (s + 1 < n) {
-            if (C::LA == 1 && !wait_q(s + 1)) { ok = false; break; }
-            issue_xt(dV_k, do_off(s + 1), tbase + C::DP_COL);
+            if (C::LA == 1 && !wait_q(g + 1)) { ok = false; break; }
+            issue_xt(dV_k, do_off(g + 1), tbase + C::DP_COL);
             tc_commit_w(BAR(C::B_DPFULL));
           }
           if (s + C::LA < n) {
-            const int s2 = s + C::LA;
-            if (C::LA > 1 && !wait_q(s2)) { ok = false; break; }
-            issue_xt(dK_k, q_off(s2), tbase + C::ST_COL + 64 * (s2 & 1));
-            tc_commit_w(BAR(C::B_SFULL + (s2 & 1)));
+            const int g2 = g + C::LA;
+            if (C::LA > 1 && !wait_q(g2)) { ok = false; break; }
+            issue_xt(dK_k, q_off(g2), tbase + C::ST_COL + 64 * (g2 & 1));
+            tc_commit_w(BAR(C::B_SFULL + (g2 & 1)));
           }
         }
-        if (ok) tc_commit_w(BAR(C::B_ACC));
+        if (!ok) break;
+        tc_commit_w(BAR(C::B_ACC));      // this unit's dK, dV are complete
+        tc_commit_w(BAR(C::B_KVEMPTY));  // and nothing reads its K, V any more
+        gs += n;
       }
       tc_commit_w(BAR(C::B_DRAIN));
       mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 17);
@@ -386,97 +473,111 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     if (C::REG_SPLIT) setmaxnreg_inc<C::COMPUTE_REGS>();
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row within the tile
-    const int key = jt * C::BC + r;
     const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
     const float sl2 = p.scale_log2;
     bool ok = true;
-    for (int s = 0; s < n; ++s) {
-      const int st = s % C::NSTAGE;
-      const int q0 = step_q0(s);
-      if (!mbar_wait_warp(BAR(C::B_QFULL + st), (s / C::NSTAGE) & 1, wc, 21)) { ok = false; break; }
-      if (!mbar_wait_warp(BAR(C::B_SFULL + (s & 1)), (s >> 1) & 1, wc, 22)) { ok = false; break; }
-      tc_fence_after();
-      const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512);
-      const float* dv = lse2 + 64;
-      uint32_t x0[32], x1[32];
-      const int scol = C::ST_COL + 64 * (s & 1);
-      tmem_ld32(tl + scol, x0);
-      tmem_ld32(tl + scol + 32, x1);
-      tmem_ld_wait();
-      reg_fence(x0);
-      reg_fence(x1);
-      float pr[64];
-      const bool diag = CAUSAL && (q0 < jt * C::BC + C::BC);
-#pragma unroll
-      for (int c = 0; c < 32; ++c) {
-        pr[c] = ex2(fmaf(__uint_as_float(x0[c]), sl2, -lse2[c]));
-        pr[32 + c] = ex2(fmaf(__uint_as_float(x1[c]), sl2, -lse2[32 + c]));
-      }
-      if (diag) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (key > q0 + c) pr[c] = 0.f;
-      }
-      // ragged N: keys and queries past the end of the sequence contribute nothing
-      if (TAIL && (key >= p.N || q0 + C::BR > p.N)) {
-#pragma unroll
-        for (int c = 0; c < 64; ++c)
-          if (key >= p.N || q0 + c >= p.N) pr[c] = 0.f;
-      }
-      uint32_t pk[32];
-#pragma unroll
-      for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-      tmem_st32(tl + scol, pk);
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_PFULL + (s & 1)));
-
-      if (!mbar_wait_warp(BAR(C::B_DPFULL), s & 1, wc, 23)) { ok = false; break; }
-      // the previous dQᵀ product must be done reading the dSᵀ tile in smem
-      if (s > 0 && !mbar_wait_warp(BAR(C::B_DQFULL), (s - 1) & 1, wc, 24)) { ok = false; break; }
-      tc_fence_after();
-      uint8_t* rowp = smem + C::DS_OFF + r * 128;
-      // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: bf16 over the
-      // consumed dPᵀ columns (A operand of dK) and into the smem tile (dQᵀ)
-#pragma unroll
-      for (int hf = 0; hf < 2; ++hf) {
-        tmem_ld32(tl + C::DP_COL + 32 * hf, x0);
+    int gs = 0;
+    for (int uc = 0; ok; ++uc) {
+      const int idx = next_unit(uc);
+      if (idx < 0) { ok = false; break; }
+      if (idx >= p.n_units) break;
+      const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+      const int key = u.jt * C::BC + r;
+      for (int s = 0; s < u.n; ++s) {
+        const int g = gs + s;
+        const int st = g % C::NSTAGE;
+        const int q0 = step_q0(u, s);
+        if (!mbar_wait_warp(BAR(C::B_QFULL + st), (g / C::NSTAGE) & 1, wc, 21)) { ok = false; break; }
+        if (!mbar_wait_warp(BAR(C::B_SFULL + (g & 1)), (g >> 1) & 1, wc, 22)) { ok = false; break; }
+        tc_fence_after();
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512);
+        const float* dv = lse2 + 64;
+        uint32_t x0[32], x1[32];
+        const int scol = C::ST_COL + 64 * (g & 1);
+        tmem_ld32(tl + scol, x0);
+        tmem_ld32(tl + scol + 32, x1);
         tmem_ld_wait();
         reg_fence(x0);
-        uint32_t dk16[16];
+        reg_fence(x1);
+        float pr[64];
+        const bool diag = CAUSAL && (q0 < u.jt * C::BC + C::BC);
 #pragma unroll
-        for (int c = 0; c < 16; ++c) {
-          const int q = 32 * hf + 2 * c;
-          const float d0 = pr[q] * (__uint_as_float(x0[2 * c]) - dv[q]);
-          const float d1 = pr[q + 1] * (__uint_as_float(x0[2 * c + 1]) - dv[q + 1]);
-          dk16[c] = pack_bf16(d0, d1);
+        for (int c = 0; c < 32; ++c) {
+          pr[c] = ex2(fmaf(__uint_as_float(x0[c]), sl2, -lse2[c]));
+          pr[32 + c] = ex2(fmaf(__uint_as_float(x1[c]), sl2, -lse2[32 + c]));
         }
-        tmem_st16(tl + C::DP_COL + 16 * hf, dk16);
+        if (diag) {
 #pragma unroll
-        for (int ch = 0; ch < 4; ++ch) {
-          const int lch = 4 * hf + ch;
-          const uint4 v = make_uint4(dk16[4 * ch], dk16[4 * ch + 1], dk16[4 * ch + 2], dk16[4 * ch + 3]);
-          *reinterpret_cast<uint4*>(rowp + ((lch ^ (r & 7)) * 16)) = v;
+          for (int c = 0; c < 64; ++c)
+            if (key > q0 + c) pr[c] = 0.f;
         }
+        // ragged N: keys and queries past the end of the sequence contribute nothing
+        if (TAIL && (key >= p.N || q0 + C::BR > p.N)) {
+#pragma unroll
+          for (int c = 0; c < 64; ++c)
+            if (key >= p.N || q0 + c >= p.N) pr[c] = 0.f;
+        }
+        uint32_t pk[32];
+#pragma unroll
+        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+        tmem_st32(tl + scol, pk);
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_PFULL + (g & 1)));
+
+        if (!mbar_wait_warp(BAR(C::B_DPFULL), g & 1, wc, 23)) { ok = false; break; }
+        // the previous dQᵀ product must be done reading the dSᵀ tile in smem
+        if (g > 0 && !mbar_wait_warp(BAR(C::B_DQFULL), (g - 1) & 1, wc, 24)) { ok = false; break; }
+        tc_fence_after();
+        uint8_t* rowp = smem + C::DS_OFF + r * 128;
+        // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: bf16 over the
+        // consumed dPᵀ columns (A operand of dK) and into the smem tile (dQᵀ)
+#pragma unroll
+        for (int hf = 0; hf < 2; ++hf) {
+          tmem_ld32(tl + C::DP_COL + 32 * hf, x0);
+          tmem_ld_wait();
+          reg_fence(x0);
+          uint32_t dk16[16];
+#pragma unroll
+          for (int c = 0; c < 16; ++c) {
+            const int q = 32 * hf + 2 * c;
+            const float d0 = pr[q] * (__uint_as_float(x0[2 * c]) - dv[q]);
+            const float d1 = pr[q + 1] * (__uint_as_float(x0[2 * c + 1]) - dv[q + 1]);
+            dk16[c] = pack_bf16(d0, d1);
+          }
+          tmem_st16(tl + C::DP_COL + 16 * hf, dk16);
+#pragma unroll
+          for (int ch = 0; ch < 4; ++ch) {
+            const int lch = 4 * hf + ch;
+            const uint4 v = make_uint4(dk16[4 * ch], dk16[4 * ch + 1], dk16[4 * ch + 2], dk16[4 * ch + 3]);
+            *reinterpret_cast<uint4*>(rowp + ((lch ^ (r & 7)) * 16)) = v;
+          }
+        }
+        fence_proxy_async_smem();
+        tmem_st_wait();
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_DSFULL));
       }
-      fence_proxy_async_smem();
-      tmem_st_wait();
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_DSFULL));
-    }
-    // dK epilogue (scaled by s)
-    // (tcgen05.ld is warp-collective: every lane loads, only rows < N are stored)
-    if (ok && mbar_wait_warp(BAR(C::B_ACC), 0, wc, 25)) {
+      if (!ok) break;
+      // dK epilogue (scaled by s); tcgen05.ld is warp-collective: every lane
+      // loads, only rows < N are stored
+      if (!mbar_wait_warp(BAR(C::B_ACC), uc & 1, wc, 25)) { ok = false; break; }
       tc_fence_after();
-      __nv_bfloat16* dst = p.dk + ((size_t)(b * p.Hkv + hkv) * p.N + key) * D + dh * C::DH;
+      __nv_bfloat16* dst = p.dk + ((size_t)(u.b * p.Hkv + u.hkv) * p.N + key) * D + u.dh * C::DH;
 #pragma unroll
       for (int oc = 0; oc < C::DH / 32; ++oc) {
         uint32_t v[32];
         tmem_ld32(tl + C::DK_COL + oc * 32, v);
         tmem_ld_wait();
         reg_fence(v);
+        if (oc == C::DH / 32 - 1) {
+          // dK has been read out of TMEM: the next unit may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(C::B_DKFREE));
+        }
         uint32_t w[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c)
@@ -487,6 +588,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
         }
       }
+      gs += u.n;
     }
     tc_fence_before();
   } else if (warp >= 8) {
@@ -500,65 +602,80 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     if (dt == 0) tma_prefetch_desc(&tmDQ);
     bool ok = true;
     int sub_seq = 0;  // staging uses so far
-    for (int s = 0; s < n && ok; ++s) {
-      if (!mbar_wait_warp(BAR(C::B_DQFULL), s & 1, wc, 31)) { ok = false; break; }
-      tc_fence_after();
-      uint32_t x0[32], x1[32];
-      tmem_ld32(tl + C::DQ_COL, x0);
-      tmem_ld32(tl + C::DQ_COL + 32, x1);
-      tmem_ld_wait();
-      reg_fence(x0);
-      reg_fence(x1);
-      tc_fence_before();
-      __syncwarp();
-      if (lane == 0) mbar_arrive(BAR(C::B_DQEMPTY));
-      const int q_row = (b * p.Hq + step_head(s)) * p.Np + step_q0(s);  // padded accumulator row
+    int gs = 0;
+    for (int uc = 0; ok; ++uc) {
+      const int idx = next_unit(uc);
+      if (idx < 0) { ok = false; break; }
+      if (idx >= p.n_units) break;
+      const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+      for (int s = 0; s < u.n && ok; ++s) {
+        const int g = gs + s;
+        if (!mbar_wait_warp(BAR(C::B_DQFULL), g & 1, wc, 31)) { ok = false; break; }
+        tc_fence_after();
+        uint32_t x0[32], x1[32];
+        tmem_ld32(tl + C::DQ_COL, x0);
+        tmem_ld32(tl + C::DQ_COL + 32, x1);
+        tmem_ld_wait();
+        reg_fence(x0);
+        reg_fence(x1);
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_DQEMPTY));
+        const int q_row = (u.b * p.Hq + step_head(u, s)) * p.Np + step_q0(u, s);  // padded accumulator row
 #pragma unroll
-      for (int sub = 0; sub < 64 / C::STG_ROWS; ++sub) {
-        // the previous reduce must have finished reading the staging tile
-        if (dt == 0) {
-          bulk_wait_read_all();
-          mbar_arrive(BAR(C::B_STGFREE));
-        }
-        if (!mbar_wait_warp(BAR(C::B_STGFREE), sub_seq & 1, wc, 33)) { ok = false; break; }
-        if (r < C::DH) {
-#pragma unroll
-          for (int qq = 0; qq < C::STG_ROWS; ++qq) {
-            const int c = sub * C::STG_ROWS + qq;
-            stg[qq * C::DH + r] = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
+        for (int sub = 0; sub < 64 / C::STG_ROWS; ++sub) {
+          // the previous reduce must have finished reading the staging tile
+          if (dt == 0) {
+            bulk_wait_read_all();
+            mbar_arrive(BAR(C::B_STGFREE));
           }
+          if (!mbar_wait_warp(BAR(C::B_STGFREE), sub_seq & 1, wc, 33)) { ok = false; break; }
+          if (r < C::DH) {
+#pragma unroll
+            for (int qq = 0; qq < C::STG_ROWS; ++qq) {
+              const int c = sub * C::STG_ROWS + qq;
+              stg[qq * C::DH + r] = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
+            }
+          }
+          fence_proxy_async_smem();
+          mbar_arrive(BAR(C::B_STGFULL));
+          if (dt == 0) {
+            if (!mbar_wait(BAR(C::B_STGFULL), sub_seq & 1, wc, 34)) { ok = false; break; }
+            tma_reduce_add_2d(&tmDQ, sbase + C::STG_OFF, u.dh * C::DH, q_row + sub * C::STG_ROWS);
+            bulk_commit_group();
+          }
+          ++sub_seq;
         }
-        fence_proxy_async_smem();
-        mbar_arrive(BAR(C::B_STGFULL));
-        if (dt == 0) {
-          if (!mbar_wait(BAR(C::B_STGFULL), sub_seq & 1, wc, 34)) { ok = false; break; }
-          tma_reduce_add_2d(&tmDQ, sbase + C::STG_OFF, dh * C::DH, q_row + sub * C::STG_ROWS);
-          bulk_commit_group();
-        }
-        ++sub_seq;
       }
-    }
-    if (dt == 0) bulk_wait_all();
-    // dV epilogue
-    if (ok && mbar_wait_warp(BAR(C::B_ACC), 0, wc, 32)) {
+      if (!ok) break;
+      // dV epilogue
+      if (!mbar_wait_warp(BAR(C::B_ACC), uc & 1, wc, 32)) { ok = false; break; }
       tc_fence_after();
-      __nv_bfloat16* dst = p.dv + ((size_t)(b * p.Hkv + hkv) * p.N + jt * C::BC + r) * D + dh * C::DH;
+      __nv_bfloat16* dst = p.dv + ((size_t)(u.b * p.Hkv + u.hkv) * p.N + u.jt * C::BC + r) * D + u.dh * C::DH;
 #pragma unroll
       for (int oc = 0; oc < C::DH / 32; ++oc) {
         uint32_t v[32];
         tmem_ld32(tl + C::DV_COL + oc * 32, v);
         tmem_ld_wait();
         reg_fence(v);
+        if (oc == C::DH / 32 - 1) {
+          // dV has been read out of TMEM: the next unit may overwrite it
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(C::B_DVFREE));
+        }
         uint32_t w[16];
 #pragma unroll
         for (int c = 0; c < 16; ++c) w[c] = pack_bf16(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
         uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
-        if (!TAIL || jt * C::BC + r < p.N) {
+        if (!TAIL || u.jt * C::BC + r < p.N) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
         }
       }
+      gs += u.n;
     }
+    if (dt == 0) bulk_wait_all();
     tc_fence_before();
   }
 

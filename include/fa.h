@@ -73,7 +73,8 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
 /* Bytes of device workspace fa_bwd needs: two fp32 [B,Hq,Np] row vectors
  * (D = rowsum(dO∘O) and LSE·log2 e) and an fp32 [B,Hq,Np,d] dQ accumulator,
  * each rounded up to 256 bytes, where Np = N rounded up to a multiple of 128
- * (per-head padding rows keep every tile aligned and private to its head).
+ * (per-head padding rows keep every tile aligned and private to its head),
+ * plus 256 bytes for the counter the main kernel's CTAs claim work from.
  * Returns 0 for invalid sizes. */
 size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
 
@@ -162,9 +163,9 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
  * exits.  Nothing is allocated or freed per call.
  *
  * Limit: the problem's fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) must not
- * exceed FA_NOALLOC_SCRATCH_BYTES (for d = 128 that is B·Hq·Np ≤ 129,055
- * padded query rows); larger problems return FA_ERR_UNSUPPORTED and enqueue
- * nothing.
+ * exceed FA_NOALLOC_SCRATCH_BYTES (for d = 128 that is B·Hq·Np ≤ 129,024
+ * padded query rows, i.e. 1008 heads of up to 128 rows); larger problems
+ * return FA_ERR_UNSUPPORTED and enqueue nothing.
  *
  * Set-up: the first call on each device, with that device current, looks up
  * the array's device address (cudaGetSymbolAddress).  Make that first call

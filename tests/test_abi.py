@@ -46,14 +46,15 @@ def test_status_strings(lib):
 
 def test_workspace_bytes_formula(lib):
     # two fp32 row vectors and an fp32 [B,Hq,Np,d] accumulator, each 256-rounded,
-    # with Np = N rounded up to a multiple of 128 (per-head padding rows)
+    # with Np = N rounded up to a multiple of 128 (per-head padding rows), and
+    # 256 bytes for the main kernel's unit counter
     B, Hq, Hkv, N, d = 8, 16, 16, 2048, 128
     rows = B * Hq * N
-    assert binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) == 2 * rows * 4 + rows * d * 4
-    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 128, 64) == 2 * 512 + 128 * 64 * 4
-    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 100, 64) == 2 * 512 + 128 * 64 * 4
-    assert binding.fa_bwd_workspace_bytes(2, 3, 1, 129, 256) == 2 * 1536 * 4 + 1536 * 256 * 4
-    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 1, 128) == 2 * 512 + 128 * 128 * 4
+    assert binding.fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) == 2 * rows * 4 + rows * d * 4 + 256
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 128, 64) == 2 * 512 + 128 * 64 * 4 + 256
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 100, 64) == 2 * 512 + 128 * 64 * 4 + 256
+    assert binding.fa_bwd_workspace_bytes(2, 3, 1, 129, 256) == 2 * 1536 * 4 + 1536 * 256 * 4 + 256
+    assert binding.fa_bwd_workspace_bytes(1, 1, 1, 1, 128) == 2 * 512 + 128 * 128 * 4 + 256
     assert binding.fa_bwd_workspace_bytes(1, 3, 2, 128, 64) == 0      # Hq % Hkv != 0
     assert binding.fa_bwd_workspace_bytes(1, 2, 2, 128, 96) == 0      # unsupported d
 
