@@ -1,0 +1,526 @@
+"""Randomised models of the mbarrier protocols of the two persistent attention
+kernels (fa_fwd_persistent_kernel, fa_bwd_kernel), run on the CPU.
+
+Each warp role of a kernel is a Python generator that performs the role's
+waits, arrivals and issues in the kernel's order.  A scheduler picks one role,
+the tensor pipe (which completes issued products and their commits in order)
+or the TMA engine (which completes loads in order) at a time, with per-role
+speeds drawn over three decades so that some roles lag far behind others.
+
+An mbarrier wait with parity bit b passes when the barrier's completed-phase
+count has the other parity; the model asserts that every wait passes exactly
+when its intended phase is the most recently completed one.  A role more than
+one phase behind would pass on a stale phase in hardware; the model reports it
+as "run-ahead".  It also asserts that buffers (Q stages, K/V slots, unit-index
+slots, TMEM accumulators) are refilled only after their last reader finished,
+that no schedule deadlocks, and that every unit of work is done exactly once.
+
+The models carry no attention arithmetic; a planted-mistake test for each
+shows that a missing wait is caught.
+"""
+
+import random
+
+import pytest
+
+
+class _Bar:
+    def __init__(self, count):
+        self.count, self.arrived, self.phases = count, 0, 0
+
+    def arrive(self):
+        self.arrived += 1
+        assert self.arrived <= self.count
+        if self.arrived == self.count:
+            self.arrived = 0
+            self.phases += 1
+
+
+def _waiter(bars):
+    def wait(name, k):
+        """Wait for the completion of phase k (0-based) of barrier ``name``."""
+        b = bars[name]
+        while True:
+            if (b.phases & 1) != (k & 1):
+                assert b.phases == k + 1, f"ambiguous pass {name}: wanted phase {k}, {b.phases} done"
+                return
+            if b.phases >= k + 2:
+                raise AssertionError(f"run-ahead {name}: wanted phase {k}, {b.phases} done")
+            yield
+    return wait
+
+
+def _run(gens, engines, rnd, max_steps=20_000_000):
+    """Drive role generators and in-order engines ({key: (queue, complete_fn)})
+    at random per-role speeds until all are finished."""
+    alive = dict(gens)
+    speed = {k: 10 ** rnd.uniform(-3, 0) for k in list(gens) + list(engines)}
+    steps = 0
+    while True:
+        choices = list(alive) + [k for k, (q, _) in engines.items() if q]
+        if not choices:
+            return
+        steps += 1
+        assert steps < max_steps, "deadlock"
+        ch = rnd.choices(choices, weights=[speed[c] for c in choices])[0]
+        if ch in engines:
+            q, complete = engines[ch]
+            complete(q.pop(0))
+        else:
+            try:
+                next(alive[ch])
+            except StopIteration:
+                del alive[ch]
+
+
+# ---------------------------------------------------------------- backward
+def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
+    """fa_bwd_kernel: ``n_ctas`` persistent CTAs claim units (``unit_len[i]`` query
+    steps each) from one counter.  Roles per CTA: the producer (lane 0 of warp
+    0), the MMA warp, four compute warps and four drain warps.  ``lookahead`` is
+    how many Sᵀ products run ahead (2 with several Q/dO stages, 1 with one)."""
+    rnd = random.Random(seed)
+    counter = [0]
+    done_units = []
+    gens, engines = {}, {}
+
+    def make_cta(c):
+        bars = {}
+        for nm in ("KVFULL", "KVEMPTY", "DPFULL", "DQFULL", "ACC"):
+            bars[nm] = _Bar(1)
+        for nm in ("DSFULL", "DQEMPTY", "DKFREE", "DVFREE"):
+            bars[nm] = _Bar(4)
+        for i in range(n_stage):
+            bars["QFULL", i] = _Bar(1)
+            bars["QEMPTY", i] = _Bar(1)
+        for i in range(2):
+            bars["SFULL", i] = _Bar(1)
+            bars["PFULL", i] = _Bar(4)
+            bars["UNITFULL", i] = _Bar(1)
+            bars["UNITEMPTY", i] = _Bar(9)
+        wait = _waiter(bars)
+        tc, tma = [], []            # in-order queues: tensor pipe, TMA
+        completed = set()           # finished products
+        loaded = set()              # finished loads
+        slot = [None, None]         # unit-index ring
+        slot_readers = [set(), set()]
+        kv_readers, stage_readers, acc_writers = {}, {}, {}
+        acc_read = {}               # (kind, uc) -> warps that read it out
+        prod_id = [0]
+
+        def issue(kind, uc, g):
+            prod_id[0] += 1
+            i = prod_id[0]
+            tc.append(("mma", i))
+            if kind in ("S", "dP", "dQ"):
+                kv_readers.setdefault(uc, set()).add(i)
+            if kind in ("S", "dP", "dV", "dK"):
+                stage_readers.setdefault(g, set()).add(i)
+            if kind in ("dV", "dK"):
+                acc_writers.setdefault(uc, set()).add(i)
+                if uc > 0:
+                    assert acc_read.get((kind, uc - 1), 0) == 4, f"{kind} of unit {uc} overwrites unread TMEM"
+
+        def commit(name):
+            tc.append(("commit", name))
+
+        def next_unit(uc, who):
+            yield from wait(("UNITFULL", uc & 1), uc >> 1)
+            entry = slot[uc & 1]
+            assert entry is not None and entry[0] == uc, f"{who} read slot of unit {entry} for {uc}"
+            assert who not in slot_readers[uc & 1]
+            slot_readers[uc & 1].add(who)
+            yield
+            bars["UNITEMPTY", uc & 1].arrive()
+            return entry[1]
+
+        def producer():
+            gs = uc = 0
+            while True:
+                idx = counter[0]
+                counter[0] += 1
+                yield
+                if uc >= 2 and mistake != "no_unit_empty_wait":
+                    yield from wait(("UNITEMPTY", uc & 1), (uc >> 1) - 1)
+                    assert len(slot_readers[uc & 1]) == 9
+                slot[uc & 1] = (uc, idx)
+                slot_readers[uc & 1] = set()
+                bars["UNITFULL", uc & 1].arrive()
+                if idx >= len(unit_len):
+                    return
+                n = unit_len[idx]
+
+                def load_q(s):
+                    g = gs + s
+                    if g >= n_stage:
+                        yield from wait(("QEMPTY", g % n_stage), g // n_stage - 1)
+                        assert stage_readers.get(g - n_stage, set()) <= completed, f"stage of step {g} reused"
+                    tma.append((("QFULL", g % n_stage), ("Q", g)))
+                pre = min(n_stage, n)
+                for s in range(pre):
+                    yield from load_q(s)
+                if uc > 0:
+                    yield from wait("KVEMPTY", uc - 1)
+                    assert kv_readers.get(uc - 1, set()) <= completed, "K/V reloaded while read"
+                tma.append(("KVFULL", ("KV", uc)))
+                for s in range(pre, n):
+                    yield from load_q(s)
+                gs += n
+                uc += 1
+
+        def mma():
+            gs = uc = 0
+            while True:
+                idx = yield from next_unit(uc, "mma")
+                if idx >= len(unit_len):
+                    return
+                n = unit_len[idx]
+                yield from wait("KVFULL", uc)
+                assert ("KV", uc) in loaded
+
+                def wait_q(g):
+                    yield from wait(("QFULL", g % n_stage), g // n_stage)
+                    assert ("Q", g) in loaded
+                for k in range(min(lookahead, n)):
+                    yield from wait_q(gs + k)
+                    issue("S", uc, gs + k)
+                    commit(("SFULL", (gs + k) & 1))
+                issue("dP", uc, gs)
+                commit("DPFULL")
+                for s in range(n):
+                    g = gs + s
+                    yield from wait(("PFULL", g & 1), g >> 1)
+                    if s == 0 and uc > 0 and mistake != "no_dvfree_wait":
+                        yield from wait("DVFREE", uc - 1)
+                    issue("dV", uc, g)
+                    yield from wait("DSFULL", g)
+                    if s == 0 and uc > 0:
+                        yield from wait("DKFREE", uc - 1)
+                    issue("dK", uc, g)
+                    commit(("QEMPTY", g % n_stage))
+                    if g > 0:
+                        yield from wait("DQEMPTY", g - 1)
+                    issue("dQ", uc, g)
+                    commit("DQFULL")
+                    if s + 1 < n:
+                        if lookahead == 1:
+                            yield from wait_q(g + 1)
+                        issue("dP", uc, g + 1)
+                        commit("DPFULL")
+                    if s + lookahead < n:
+                        g2 = g + lookahead
+                        if lookahead > 1:
+                            yield from wait_q(g2)
+                        issue("S", uc, g2)
+                        commit(("SFULL", g2 & 1))
+                commit("ACC")
+                commit("KVEMPTY")
+                done_units.append(idx)
+                gs += n
+                uc += 1
+
+        def epilogue_warp(w, kind, free_bar):
+            # compute warps (kind "dK") or drain warps (kind "dV")
+            gs = uc = 0
+            while True:
+                idx = yield from next_unit(uc, (kind, w))
+                if idx >= len(unit_len):
+                    return
+                n = unit_len[idx]
+                for s in range(n):
+                    g = gs + s
+                    if kind == "dK":
+                        yield from wait(("QFULL", g % n_stage), g // n_stage)
+                        yield from wait(("SFULL", g & 1), g >> 1)
+                        yield
+                        bars["PFULL", g & 1].arrive()
+                        yield from wait("DPFULL", g)
+                        if g > 0:
+                            yield from wait("DQFULL", g - 1)
+                        yield
+                        bars["DSFULL"].arrive()
+                    else:
+                        yield from wait("DQFULL", g)
+                        yield
+                        bars["DQEMPTY"].arrive()
+                yield from wait("ACC", uc)
+                assert acc_writers.get(uc, set()) <= completed
+                yield
+                acc_read[kind, uc] = acc_read.get((kind, uc), 0) + 1
+                bars[free_bar].arrive()
+                gs += n
+                uc += 1
+
+        def tc_done(item):
+            kind, x = item
+            if kind == "commit":
+                bars[x].arrive()
+            else:
+                completed.add(x)
+
+        def tma_done(item):
+            bar, what = item
+            loaded.add(what)
+            bars[bar].arrive()
+
+        gens[c, "producer"] = producer()
+        gens[c, "mma"] = mma()
+        for w in range(4):
+            gens[c, "compute", w] = epilogue_warp(w, "dK", "DKFREE")
+            gens[c, "drain", w] = epilogue_warp(w, "dV", "DVFREE")
+        engines[c, "tc"] = (tc, tc_done)
+        engines[c, "tma"] = (tma, tma_done)
+
+    for c in range(n_ctas):
+        make_cta(c)
+    _run(gens, engines, rnd)
+    assert sorted(done_units) == list(range(len(unit_len))), "units lost or repeated"
+    assert counter[0] == len(unit_len) + n_ctas
+
+
+BWD_UNITS = ([1], [3, 1], [1, 1, 1, 1, 1], [5, 2, 8], [1, 7, 2, 1, 3], [2, 1, 3, 1, 1, 2, 5, 1])
+
+
+@pytest.mark.parametrize("n_stage,lookahead", [(3, 2), (1, 1)])
+@pytest.mark.parametrize("n_ctas", [1, 3])
+def test_backward_protocol(n_stage, lookahead, n_ctas):
+    for units in BWD_UNITS:
+        for seed in range(4):
+            simulate_bwd(units, n_ctas, n_stage, lookahead, seed)
+
+
+@pytest.mark.parametrize("mistake", ["no_unit_empty_wait", "no_dvfree_wait"])
+def test_backward_model_catches_a_missing_wait(mistake):
+    caught = 0
+    for seed in range(40):
+        try:
+            simulate_bwd([1, 1, 1, 1, 1, 1], 2, 3, 2, seed, mistake)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+# ----------------------------------------------------------------- forward
+def simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed, mistake=None):
+    """fa_fwd_persistent_kernel: items are pairs of 128-row query tiles of one
+    (b, h), dealt to ``n_ctas`` CTAs in a fixed order.  Roles per CTA: the
+    producer, the MMA warp and the two softmax warpgroups (one per query
+    tile).  K and V blocks are separate "units" streamed through ``n_slot``
+    slots; with a causal mask the second tile's diagonal block comes first."""
+    rnd = random.Random(seed)
+    n_pairs = (n_qtiles + 1) // 2
+    n_items = n_pairs * BH
+    issued = {"S": [], "PV": []}
+
+    def item(idx):
+        if causal:
+            pair, bh = n_pairs - 1 - idx // BH, idx % BH
+        else:
+            bh, pair = idx // n_pairs, idx % n_pairs
+        qt0 = 2 * pair
+        has1 = qt0 + 1 < n_qtiles
+        n0 = qt0 + 1 if causal else n_qtiles
+        n1 = (qt0 + 2 if causal else n_qtiles) if has1 else 0
+        skew = 1 if (causal and has1) else 0
+        return dict(qt0=qt0, n0=n0, n1=n1, skew=skew, nit=n0 + skew)
+
+    def kv_block(w, jj):
+        return w["qt0"] + 1 if (w["skew"] and jj == 0) else jj - w["skew"]
+
+    def first(w, t):
+        return w["skew"] if t == 0 else 0
+
+    def has(w, t):
+        return t == 0 or w["n1"] > 0
+
+    def deal(k, c):
+        return k * n_ctas + ((n_ctas - 1 - c) if (causal and (k & 1)) else c)
+
+    n_rounds = (n_items + n_ctas - 1) // n_ctas
+    gens, engines = {}, {}
+    all_items = []
+
+    def make_cta(c):
+        items = [deal(k, c) for k in range(n_rounds) if deal(k, c) < n_items]
+        all_items.extend(items)
+        bars = {}
+        for t in range(2):
+            for nm in ("QFULL", "QEMPTY", "SFULL", "ODONE"):
+                bars[nm, t] = _Bar(1)
+            bars["PFULL", t] = _Bar(4)
+            bars["PFULL2", t] = _Bar(4)
+        for s in range(n_slot):
+            bars["KVFULL", s] = _Bar(1)
+            bars["KVEMPTY", s] = _Bar(1)
+        wait = _waiter(bars)
+        tc, tma = [], []
+        slot_unit, released, loaded = {}, set(), set()
+        q_tile = {0: None, 1: None}
+        readers = {}
+        unit_of = {}
+        u_acc = 0
+        for idx in items:
+            for u in range(2 * item(idx)["nit"]):
+                unit_of[u_acc + u] = (idx, u)
+            u_acc += 2 * item(idx)["nit"]
+
+        def producer():
+            useq = 0
+            q_loads = [0, 0]
+            for idx in items:
+                w = item(idx)
+                for t in range(2):
+                    if not has(w, t):
+                        continue
+                    if q_loads[t] > 0 and mistake != "no_qempty_wait":
+                        yield from wait(("QEMPTY", t), q_loads[t] - 1)
+                    q_tile[t] = (idx, t)
+                    tma.append((("QFULL", t), None))
+                    q_loads[t] += 1
+                for u in range(2 * w["nit"]):
+                    U = useq + u
+                    s = U % n_slot
+                    if U >= n_slot:
+                        yield from wait(("KVEMPTY", s), U // n_slot - 1)
+                    if s in slot_unit:
+                        assert slot_unit[s] in released, f"slot {s} refilled while unit {slot_unit[s]} is read"
+                    slot_unit[s] = U
+                    tma.append((("KVFULL", s), U))
+                useq += 2 * w["nit"]
+
+        def mma():
+            waited = [-1]
+            q_seen = [0, 0]
+            p_seen = [0, 0]
+
+            def wait_upto(U):
+                # K/V units are waited in load order, never skipping one
+                while waited[0] < U:
+                    waited[0] += 1
+                    yield from wait(("KVFULL", waited[0] % n_slot), waited[0] // n_slot)
+                    assert waited[0] in loaded
+
+            def release(U, w, jj, t_read):
+                readers.setdefault(U, set()).add(t_read)
+                if t_read == 1 or w["n1"] == 0:
+                    need = {t for t in range(2) if has(w, t) and jj >= first(w, t)}
+                    assert readers[U] == need
+                    released.add(U)
+                    tc.append(("commit", ("KVEMPTY", U % n_slot)))
+
+            def issue_s(t, w, idx, base, jj):
+                if jj == first(w, t):
+                    yield from wait(("QFULL", t), q_seen[t])
+                    q_seen[t] += 1
+                assert q_tile[t] == (idx, t), f"Q tile {t} overwritten: {q_tile[t]} for item {idx}"
+                U = base + 2 * jj
+                yield from wait_upto(U)
+                assert unit_of[U] == (idx, 2 * jj) and U not in released
+                issued["S"].append((idx, t, kv_block(w, jj)))
+                tc.append(("commit", ("SFULL", t)))
+                if jj == w["nit"] - 1:
+                    tc.append(("commit", ("QEMPTY", t)))
+                release(U, w, jj, t)
+
+            if not items:
+                return
+            idx, w, base = items[0], item(items[0]), 0
+            for t in range(2):
+                if has(w, t):
+                    yield from issue_s(t, w, idx, base, first(w, t))
+            for pos in range(len(items)):
+                nxt = items[pos + 1] if pos + 1 < len(items) else None
+                w2 = item(nxt) if nxt is not None else None
+                base2 = base + 2 * w["nit"]
+                for jj in range(w["nit"]):
+                    for t in range(2):
+                        if not has(w, t) or jj < first(w, t):
+                            continue
+                        Uv = base + 2 * jj + 1
+                        yield from wait(("PFULL", t), p_seen[t])
+                        yield from wait_upto(Uv)
+                        assert unit_of[Uv] == (idx, 2 * jj + 1) and Uv not in released
+                        yield from wait(("PFULL2", t), p_seen[t])
+                        issued["PV"].append((idx, t, kv_block(w, jj)))
+                        tc.append(("commit", ("ODONE", t)))
+                        p_seen[t] += 1
+                        release(Uv, w, jj, t)
+                        if jj + 1 < w["nit"]:
+                            yield from issue_s(t, w, idx, base, jj + 1)
+                        elif nxt is not None and has(w2, t):
+                            # the next item's first QKᵀ right after this tile's last PV
+                            yield from issue_s(t, w2, nxt, base2, first(w2, t))
+                if nxt is None:
+                    break
+                if not has(w, 1) and has(w2, 1):
+                    yield from issue_s(1, w2, nxt, base2, 0)
+                idx, w, base = nxt, w2, base2
+
+        def softmax(t):
+            done = 0
+            for idx in items:
+                w = item(idx)
+                if not has(w, t):
+                    continue
+                n = w["n0"] if t == 0 else w["n1"]
+                for j in range(n):
+                    yield from wait(("SFULL", t), done + j)
+                    if j > 0 and rnd.random() < 0.3:   # conditional rescale of O
+                        yield from wait(("ODONE", t), done + j - 1)
+                    for _ in range(4):
+                        bars["PFULL", t].arrive()
+                    yield
+                    for _ in range(4):
+                        bars["PFULL2", t].arrive()
+                yield from wait(("ODONE", t), done + n - 1)
+                done += n
+
+        def tc_done(entry):
+            bars[entry[1]].arrive()
+
+        def tma_done(entry):
+            bar, unit = entry
+            if unit is not None:
+                loaded.add(unit)
+            bars[bar].arrive()
+
+        gens[c, "producer"] = producer()
+        gens[c, "mma"] = mma()
+        gens[c, "softmax", 0] = softmax(0)
+        gens[c, "softmax", 1] = softmax(1)
+        engines[c, "tc"] = (tc, tc_done)
+        engines[c, "tma"] = (tma, tma_done)
+
+    for c in range(n_ctas):
+        make_cta(c)
+    _run(gens, engines, rnd)
+    assert sorted(all_items) == list(range(n_items))
+    # every query tile met exactly the K/V blocks the mask leaves visible, once each
+    for kind in ("S", "PV"):
+        got = sorted(issued[kind])
+        want = []
+        for idx in range(n_items):
+            w = item(idx)
+            for t in range(2):
+                if has(w, t):
+                    qt = w["qt0"] + t
+                    want += [(idx, t, j) for j in (range(qt + 1) if causal else range(n_qtiles))]
+        assert got == sorted(want), kind
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n_slot", [5, 8])
+def test_forward_protocol(causal, n_slot):
+    for n_qtiles in (1, 2, 3, 5, 8):
+        for BH, n_ctas in ((1, 1), (3, 2), (5, 3)):
+            simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed=n_qtiles * 7 + BH)
+
+
+def test_forward_model_catches_a_missing_wait():
+    caught = 0
+    for seed in range(20):
+        try:
+            simulate_fwd(4, 3, True, 1, 5, seed, mistake="no_qempty_wait")
+        except AssertionError:
+            caught += 1
+    assert caught > 0
