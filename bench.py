@@ -455,6 +455,26 @@ def _l2_note(*tensors) -> str:
     return f"inputs fit in L2 ({mib:.1f} MiB; not flushed: a small parity-sized case, not a bench line)"
 
 
+def logit_extremes(q, k, scale: float, causal: bool, rows_per_chunk: int = 2048):
+    """Largest |q·k| and |s·q·k| over every visible (query, key) pair of batch 0, query
+    head 0 (its kv head is 0), computed on the host in fp32 from the bf16 inputs.  A
+    record of how peaked the softmax rows are (the d = 256 workload's Q, K ~ N(0, 9)
+    is there to give raw logits far above 100)."""
+    import numpy as np
+    qh = q[0, 0].float().cpu().numpy()
+    kh = k[0, 0].float().cpu().numpy()
+    n = qh.shape[0]
+    best = 0.0
+    for r0 in range(0, n, rows_per_chunk):
+        s = qh[r0:r0 + rows_per_chunk] @ kh.T
+        if causal:
+            rows = np.arange(r0, min(n, r0 + rows_per_chunk))[:, None]
+            s = np.where(np.arange(n)[None, :] <= rows, s, 0.0)
+        best = max(best, float(np.abs(s).max()))
+    return {"max_abs_raw": best, "max_abs_scaled": best * scale,
+            "sample": "batch 0, query head 0, all visible (query, key) pairs, fp32 on the host"}
+
+
 def run_ours(args, w, rank, world, local_rank):
     import torch
     import torch.distributed as dist
@@ -608,6 +628,7 @@ def run_ours(args, w, rank, world, local_rank):
         "clocks": clocks,
     }
     if rank == 0:
+        line["logits"] = logit_extremes(q, k, scale, w.causal)
         print(json.dumps(line), flush=True)
 
 
