@@ -311,7 +311,10 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restr
 // Split plan of a decode call: row groups of RMAX (4, 8 or 16) query rows,
 // and enough key splits for about kDecodeCtas CTAs in all (a pure function of
 // the sizes, so that fa_decode_workspace_bytes needs no device).
-constexpr int kDecodeCtas = 1024;
+#ifndef FA_DECODE_CTAS
+#define FA_DECODE_CTAS 1024
+#endif
+constexpr int kDecodeCtas = FA_DECODE_CTAS;
 constexpr int kDecodeMaxSplit = 256;
 struct DecodePlan {
   int rmax = 4, n_rg = 1, n_split = 1, tiles_per_split = 1;

@@ -43,18 +43,30 @@ template <int D, int RMAX>
 struct DecCfg {
   static constexpr int THREADS = 256;
   static constexpr int KT = 64;                  // keys per tile
-  static constexpr int ROW_BYTES = D * 2 + 16;   // padded K/V row in shared memory
+  // K/V rows are stored unpadded; the 16-byte chunk c of tile row k sits at
+  // chunk position c ^ (k & 7), so that eight consecutive rows reading one
+  // chunk, and one row's eight consecutive chunks, hit distinct banks
+  static constexpr int ROW_BYTES = D * 2;
   static constexpr int TILE_BYTES = KT * ROW_BYTES;
-  static constexpr int Q_OFF = 0;                                  // fp32 [RMAX][D]
+  // score phase: thread = (key, part); part p sums the chunks p, p + PARTS, ...
+  static constexpr int PARTS = THREADS / KT;
+  static constexpr int CH_PER_PART = D / 8 / PARTS;
+  // PV phase: thread = (8-column chunk, group of 4 rows, key group)
+  static constexpr int NCH = D / 8;
+  static constexpr int NRG4 = RMAX / 4;
+  static constexpr int KG = THREADS / (NCH * NRG4);   // key groups
+  static constexpr int KPG = KT / KG;                  // keys per group (key = group + KG·j)
+  static constexpr int Q_OFF = 0;                                  // fp32 [RMAX][D], log2 units
   static constexpr int K_OFF = Q_OFF + RMAX * D * 4;               // 2 stages
   static constexpr int V_OFF = K_OFF + 2 * TILE_BYTES;             // 2 stages
-  static constexpr int S_OFF = V_OFF + 2 * TILE_BYTES;             // fp32 [RMAX][KT]: scores, then P
-  static constexpr int ST_OFF = S_OFF + RMAX * KT * 4;             // fp32 m, l, alpha [RMAX] each
+  static constexpr int SP_OFF = V_OFF + 2 * TILE_BYTES;            // fp32 [PARTS][RMAX][KT]: partial scores
+  static constexpr int PT_OFF = SP_OFF + PARTS * RMAX * KT * 4;    // fp32 [KT][RMAX]: P, key-major
+  static constexpr int ST_OFF = PT_OFF + KT * RMAX * 4;            // fp32 m, l, alpha [RMAX] each
   static constexpr int SMEM_BYTES = ST_OFF + 3 * RMAX * 4;
-  static constexpr int SR = RMAX * KT / THREADS;                   // score rows per thread (≥ 1)
-  static constexpr int PV_ITEMS = RMAX * (D / 2);                  // (row, column pair) items
-  static constexpr int PR = (PV_ITEMS + THREADS - 1) / THREADS;    // items per thread
-  static_assert(RMAX % 4 == 0 && SR >= 1, "four rows per 64-key tile at least");
+  static constexpr int RED_BYTES = KG * RMAX * D * 4;              // final sum over key groups (over K/V)
+  static_assert(RMAX % 4 == 0 && CH_PER_PART >= 1 && NCH % 8 == 0, "tile shape");
+  static_assert(KG >= 1 && KT % KG == 0 && THREADS % (NCH * NRG4) == 0, "PV thread map");
+  static_assert(RED_BYTES <= 4 * TILE_BYTES, "key-group sums fit over the K/V stages");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -69,6 +81,7 @@ __device__ __forceinline__ void cp_async_wait() {
 // two bf16 in one 32-bit word -> two floats (exact)
 __device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
 __device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t x) { return f2_make(bf_lo(x), bf_hi(x)); }
 
 // Query row r of row group rg -> (head within the group g, query index i).
 __device__ __forceinline__ void dec_row(const DecodeParams& p, int rg, int r, int RMAX, int& g, int& i) {
@@ -83,7 +96,8 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
   using C = DecCfg<D, RMAX>;
   extern __shared__ __align__(16) uint8_t smem[];
   float* Qs = reinterpret_cast<float*>(smem + C::Q_OFF);
-  float* S = reinterpret_cast<float*>(smem + C::S_OFF);
+  float* SP = reinterpret_cast<float*>(smem + C::SP_OFF);
+  float* PT = reinterpret_cast<float*>(smem + C::PT_OFF);
   float* m_s = reinterpret_cast<float*>(smem + C::ST_OFF);
   float* l_s = m_s + RMAX;
   float* a_s = l_s + RMAX;
@@ -97,7 +111,7 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
   const int b = unit / (p.n_rg * p.Hkv);
   const int rows = min(RMAX, p.R - rg * RMAX);  // real rows of this group
 
-  // query rows, pre-scaled to log2 units
+  // query rows, pre-scaled to log2 units (rows past `rows` are zero)
   for (int e = tid; e < RMAX * D; e += C::THREADS) {
     const int r = e / D, c = e - r * D;
     float x = 0.f;
@@ -122,27 +136,35 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
   // K and V tile t into stage st: 16-byte chunks, rows past Nk zero-filled
   // (their source address is clamped to a valid row and nothing is read)
   auto load_tile = [&](int t, int st) {
-    constexpr int CHUNKS = C::KT * D / 8;
+    constexpr int CHUNKS = C::KT * C::NCH;
     for (int e = tid; e < CHUNKS; e += C::THREADS) {
-      const int row = e / (D / 8), ch = e - row * (D / 8);
+      const int row = e / C::NCH, ch = e - row * C::NCH;
       const int key = t * C::KT + row;
       const bool in = key < p.Nk;
       const size_t src = (kv_base + (in ? key : 0)) * D + ch * 8;
-      const uint32_t off = (uint32_t)(row * C::ROW_BYTES + ch * 16);
+      const uint32_t off = (uint32_t)(row * C::ROW_BYTES + ((ch ^ (row & 7)) << 4));
       cp_async16(sbase + C::K_OFF + st * C::TILE_BYTES + off, p.k + src, in ? 16u : 0u);
       cp_async16(sbase + C::V_OFF + st * C::TILE_BYTES + off, p.v + src, in ? 16u : 0u);
     }
     cp_async_commit();
   };
 
-  // output accumulators: item = tid + THREADS·j -> (row, column pair)
-  float acc[C::PR][2];
-#pragma unroll
-  for (int j = 0; j < C::PR; ++j) acc[j][0] = acc[j][1] = 0.f;
-
   const int warp = tid >> 5, lane = tid & 31;
-  const int kk = tid % C::KT;          // key of this thread in the score phase
-  const int r0 = tid / C::KT;          // first score row of this thread
+  // score phase map
+  const int ks = tid % C::KT;     // tile row (key) of this thread
+  const int part = tid / C::KT;   // warp-uniform
+  // PV phase map
+  const int c8 = tid % C::NCH;
+  const int g4 = (tid / C::NCH) % C::NRG4;
+  const int kg = tid / (C::NCH * C::NRG4);
+  // O accumulators of rows 4·g4 .. 4·g4+3, columns 8·c8 .. 8·c8+7, as fp32 pairs
+  uint64_t acc[4][4];
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr)
+#pragma unroll
+    for (int i = 0; i < 4; ++i) acc[rr][i] = 0;
+  const uint64_t zero2 = 0;
+
   if (t0 < t1) load_tile(t0, 0);
   for (int t = t0; t < t1; ++t) {
     const int st = (t - t0) & 1;
@@ -154,50 +176,57 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
     }
     __syncthreads();
 
-    // scores S[r][kk] = Q_r · K_kk (log2 units), masked
+    // partial scores of this thread's part of the head dimension, all rows
     {
-      const uint8_t* krow = smem + C::K_OFF + st * C::TILE_BYTES + kk * C::ROW_BYTES;
-      float s[C::SR];
+      const uint8_t* krow = smem + C::K_OFF + st * C::TILE_BYTES + ks * C::ROW_BYTES;
+      uint64_t s2[RMAX];
 #pragma unroll
-      for (int j = 0; j < C::SR; ++j) s[j] = 0.f;
-#pragma unroll 4
-      for (int ch = 0; ch < D / 8; ++ch) {
-        const uint4 kv4 = *reinterpret_cast<const uint4*>(krow + ch * 16);
-        const float kf[8] = {bf_lo(kv4.x), bf_hi(kv4.x), bf_lo(kv4.y), bf_hi(kv4.y),
-                             bf_lo(kv4.z), bf_hi(kv4.z), bf_lo(kv4.w), bf_hi(kv4.w)};
+      for (int r = 0; r < RMAX; ++r) s2[r] = 0;
 #pragma unroll
-        for (int j = 0; j < C::SR; ++j) {
-          const float4* qv = reinterpret_cast<const float4*>(Qs + (r0 + 4 * j) * D + ch * 8);
-          const float4 qa = qv[0], qb = qv[1];
-          s[j] = fmaf(qa.x, kf[0], s[j]);
-          s[j] = fmaf(qa.y, kf[1], s[j]);
-          s[j] = fmaf(qa.z, kf[2], s[j]);
-          s[j] = fmaf(qa.w, kf[3], s[j]);
-          s[j] = fmaf(qb.x, kf[4], s[j]);
-          s[j] = fmaf(qb.y, kf[5], s[j]);
-          s[j] = fmaf(qb.z, kf[6], s[j]);
-          s[j] = fmaf(qb.w, kf[7], s[j]);
+      for (int i = 0; i < C::CH_PER_PART; ++i) {
+        const int ch = part + C::PARTS * i;
+        const uint4 w = *reinterpret_cast<const uint4*>(krow + ((ch ^ (ks & 7)) << 4));
+        const uint64_t k01 = bf2_to_f2(w.x), k23 = bf2_to_f2(w.y), k45 = bf2_to_f2(w.z), k67 = bf2_to_f2(w.w);
+#pragma unroll
+        for (int r = 0; r < RMAX; ++r) {
+          const ulonglong2* qv = reinterpret_cast<const ulonglong2*>(Qs + r * D + ch * 8);
+          const ulonglong2 qa = qv[0], qb = qv[1];
+          s2[r] = f2_fma(qa.x, k01, s2[r]);
+          s2[r] = f2_fma(qa.y, k23, s2[r]);
+          s2[r] = f2_fma(qb.x, k45, s2[r]);
+          s2[r] = f2_fma(qb.y, k67, s2[r]);
         }
       }
-      const int key = t * C::KT + kk;
+      float* sp = SP + part * RMAX * C::KT + ks;
 #pragma unroll
-      for (int j = 0; j < C::SR; ++j) {
-        const int r = r0 + 4 * j;
-        bool vis = (r < rows) && (key < p.Nk);
-        if (CAUSAL && vis) {
-          int g, i;
-          dec_row(p, rg, r, RMAX, g, i);
-          vis = key <= p.Nk - p.Nq + i;
-        }
-        S[r * C::KT + kk] = vis ? s[j] : -INFINITY;
+      for (int r = 0; r < RMAX; ++r) {
+        float lo, hi;
+        f2_split(s2[r], lo, hi);
+        sp[r * C::KT] = lo + hi;
       }
     }
     __syncthreads();
 
-    // online softmax, one warp per row: P over S, running m and l, rescale factor
-    for (int r = warp; r < rows; r += C::THREADS / 32) {
-      float* sr = S + r * C::KT;
-      const float x0 = sr[lane], x1 = sr[lane + 32];
+    // one warp per row: sum the parts, mask, online softmax; P stored key-major
+    for (int r = warp; r < RMAX; r += C::THREADS / 32) {
+      float x0 = 0.f, x1 = 0.f;
+#pragma unroll
+      for (int pp = 0; pp < C::PARTS; ++pp) {
+        x0 += SP[(pp * RMAX + r) * C::KT + lane];
+        x1 += SP[(pp * RMAX + r) * C::KT + lane + 32];
+      }
+      int last = -1;  // last visible key of this row (-1: a padding row sees none)
+      if (r < rows) {
+        last = p.Nk - 1;
+        if (CAUSAL) {
+          int g, i;
+          dec_row(p, rg, r, RMAX, g, i);
+          last = p.Nk - p.Nq + i;
+        }
+      }
+      const int key0 = t * C::KT + lane;
+      if (key0 > last) x0 = -INFINITY;
+      if (key0 + 32 > last) x1 = -INFINITY;
       float mx = fmaxf(x0, x1);
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) mx = fmaxf(mx, __shfl_xor_sync(0xffffffffu, mx, off));
@@ -212,8 +241,8 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
       float sum = p0 + p1;
 #pragma unroll
       for (int off = 16; off > 0; off >>= 1) sum += __shfl_xor_sync(0xffffffffu, sum, off);
-      sr[lane] = p0;
-      sr[lane + 32] = p1;
+      PT[lane * RMAX + r] = p0;
+      PT[(lane + 32) * RMAX + r] = p1;
       if (lane == 0) {
         l_s[r] = l_s[r] * alpha + sum;
         m_s[r] = m_new;
@@ -222,43 +251,63 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
     }
     __syncthreads();
 
-    // O[r][2cp..2cp+1] = alpha_r·O + Σ_kk P[r][kk]·V[kk][2cp..2cp+1]
+    // O[r][cols] = alpha_r·O + Σ_key P[r][key]·V[key][cols] over this thread's keys
     {
-      const uint8_t* vt = smem + C::V_OFF + st * C::TILE_BYTES;
 #pragma unroll
-      for (int j = 0; j < C::PR; ++j) {
-        const int item = tid + C::THREADS * j;
-        if (item < C::PV_ITEMS) {
-          const int r = item / (D / 2), cp = item - r * (D / 2);
-          if (r < rows) {
-            const float* pr = S + r * C::KT;
-            float o0 = acc[j][0] * a_s[r], o1 = acc[j][1] * a_s[r];
-#pragma unroll 8
-            for (int key = 0; key < C::KT; ++key) {
-              const uint32_t w = *reinterpret_cast<const uint32_t*>(vt + key * C::ROW_BYTES + cp * 4);
-              const float pk = pr[key];
-              o0 = fmaf(pk, bf_lo(w), o0);
-              o1 = fmaf(pk, bf_hi(w), o1);
-            }
-            acc[j][0] = o0;
-            acc[j][1] = o1;
-          }
+      for (int rr = 0; rr < 4; ++rr) {
+        const float a = a_s[4 * g4 + rr];
+        const uint64_t a2 = f2_make(a, a);
+#pragma unroll
+        for (int i = 0; i < 4; ++i) acc[rr][i] = f2_fma(acc[rr][i], a2, zero2);
+      }
+      const uint8_t* vt = smem + C::V_OFF + st * C::TILE_BYTES;
+#pragma unroll 4
+      for (int j = 0; j < C::KPG; ++j) {
+        const int key = kg + C::KG * j;
+        const uint4 w = *reinterpret_cast<const uint4*>(vt + key * C::ROW_BYTES + ((c8 ^ (key & 7)) << 4));
+        const uint64_t v01 = bf2_to_f2(w.x), v23 = bf2_to_f2(w.y), v45 = bf2_to_f2(w.z), v67 = bf2_to_f2(w.w);
+        const float4 p4 = *reinterpret_cast<const float4*>(PT + key * RMAX + 4 * g4);
+        const float pr[4] = {p4.x, p4.y, p4.z, p4.w};
+#pragma unroll
+        for (int rr = 0; rr < 4; ++rr) {
+          const uint64_t p2 = f2_make(pr[rr], pr[rr]);
+          acc[rr][0] = f2_fma(p2, v01, acc[rr][0]);
+          acc[rr][1] = f2_fma(p2, v23, acc[rr][1]);
+          acc[rr][2] = f2_fma(p2, v45, acc[rr][2]);
+          acc[rr][3] = f2_fma(p2, v67, acc[rr][3]);
         }
       }
     }
     __syncthreads();  // this stage is refilled by the next iteration's prefetch
   }
 
-  // partial results of this split
+  // sum the key groups' partial outputs (over the K/V stages, all reads done),
+  // then write this split's unnormalised O, m and l
+  float* red = reinterpret_cast<float*>(smem + C::K_OFF);  // [KG][RMAX][D]
+#pragma unroll
+  for (int rr = 0; rr < 4; ++rr) {
+    float o[8];
+#pragma unroll
+    for (int i = 0; i < 4; ++i) f2_split(acc[rr][i], o[2 * i], o[2 * i + 1]);
+    float4* dst = reinterpret_cast<float4*>(red + ((size_t)kg * RMAX + 4 * g4 + rr) * D + 8 * c8);
+    dst[0] = make_float4(o[0], o[1], o[2], o[3]);
+    dst[1] = make_float4(o[4], o[5], o[6], o[7]);
+  }
+  __syncthreads();
   const size_t units = (size_t)p.B * p.Hkv * p.n_rg;
   float* po = p.part_o + ((size_t)split * units + unit) * RMAX * D;
+  for (int item = tid; item < rows * (D / 4); item += C::THREADS) {
+    const int r = item / (D / 4), c4 = item - r * (D / 4);
+    float4 sum = make_float4(0.f, 0.f, 0.f, 0.f);
 #pragma unroll
-  for (int j = 0; j < C::PR; ++j) {
-    const int item = tid + C::THREADS * j;
-    if (item < C::PV_ITEMS) {
-      const int r = item / (D / 2), cp = item - r * (D / 2);
-      if (r < rows) *reinterpret_cast<float2*>(po + r * D + 2 * cp) = make_float2(acc[j][0], acc[j][1]);
+    for (int g = 0; g < C::KG; ++g) {
+      const float4 x = reinterpret_cast<const float4*>(red + ((size_t)g * RMAX + r) * D)[c4];
+      sum.x += x.x;
+      sum.y += x.y;
+      sum.z += x.z;
+      sum.w += x.w;
     }
+    reinterpret_cast<float4*>(po + r * D)[c4] = sum;
   }
   if (tid < rows) {
     float* pml = p.part_ml + (((size_t)split * units + unit) * RMAX + tid) * 2;
