@@ -327,7 +327,8 @@ def run_decode(args, w, rank, world, local_rank):
         "roofline": {"kernel": "fa_decode_split_kernel", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "peak_source": peaks["source"] + " HBM copy (MEASURED_PEAKS.json)",
-                     "bytes_per_launch": w.hbm_bytes(), "ms_per_launch": ms_split, "traffic": None},
+                     "bytes_per_launch": w.hbm_bytes(), "ms_per_launch": ms_split,
+                     "traffic": MEASURED_DECODE_TRAFFIC.get(w.name)},
         "ms": {"split_kernel": ms_split, "call": ms_step},
         "cpu_baseline": cpu,
         "e2e": e2e,
@@ -445,6 +446,10 @@ L2_BYTES = 126 * 2**20
 # capture of the current kernel (profiles/fa_kernels_d128_train_ncu_full.md).  Must be reset
 # to None whenever fa_bwd_kernel changes.
 MEASURED_TRAFFIC = {"train_b8_h16_n2048_d128": 631.0e6}
+
+# The same for one fa_decode_split_kernel launch (profiles/fa_decode_split_b8_hq32_hkv8_nk32768_d128.md);
+# reset to None whenever that kernel changes.
+MEASURED_DECODE_TRAFFIC = {"decode_b8_hq32_hkv8_nk32768_d128": 1079.4e6}
 
 
 def _l2_note(*tensors) -> str:
