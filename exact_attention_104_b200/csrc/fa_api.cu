@@ -4,6 +4,7 @@
 #include <cuda_runtime.h>
 
 #include <algorithm>
+#include <atomic>
 #include <cmath>
 #include <cstdint>
 #include <mutex>
@@ -26,7 +27,7 @@ static __device__ __align__(256) unsigned char g_fa_noalloc_scratch[FA_NOALLOC_S
 namespace {
 
 constexpr int kMaxDevices = 64;
-long long g_wait_cap = 1LL << 31;
+std::atomic<long long> g_wait_cap{1LL << 31};  // may be set from any host thread
 
 // pending one-shot profiling events of this host thread (fa_profile_next)
 thread_local cudaEvent_t t_prof_start = nullptr;
@@ -430,7 +431,7 @@ fa_status fa_selftest_exp2(const float* x, float* y, long long n, int use_poly, 
 
 fa_status fa_set_wait_cap(long long cycles) {
   if (cycles < 0) return FA_ERR_INVALID_ARG;
-  g_wait_cap = cycles == 0 ? (1LL << 31) : cycles;
+  g_wait_cap.store(cycles == 0 ? (1LL << 31) : cycles, std::memory_order_relaxed);
   return FA_OK;
 }
 
@@ -473,7 +474,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   p.G = Hq / Hkv;
   p.n_qtiles = (N + 127) / 128;
   p.scale_log2 = scale * fa::kLog2e;
-  p.wait_cap = g_wait_cap;
+  p.wait_cap = g_wait_cap.load(std::memory_order_relaxed);
   p.err = di->err;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
   const bool tail = (N % 128) != 0;
@@ -577,7 +578,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   p.G = Hq / Hkv;
   p.scale = scale;
   p.scale_log2 = scale * fa::kLog2e;
-  p.wait_cap = g_wait_cap;
+  p.wait_cap = g_wait_cap.load(std::memory_order_relaxed);
   p.err = di->err;
   const bool tail = (N % 128) != 0;
   auto main_kernel = [&](auto dtag) -> fa_status {

@@ -82,7 +82,10 @@ size_t fa_bwd_workspace_bytes(int B, int Hq, int Hkv, int N, int d);
  * gradient dout, writes dq, dk, dv (bf16).  dk and dv are summed over the
  * query heads that share a key/value head.  `workspace` (device, 256-byte
  * aligned, at least fa_bwd_workspace_bytes) is scratch owned by the caller;
- * its contents on entry do not matter.  Enqueues three kernels on `stream`. */
+ * its contents on entry do not matter, and it is in use until the call's
+ * kernels have finished, so calls that may run at the same time (on
+ * different streams) need separate workspaces.  Enqueues three kernels on
+ * `stream`. */
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
                  const void* dout, void* dq, void* dk, void* dv,
                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
