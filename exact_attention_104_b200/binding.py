@@ -13,9 +13,11 @@ import os
 
 import torch
 
-LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+# FA_B200_DEBUG=1 selects the debug build (device-side checks, -DFA_DEBUG)
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)),
+                        "libfa_b200_debug.so" if os.environ.get("FA_B200_DEBUG") == "1" else "libfa_b200.so")
 
-FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT = range(5)
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_DEVICE_CHECK = range(6)
 
 _lib = None
 
@@ -33,7 +35,8 @@ def lib() -> ctypes.CDLL:
         return _lib
     if not os.path.exists(LIB_PATH):
         raise FAError(FA_ERR_UNSUPPORTED, f"{LIB_PATH} is missing; build it with "
-                      "`python -m exact_attention_104_b200.build`")
+                      "`python -m exact_attention_104_b200.build`"
+                      + (" --debug" if LIB_PATH.endswith("_debug.so") else ""))
     L = ctypes.CDLL(LIB_PATH)
     vp, i, f, z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]

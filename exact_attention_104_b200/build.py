@@ -1,8 +1,10 @@
 """Builds libfa_b200.so in-tree with nvcc for sm_100a.
 
-Usage: ``python -m exact_attention_104_b200.build [--verbose]``.  The library
-is rebuilt only when a source under ``csrc/`` or the C header is newer than
-it (``force=True`` rebuilds unconditionally).
+Usage: ``python -m exact_attention_104_b200.build [--verbose] [--debug]``.  The
+library is rebuilt only when a source under ``csrc/`` or the C header is newer
+than it (``force=True`` rebuilds unconditionally).  ``--debug`` builds
+``libfa_b200_debug.so`` instead, with the device-side checks of ``-DFA_DEBUG``
+(the binding loads it when ``FA_B200_DEBUG=1``).
 """
 
 from __future__ import annotations
@@ -18,6 +20,7 @@ ROOT = os.path.dirname(PKG_DIR)
 CSRC = os.path.join(PKG_DIR, "csrc")
 INCLUDE = os.path.join(ROOT, "include")
 LIB_PATH = os.path.join(PKG_DIR, "libfa_b200.so")
+DEBUG_LIB_PATH = os.path.join(PKG_DIR, "libfa_b200_debug.so")
 
 ARCH_FLAGS = ["-gencode", "arch=compute_100a,code=sm_100a"]
 
@@ -34,21 +37,26 @@ def _sources():
                   + glob.glob(os.path.join(INCLUDE, "*.h")))
 
 
-def needs_build() -> bool:
-    if not os.path.exists(LIB_PATH):
+def needs_build(path: str = LIB_PATH) -> bool:
+    if not os.path.exists(path):
         return True
-    t = os.path.getmtime(LIB_PATH)
+    t = os.path.getmtime(path)
     return any(os.path.getmtime(s) > t for s in _sources())
 
 
-def build(force: bool = False, verbose: bool = False) -> str:
-    if not force and not needs_build():
-        return LIB_PATH
+def build(force: bool = False, verbose: bool = False, debug: bool = False, out: str | None = None) -> str:
+    """Compile the library; returns its path.  ``debug`` adds -DFA_DEBUG and,
+    unless ``out`` names another file, writes libfa_b200_debug.so."""
+    path = out or (DEBUG_LIB_PATH if debug else LIB_PATH)
+    if not force and not needs_build(path):
+        return path
     cmd = [
         _nvcc(), *ARCH_FLAGS, "-lineinfo", "-O3", "-std=c++17", "--expt-relaxed-constexpr",
         "-Xcompiler", "-fPIC", "-shared", "-I", INCLUDE, "-I", CSRC,
-        "-o", LIB_PATH + ".tmp", os.path.join(CSRC, "fa_api.cu"),
+        "-o", path + ".tmp", os.path.join(CSRC, "fa_api.cu"),
     ]
+    if debug:
+        cmd.insert(1, "-DFA_DEBUG")
     if verbose:
         cmd.insert(1, "-Xptxas=-v")
     proc = subprocess.run(cmd, capture_output=True, text=True)
@@ -56,10 +64,9 @@ def build(force: bool = False, verbose: bool = False) -> str:
         raise RuntimeError("nvcc failed:\n" + " ".join(cmd) + "\n" + proc.stdout + proc.stderr)
     if verbose:
         sys.stdout.write(proc.stdout + proc.stderr)
-    os.replace(LIB_PATH + ".tmp", LIB_PATH)
-    return LIB_PATH
+    os.replace(path + ".tmp", path)
+    return path
 
 
 if __name__ == "__main__":
-    build(force=True, verbose="--verbose" in sys.argv)
-    print(LIB_PATH)
+    print(build(force=True, verbose="--verbose" in sys.argv, debug="--debug" in sys.argv))

@@ -16,9 +16,6 @@
 #include "fa_fwd.cuh"
 #include "fa_fwd_persistent.cuh"
 
-// Device error word: kernels that abandon a bounded wait record it here.
-__device__ int g_fa_err = 0;
-
 // Scratch of fa_bwd_noalloc: a fixed device array instead of a caller buffer.
 // Host code must not pass this symbol to a kernel (on the host it names a
 // stand-in, not device memory); noalloc_scratch() resolves its device address.
@@ -395,6 +392,7 @@ const char* fa_status_string(fa_status s) {
     case FA_ERR_UNSUPPORTED: return "unsupported configuration";
     case FA_ERR_CUDA: return "CUDA error";
     case FA_ERR_TIMEOUT: return "device wait timed out";
+    case FA_ERR_DEVICE_CHECK: return "device-side check failed (debug build)";
   }
   return "unknown status";
 }
@@ -620,7 +618,8 @@ fa_status fa_device_status(void* stream) {
   if (cudaMemcpy(&host, di->err, sizeof(int), cudaMemcpyDeviceToHost) != cudaSuccess) return FA_ERR_CUDA;
   if (host != 0 && cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return FA_ERR_CUDA;
-  return host != 0 ? FA_ERR_TIMEOUT : FA_OK;
+  if (host == 0) return FA_OK;
+  return (host & 0xff) == fa::kDevCheck ? FA_ERR_DEVICE_CHECK : FA_ERR_TIMEOUT;
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,

@@ -10,13 +10,17 @@
 #include <cuda.h>
 #include <cuda_bf16.h>
 
+// Device error word: kernels that abandon a bounded wait (or, in debug builds,
+// fail a device-side check) record it here; fa_device_status reads and clears it.
+__device__ int g_fa_err = 0;
+
 namespace fa {
 
 constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
-// Device error word values (a timeout records the wait site in bits 8..15).
-enum : int { kDevOk = 0, kDevTimeout = 4 };
+// Device error word values (the failing site goes in bits 8..15).
+enum : int { kDevOk = 0, kDevTimeout = 4, kDevCheck = 5 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -97,8 +101,30 @@ __device__ __forceinline__ void tma_prefetch_desc(const CUtensorMap* m) {
   asm volatile("prefetch.tensormap [%0];" ::"l"(reinterpret_cast<uint64_t>(m)) : "memory");
 }
 
+// Debug builds (-DFA_DEBUG) check every bulk copy against the rules that make
+// one fault instead of failing cleanly: the innermost coordinate of a tiled
+// copy must start on a 16-byte boundary (every tensor map here has 2- or
+// 4-byte elements and is addressed in steps of 8 elements), a tiled store or
+// reduce must not start at a negative coordinate, and a tiled shared-memory
+// box must be 128-byte aligned (16 bytes for plain bulk copies and the
+// unswizzled reduce source).  A failing check records kDevCheck with its site
+// in the device error word (first failure wins) and skips the copy; whoever
+// waits for it gives up through its bounded wait.  Release builds compile the
+// checks away.
+#ifdef FA_DEBUG
+__device__ __forceinline__ bool dbg_ok(bool ok, int site) {
+  if (!ok) atomicCAS(&g_fa_err, 0, kDevCheck | (site << 8));
+  return ok;
+}
+#define FA_DBG_GUARD(cond, site) \
+  if (!::fa::dbg_ok((cond), (site))) return
+#else
+#define FA_DBG_GUARD(cond, site)
+#endif
+
 // 2-D tiled load of one box into shared memory, completing on `bar`.
 __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y) {
+  FA_DBG_GUARD((x & 7) == 0 && x >= 0 && (dst & 127u) == 0, 101);
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1, {%3, %4}], [%2];" ::"r"(
           dst),
@@ -109,6 +135,7 @@ __device__ __forceinline__ void tma_load_2d(uint32_t dst, const CUtensorMap* m, 
 // Same with an L2 eviction-priority hint (policy from createpolicy).
 __device__ __forceinline__ void tma_load_2d_hint(uint32_t dst, const CUtensorMap* m, uint32_t bar, int x, int y,
                                                  uint64_t policy) {
+  FA_DBG_GUARD((x & 7) == 0 && x >= 0 && (dst & 127u) == 0, 102);
   asm volatile(
       "cp.async.bulk.tensor.2d.shared::cluster.global.mbarrier::complete_tx::bytes.L2::cache_hint [%0], [%1, {%3, "
       "%4}], [%2], %5;" ::"r"(dst),
@@ -131,6 +158,7 @@ __device__ __forceinline__ uint64_t policy_evict_first() {
 // Contiguous global->shared bulk copy (both addresses 16-byte aligned, size a
 // multiple of 16), completing on `bar`.
 __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_t bytes, uint32_t bar) {
+  FA_DBG_GUARD((dst & 15u) == 0 && (reinterpret_cast<uintptr_t>(src) & 15u) == 0 && (bytes & 15u) == 0, 103);
   asm volatile("cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(dst),
                "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(bar)
                : "memory");
@@ -140,6 +168,7 @@ __device__ __forceinline__ void bulk_load(uint32_t dst, const void* src, uint32_
 // type of the tensor map, here f32), tracked by the bulk async-group of the
 // issuing thread.
 __device__ __forceinline__ void tma_reduce_add_2d(const CUtensorMap* m, uint32_t src, int x, int y) {
+  FA_DBG_GUARD((x & 7) == 0 && x >= 0 && y >= 0 && (src & 15u) == 0, 104);
   asm volatile(
       "cp.reduce.async.bulk.tensor.2d.global.shared::cta.add.tile.bulk_group [%0, {%2, %3}], [%1];" ::"l"(
           reinterpret_cast<uint64_t>(m)),

@@ -42,7 +42,13 @@
  *                       rounded up to 128), or no sm_100 device;
  *   FA_ERR_CUDA         a CUDA launch or attribute call failed;
  *   FA_ERR_TIMEOUT      (fa_device_status only) a kernel gave up a bounded
- *                       wait and returned early; its outputs are invalid.
+ *                       wait and returned early; its outputs are invalid;
+ *   FA_ERR_DEVICE_CHECK (fa_device_status, debug builds only) a device-side
+ *                       check of a bulk-copy coordinate or address failed
+ *                       and the copy was skipped; outputs are invalid.  The
+ *                       library is a debug build when compiled with
+ *                       -DFA_DEBUG (python -m exact_attention_104_b200.build
+ *                       --debug writes libfa_b200_debug.so).
  * A problem with B == 0 or N == 0 is empty: nothing is enqueued, FA_OK.
  */
 #ifndef FA_B200_H
@@ -59,7 +65,8 @@ typedef enum {
   FA_ERR_INVALID_ARG = 1,
   FA_ERR_UNSUPPORTED = 2,
   FA_ERR_CUDA = 3,
-  FA_ERR_TIMEOUT = 4
+  FA_ERR_TIMEOUT = 4,
+  FA_ERR_DEVICE_CHECK = 5
 } fa_status;
 
 /* Forward pass: writes O (bf16) and LSE (fp32, natural log).
@@ -92,7 +99,8 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
                  void* workspace, size_t workspace_bytes, void* stream);
 
 /* Synchronises `stream`, then reads and clears the current device's error
- * word.  FA_ERR_TIMEOUT if a kernel abandoned a bounded wait since the last
+ * word.  FA_ERR_DEVICE_CHECK if a debug build's device-side check failed,
+ * else FA_ERR_TIMEOUT if a kernel abandoned a bounded wait since the last
  * call, FA_ERR_CUDA if the stream reported a CUDA error, else FA_OK. */
 fa_status fa_device_status(void* stream);
 

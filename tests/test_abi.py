@@ -39,9 +39,21 @@ def test_library_exports_every_declared_symbol(lib):
 
 
 def test_status_strings(lib):
-    for code in range(5):
-        assert binding.fa_status_string(code)
+    for code in range(6):
+        assert binding.fa_status_string(code) != "unknown status"
+    assert binding.fa_status_string(binding.FA_ERR_DEVICE_CHECK) == "device-side check failed (debug build)"
     assert binding.fa_status_string(99) == "unknown status"
+
+
+def test_debug_build_compiles_and_exports_the_same_symbols(tmp_path):
+    # the -DFA_DEBUG variant (device-side checks of bulk-copy coordinates)
+    path = build(force=True, debug=True, out=str(tmp_path / "libfa_b200_debug.so"))
+    dbg = ctypes.CDLL(path)
+    for name in _declared_functions():
+        assert hasattr(dbg, name), name
+    dbg.fa_status_string.argtypes = [ctypes.c_int]
+    dbg.fa_status_string.restype = ctypes.c_char_p
+    assert dbg.fa_status_string(binding.FA_ERR_DEVICE_CHECK) == b"device-side check failed (debug build)"
 
 
 def test_workspace_bytes_formula(lib):
