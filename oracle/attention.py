@@ -22,7 +22,7 @@ definition written out in float64, materialising the score matrix S and the
 probability matrix P for each (batch, query head), exactly as P3's three steps
 describe (S = Q Kᵀ / √d, softmax, then P V).
 
-Readings taken where the pages are silent (each is listed in the design doc):
+Readings taken where the pages are silent:
 
 * scale ``s`` is applied to the scores before the mask and the softmax (P3
   formula uses 1/√d_k; callers pass ``scale``);
