@@ -443,11 +443,11 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
 L2_BYTES = 126 * 2**20
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one fa_bwd_kernel launch, from one ncu
-# capture of the current kernel (profiles/fa_kernels_d128_train_ncu_full.md).  Must be reset
+# capture of the current kernel (summarised under profiles/).  Must be reset
 # to None whenever fa_bwd_kernel changes.
 MEASURED_TRAFFIC = {"train_b8_h16_n2048_d128": 631.0e6}
 
-# The same for one fa_decode_split_kernel launch (profiles/fa_decode_split_b8_hq32_hkv8_nk32768_d128.md);
+# The same for one fa_decode_split_kernel launch (also summarised under profiles/);
 # reset to None whenever that kernel changes.
 MEASURED_DECODE_TRAFFIC = {"decode_b8_hq32_hkv8_nk32768_d128": 1079.4e6}
 
