@@ -524,3 +524,186 @@ def test_forward_model_catches_a_missing_wait():
         except AssertionError:
             caught += 1
     assert caught > 0
+
+
+# --------------------------------------------- forward, three S buffers (planned)
+def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mistake=None):
+    """The schedule planned for the d = 64 forward, where TMEM has room for a
+    third S buffer: QKᵀ number n (in today's issue order) goes to buffer
+    n mod 3, and after every PV (and in the prologue) the MMA warp issues as
+    many next QKᵀs as are allowed, a buffer being reusable once the PV that read
+    its previous occupant has been issued.  S-full and P-full barriers are per
+    (tile, buffer); each softmax warpgroup waits for its previous PV, in order,
+    after its exponentials and before it releases P.  K/V streaming is unchanged
+    from simulate_fwd and left out here.  The kernel still uses the two-buffer
+    schedule of simulate_fwd; this model checks the planned one."""
+    rnd = random.Random(seed)
+    n_pairs = (n_qtiles + 1) // 2
+    n_items = n_pairs * BH
+    done = {"S": [], "PV": []}
+
+    def item(idx):
+        if causal:
+            pair, bh = n_pairs - 1 - idx // BH, idx % BH
+        else:
+            bh, pair = idx // n_pairs, idx % n_pairs
+        qt0 = 2 * pair
+        has1 = qt0 + 1 < n_qtiles
+        n0 = qt0 + 1 if causal else n_qtiles
+        n1 = (qt0 + 2 if causal else n_qtiles) if has1 else 0
+        skew = 1 if (causal and has1) else 0
+        return dict(qt0=qt0, n0=n0, n1=n1, skew=skew, nit=n0 + skew)
+
+    def kvb(w, jj):
+        return w["qt0"] + 1 if (w["skew"] and jj == 0) else jj - w["skew"]
+
+    def first(w, t):
+        return w["skew"] if t == 0 else 0
+
+    def has(w, t):
+        return t == 0 or w["n1"] > 0
+
+    def deal(k, c):
+        return k * n_ctas + ((n_ctas - 1 - c) if (causal and (k & 1)) else c)
+
+    n_rounds = (n_items + n_ctas - 1) // n_ctas
+    gens, engines = {}, {}
+
+    def make_cta(c):
+        items = [deal(k, c) for k in range(n_rounds) if deal(k, c) < n_items]
+        # the QKᵀ sequence in today's issue order, and the PV order
+        seq, pv_order = [], []
+        if items:
+            w0 = item(items[0])
+            for t in range(2):
+                if has(w0, t):
+                    seq.append((items[0], t, first(w0, t)))
+            for pos, idx in enumerate(items):
+                w = item(idx)
+                nxt = items[pos + 1] if pos + 1 < len(items) else None
+                w2 = item(nxt) if nxt is not None else None
+                for jj in range(w["nit"]):
+                    for t in range(2):
+                        if not has(w, t) or jj < first(w, t):
+                            continue
+                        pv_order.append((idx, t, jj))
+                        if jj + 1 < w["nit"]:
+                            seq.append((idx, t, jj + 1))
+                        elif nxt is not None and has(w2, t):
+                            seq.append((nxt, t, first(w2, t)))
+                if nxt is not None and not has(w, 1) and has(w2, 1):
+                    seq.append((nxt, 1, 0))
+        seq_no = {e: n for n, e in enumerate(seq)}
+        assert len(seq_no) == len(seq) == len(pv_order)
+        # phase index of QKᵀ n on its (tile, buffer) barriers: how many earlier
+        # QKᵀs of the same tile went to the same buffer
+        phase = {}
+        cnt = {}
+        for n, e in enumerate(seq):
+            key = (e[1], n % nbuf)
+            phase[n] = cnt.get(key, 0)
+            cnt[key] = phase[n] + 1
+        bars = {}
+        for t in range(2):
+            for b in range(nbuf):
+                bars["SFULL", t, b] = _Bar(1)   # per (tile, buffer)
+                bars["PFULL", t, b] = _Bar(4)
+            bars["ODONE", t] = _Bar(1)
+        wait = _waiter(bars)
+        tc = []
+        buf_owner = {}        # buffer -> QKᵀ number written last
+        pv_issued = set()     # QKᵀ numbers whose PV has been issued
+        p_written = set()
+
+        def mma():
+            nxt = [0]
+
+            def try_issue():
+                while nxt[0] < len(seq):
+                    n = nxt[0]
+                    b = n % nbuf
+                    if n >= nbuf and (n - nbuf) not in pv_issued and mistake != "no_buffer_rule":
+                        return
+                    if b in buf_owner:
+                        assert buf_owner[b] in pv_issued, "S overwrites an unconsumed P"
+                    buf_owner[b] = n
+                    done["S"].append(seq[n])
+                    tc.append(("commit", ("SFULL", seq[n][1], b)))
+                    nxt[0] += 1
+            try_issue()
+            for (idx, t, jj) in pv_order:
+                n = seq_no[(idx, t, jj)]
+                yield from wait(("PFULL", t, n % nbuf), phase[n])
+                assert n in p_written and n not in pv_issued
+                pv_issued.add(n)
+                done["PV"].append((idx, t, jj))
+                tc.append(("commit", ("ODONE", t)))
+                yield
+                try_issue()
+            assert nxt[0] == len(seq), "QKᵀs left unissued"
+
+        def softmax(t):
+            mine = [n for n, e in enumerate(seq) if e[1] == t]
+            seen = [-1]
+
+            def odone_upto(k):
+                # PV completions are waited in order, never skipping one
+                while seen[0] < k:
+                    seen[0] += 1
+                    yield from wait(("ODONE", t), seen[0])
+            for j, n in enumerate(mine):
+                yield from wait(("SFULL", t, n % nbuf), phase[n])
+                assert buf_owner.get(n % nbuf) == n or buf_owner.get(n % nbuf, -1) > n
+                yield                                   # S load, row max, exponentials
+                # the previous PV must be done before O is rescaled (rare) and
+                # before this P is released; PV(j) cannot have started yet, so
+                # at most one ODONE phase is outstanding here
+                if j > 0:
+                    yield from odone_upto(j - 1)
+                yield                                   # rescale of O, P store
+                assert buf_owner[n % nbuf] == n, "S overwritten before its softmax finished"
+                p_written.add(n)
+                for _ in range(4):
+                    bars["PFULL", t, n % nbuf].arrive()
+            if mine:
+                yield from odone_upto(len(mine) - 1)
+
+        def tc_done(entry):
+            bars[entry[1]].arrive()
+
+        gens[c, "mma"] = mma()
+        gens[c, "sm", 0] = softmax(0)
+        gens[c, "sm", 1] = softmax(1)
+        engines[c, "tc"] = (tc, tc_done)
+
+    for c in range(n_ctas):
+        make_cta(c)
+    _run(gens, engines, rnd)
+    for kind in ("S", "PV"):
+        got = sorted((i, t, kvb(item(i), jj)) for (i, t, jj) in done[kind])
+        want = []
+        for idx in range(n_items):
+            w = item(idx)
+            for t in range(2):
+                if has(w, t):
+                    qt = w["qt0"] + t
+                    want += [(idx, t, j) for j in (range(qt + 1) if causal else range(n_qtiles))]
+        assert got == sorted(want), kind
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_three_buffer_forward_schedule(causal):
+    for n_qtiles in (1, 2, 3, 5, 8):
+        for BH, n_ctas in ((1, 1), (3, 2), (5, 3)):
+            for seed in range(3):
+                simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed)
+
+
+def test_three_buffer_model_catches_a_buffer_reused_too_early():
+    caught = 0
+    for seed in range(10):
+        try:
+            simulate_fwd_three_buffers(5, 3, True, 2, seed, mistake="no_buffer_rule")
+        except AssertionError:
+            caught += 1
+    assert caught > 0
