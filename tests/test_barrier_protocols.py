@@ -527,16 +527,21 @@ def test_forward_model_catches_a_missing_wait():
 
 
 # --------------------------------------------- forward, three S buffers (planned)
-def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mistake=None):
+def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slot=8, mistake=None):
     """The schedule planned for the d = 64 forward, where TMEM has room for a
     third S buffer: QKᵀ number n (in today's issue order) goes to buffer
-    n mod 3, and after every PV (and in the prologue) the MMA warp issues as
+    n mod nbuf, and after every PV (and in the prologue) the MMA warp issues as
     many next QKᵀs as are allowed, a buffer being reusable once the PV that read
     its previous occupant has been issued.  S-full and P-full barriers are per
     (tile, buffer); each softmax warpgroup waits for its previous PV, in order,
-    after its exponentials and before it releases P.  K/V streaming is unchanged
-    from simulate_fwd and left out here.  The kernel still uses the two-buffer
-    schedule of simulate_fwd; this model checks the planned one."""
+    after its exponentials and before it releases P.  Q tiles and K/V units are
+    loaded as in simulate_fwd (K and V of each iteration through ``n_slot``
+    slots, units waited in load order, released by their last reader).  The
+    kernel still uses the two-buffer schedule of simulate_fwd; this model checks
+    the planned one (nbuf = 2 is the same schedule with two buffers).  Since
+    QKᵀs are issued earlier, the K/V ring must be deeper: with three buffers
+    the model deadlocks at 5 slots and runs at 6 (two buffers: 3 and 4); the
+    d = 64 kernel has 8."""
     rnd = random.Random(seed)
     n_pairs = (n_qtiles + 1) // 2
     n_items = n_pairs * BH
@@ -571,6 +576,11 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mista
 
     def make_cta(c):
         items = [deal(k, c) for k in range(n_rounds) if deal(k, c) < n_items]
+        base_of = {}
+        acc = 0
+        for idx in items:
+            base_of[idx] = acc
+            acc += 2 * item(idx)["nit"]
         # the QKᵀ sequence in today's issue order, and the PV order
         seq, pv_order = [], []
         if items:
@@ -609,14 +619,58 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mista
                 bars["SFULL", t, b] = _Bar(1)   # per (tile, buffer)
                 bars["PFULL", t, b] = _Bar(4)
             bars["ODONE", t] = _Bar(1)
+            bars["QFULL", t] = _Bar(1)
+            bars["QEMPTY", t] = _Bar(1)
+        for sl in range(n_slot):
+            bars["KVFULL", sl] = _Bar(1)
+            bars["KVEMPTY", sl] = _Bar(1)
         wait = _waiter(bars)
-        tc = []
+        tc, tma = [], []
         buf_owner = {}        # buffer -> QKᵀ number written last
         pv_issued = set()     # QKᵀ numbers whose PV has been issued
         p_written = set()
+        q_tile = {0: None, 1: None}
+        slot_unit, released, loaded = {}, set(), set()
+
+        def producer():
+            useq = 0
+            q_loads = [0, 0]
+            for idx in items:
+                w = item(idx)
+                for t in range(2):
+                    if not has(w, t):
+                        continue
+                    if q_loads[t] > 0:
+                        yield from wait(("QEMPTY", t), q_loads[t] - 1)
+                    q_tile[t] = idx
+                    tma.append((("QFULL", t), None))
+                    q_loads[t] += 1
+                for u in range(2 * w["nit"]):
+                    U = useq + u
+                    sl = U % n_slot
+                    if U >= n_slot:
+                        yield from wait(("KVEMPTY", sl), U // n_slot - 1)
+                    if sl in slot_unit:
+                        assert slot_unit[sl] in released, f"slot {sl} refilled while unit {slot_unit[sl]} is read"
+                    slot_unit[sl] = U
+                    tma.append((("KVFULL", sl), U))
+                useq += 2 * w["nit"]
 
         def mma():
             nxt = [0]
+            waited = [-1]
+            q_seen = [0, 0]
+
+            def wait_upto(U):
+                while waited[0] < U:
+                    waited[0] += 1
+                    yield from wait(("KVFULL", waited[0] % n_slot), waited[0] // n_slot)
+                    assert waited[0] in loaded
+
+            def release(U):
+                assert U not in released
+                released.add(U)
+                tc.append(("commit", ("KVEMPTY", U % n_slot)))
 
             def try_issue():
                 while nxt[0] < len(seq):
@@ -624,22 +678,39 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mista
                     b = n % nbuf
                     if n >= nbuf and (n - nbuf) not in pv_issued and mistake != "no_buffer_rule":
                         return
+                    idx, t, jj = seq[n]
+                    w = item(idx)
+                    if jj == first(w, t):
+                        yield from wait(("QFULL", t), q_seen[t])
+                        q_seen[t] += 1
+                    assert q_tile[t] == idx, "Q tile overwritten"
+                    U = base_of[idx] + 2 * jj
+                    yield from wait_upto(U)
                     if b in buf_owner:
                         assert buf_owner[b] in pv_issued, "S overwrites an unconsumed P"
                     buf_owner[b] = n
                     done["S"].append(seq[n])
-                    tc.append(("commit", ("SFULL", seq[n][1], b)))
+                    tc.append(("commit", ("SFULL", t, b)))
+                    if jj == w["nit"] - 1:
+                        tc.append(("commit", ("QEMPTY", t)))
+                    if t == 1 or w["n1"] == 0:
+                        release(U)
                     nxt[0] += 1
-            try_issue()
+            yield from try_issue()
             for (idx, t, jj) in pv_order:
                 n = seq_no[(idx, t, jj)]
+                w = item(idx)
                 yield from wait(("PFULL", t, n % nbuf), phase[n])
-                assert n in p_written and n not in pv_issued
+                Uv = base_of[idx] + 2 * jj + 1
+                yield from wait_upto(Uv)
+                assert n in p_written and n not in pv_issued and Uv not in released
                 pv_issued.add(n)
                 done["PV"].append((idx, t, jj))
                 tc.append(("commit", ("ODONE", t)))
+                if t == 1 or w["n1"] == 0:
+                    release(Uv)
                 yield
-                try_issue()
+                yield from try_issue()
             assert nxt[0] == len(seq), "QKᵀs left unissued"
 
         def softmax(t):
@@ -653,7 +724,6 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mista
                     yield from wait(("ODONE", t), seen[0])
             for j, n in enumerate(mine):
                 yield from wait(("SFULL", t, n % nbuf), phase[n])
-                assert buf_owner.get(n % nbuf) == n or buf_owner.get(n % nbuf, -1) > n
                 yield                                   # S load, row max, exponentials
                 # the previous PV must be done before O is rescaled (rare) and
                 # before this P is released; PV(j) cannot have started yet, so
@@ -671,10 +741,18 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mista
         def tc_done(entry):
             bars[entry[1]].arrive()
 
+        def tma_done(entry):
+            bar, unit = entry
+            if unit is not None:
+                loaded.add(unit)
+            bars[bar].arrive()
+
+        gens[c, "producer"] = producer()
         gens[c, "mma"] = mma()
         gens[c, "sm", 0] = softmax(0)
         gens[c, "sm", 1] = softmax(1)
         engines[c, "tc"] = (tc, tc_done)
+        engines[c, "tma"] = (tma, tma_done)
 
     for c in range(n_ctas):
         make_cta(c)
@@ -691,12 +769,13 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, mista
         assert got == sorted(want), kind
 
 
+@pytest.mark.parametrize("nbuf,n_slot", [(3, 8), (2, 5)])
 @pytest.mark.parametrize("causal", [False, True])
-def test_three_buffer_forward_schedule(causal):
+def test_three_buffer_forward_schedule(causal, nbuf, n_slot):
     for n_qtiles in (1, 2, 3, 5, 8):
         for BH, n_ctas in ((1, 1), (3, 2), (5, 3)):
             for seed in range(3):
-                simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed)
+                simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=nbuf, n_slot=n_slot)
 
 
 def test_three_buffer_model_catches_a_buffer_reused_too_early():
