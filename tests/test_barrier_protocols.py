@@ -527,14 +527,18 @@ def test_forward_model_catches_a_missing_wait():
 
 
 # --------------------------------------------- forward, three S buffers (planned)
-def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slot=8, mistake=None):
+def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slot=8, ring=4, mistake=None):
     """The schedule planned for the d = 64 forward, where TMEM has room for a
     third S buffer: QKᵀ number n (in today's issue order) goes to buffer
     n mod nbuf, and after every PV (and in the prologue) the MMA warp issues as
     many next QKᵀs as are allowed, a buffer being reusable once the PV that read
     its previous occupant has been issued.  S-full and P-full barriers are per
     (tile, buffer); each softmax warpgroup waits for its previous PV, in order,
-    after its exponentials and before it releases P.  Q tiles and K/V units are
+    after its exponentials and before it releases P.  The softmax warpgroups
+    learn each QKᵀ's sequence number from a per-tile ring of ``ring`` slots in
+    shared memory, which the MMA warp fills before it issues the product
+    (one full-barrier per slot, no empty-barrier: the MMA warp runs at most
+    nbuf QKᵀs ahead of the PVs).  Q tiles and K/V units are
     loaded as in simulate_fwd (K and V of each iteration through ``n_slot``
     slots, units waited in load order, released by their last reader).  The
     kernel still uses the two-buffer schedule of simulate_fwd; this model checks
@@ -621,6 +625,8 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slo
             bars["ODONE", t] = _Bar(1)
             bars["QFULL", t] = _Bar(1)
             bars["QEMPTY", t] = _Bar(1)
+            for r in range(ring):
+                bars["NFULL", t, r] = _Bar(1)
         for sl in range(n_slot):
             bars["KVFULL", sl] = _Bar(1)
             bars["KVEMPTY", sl] = _Bar(1)
@@ -630,6 +636,9 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slo
         pv_issued = set()     # QKᵀ numbers whose PV has been issued
         p_written = set()
         q_tile = {0: None, 1: None}
+        ring_slot = {}                   # (tile, slot) -> sequence number written last
+        ring_read = set()                # (tile, tile QKᵀ count) entries read
+        issued_per_tile = [0, 0]
         slot_unit, released, loaded = {}, set(), set()
 
         def producer():
@@ -689,6 +698,12 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slo
                     if b in buf_owner:
                         assert buf_owner[b] in pv_issued, "S overwrites an unconsumed P"
                     buf_owner[b] = n
+                    g = issued_per_tile[t]
+                    if g >= ring:
+                        assert (t, g - ring) in ring_read, "ring slot overwritten before it was read"
+                    ring_slot[t, g % ring] = n
+                    bars["NFULL", t, g % ring].arrive()
+                    issued_per_tile[t] = g + 1
                     done["S"].append(seq[n])
                     tc.append(("commit", ("SFULL", t, b)))
                     if jj == w["nit"] - 1:
@@ -723,6 +738,9 @@ def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slo
                     seen[0] += 1
                     yield from wait(("ODONE", t), seen[0])
             for j, n in enumerate(mine):
+                yield from wait(("NFULL", t, j % ring), j // ring)
+                assert ring_slot[t, j % ring] == n, "wrong sequence number in the ring"
+                ring_read.add((t, j))
                 yield from wait(("SFULL", t, n % nbuf), phase[n])
                 yield                                   # S load, row max, exponentials
                 # the previous PV must be done before O is rescaled (rare) and
