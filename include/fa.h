@@ -112,11 +112,12 @@ const char* fa_status_string(fa_status s);
  * default (2^31 cycles, about one second).  Affects later launches only. */
 fa_status fa_set_wait_cap(long long cycles);
 
-/* One-shot profiling hook for the calling host thread: the next fa_fwd or
- * fa_bwd call records `start_event` on its stream immediately before its
- * attention kernel (fa_fwd's fused kernel; fa_bwd's dK/dV/dQ kernel, after
- * the preprocessing kernel) and `stop_event` immediately after it, then
- * forgets both.  The events are cudaEvent_t handles owned by the caller;
+/* One-shot profiling hook for the calling host thread: the next fa_fwd,
+ * fa_bwd or fa_fwd_decode call records `start_event` on its stream
+ * immediately before its main kernel (fa_fwd's fused kernel; fa_bwd's
+ * dK/dV/dQ kernel, after the preprocessing kernel; fa_fwd_decode's split
+ * kernel, before the combine kernel) and `stop_event` immediately after it,
+ * then forgets both.  The events are cudaEvent_t handles owned by the caller;
  * NULL for both cancels a pending request. */
 fa_status fa_profile_next(void* start_event, void* stop_event);
 
