@@ -6,7 +6,7 @@ takes no workspace and uses the library's fixed 64 MiB device scratch array.
 Checked through the C ABI against the ordinary workspace entry point, fa_bwd,
 on two calls in a row (the array keeps the previous call's contents, so the
 second call shows that nothing stale leaks into the result).  This file is
-named to be collected last."""
+named to be collected after the parity tests."""
 
 import pytest
 import torch
