@@ -245,11 +245,7 @@ def run_decode(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(x, world, dev)
 
     for _ in range(args.warmup):
         step()
@@ -458,6 +454,19 @@ def _l2_note(*tensors) -> str:
     return f"inputs fit in L2 ({mib:.1f} MiB; not flushed: a small parity-sized case, not a bench line)"
 
 
+def reduce_max_over_ranks(x: float, world: int, device) -> float:
+    """The largest of the ranks' values of x (a per-rank elapsed time): every
+    multi-GPU figure is timed on the slowest rank.  ``device`` holds the
+    one-element tensor the collective reduces (a CUDA device under NCCL)."""
+    if world == 1:
+        return x
+    import torch
+    import torch.distributed as dist
+    t = torch.tensor([x], dtype=torch.float64, device=device)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
 def logit_extremes(q, k, scale: float, causal: bool, rows_per_chunk: int = 2048):
     """Largest |q·k| and |s·q·k| over every visible (query, key) pair of batch 0, query
     head 0 (its kv head is 0), computed on the host in fp32 from the bf16 inputs.  A
@@ -521,11 +530,7 @@ def run_ours(args, w, rank, world, local_rank):
         torch.cuda.synchronize()
 
     def max_over_ranks(x: float) -> float:
-        if world == 1:
-            return x
-        t = torch.tensor([x], dtype=torch.float64, device=dev)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
-        return float(t.item())
+        return reduce_max_over_ranks(x, world, dev)
 
     for _ in range(args.warmup):
         fwd()

@@ -43,3 +43,7 @@ def test_logit_extremes_ignore_masked_pairs_and_other_heads():
     q, k = q.bfloat16(), k.bfloat16()
     assert bench.logit_extremes(q, k, 1.0, True)["max_abs_raw"] == 5.0
     assert bench.logit_extremes(q, k, 1.0, False)["max_abs_raw"] == 40.0
+
+
+def test_single_rank_time_is_its_own_maximum():
+    assert bench.reduce_max_over_ranks(2.5, 1, "cpu") == 2.5

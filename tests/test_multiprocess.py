@@ -2,15 +2,24 @@
 independent (batch, kv-head) units across ranks and the max-over-ranks
 timing reduction bench.py uses."""
 
+import importlib.util
 import os
 import socket
 
 import pytest
-import torch
 import torch.distributed as dist
 import torch.multiprocessing as mp
 
 from exact_attention_104_b200.workloads import shard_units
+
+_ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+
+
+def _bench():
+    spec = importlib.util.spec_from_file_location("bench", os.path.join(_ROOT, "bench.py"))
+    mod = importlib.util.module_from_spec(spec)
+    spec.loader.exec_module(mod)
+    return mod
 
 
 def _free_port():
@@ -29,11 +38,11 @@ def _worker(rank, world, port, B, Hkv, q):
         mine = shard_units(B, Hkv, rank, world)
         gathered = [None] * world
         dist.all_gather_object(gathered, mine)
-        # per-rank elapsed time, reduced with MAX as the bench does
-        t = torch.tensor([float(rank + 1) * 1.5], dtype=torch.float64)
-        dist.all_reduce(t, op=dist.ReduceOp.MAX)
+        # per-rank elapsed time, reduced by bench.py's own helper (gloo on CPU
+        # here; NCCL on CUDA tensors in the bench)
+        tmax = _bench().reduce_max_over_ranks(float(rank + 1) * 1.5, world, "cpu")
         if rank == 0:
-            q.put((gathered, float(t.item())))
+            q.put((gathered, tmax))
     finally:
         dist.destroy_process_group()
 
