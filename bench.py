@@ -1,9 +1,9 @@
 """Benchmark: exact attention forward + backward on B200, through the C ABI.
 
 One step = one forward pass (fa_fwd) and one backward pass (fa_bwd) over the
-whole workload, with inputs resident in HBM.  The default workload is
-B=8, Hq=Hkv=16, N=2048, d=128, non-causal, bf16, seeded synthetic N(0,1)
-inputs.  Prints ONE JSON line (rank 0).
+whole workload, with inputs resident in HBM.  The default workload is the
+long causal sequence B=1, Hq=Hkv=16, N=16384, d=128, bf16, seeded synthetic
+N(0,1) inputs.  Prints ONE JSON line (rank 0).
 
   python bench.py [--gpus N] [--steps K] [--warmup W] [--impl ours|reference]
                   [--workload NAME|all] [--no-e2e] [--no-cpu-baseline]
@@ -15,7 +15,8 @@ of the same size (weak scaling; attention over distinct batches needs no data
 exchange), timed with CUDA events, max over ranks.
 
 --impl reference times the fp64 CPU oracle on this host's cores on a bounded
-sample of the same workload (one (batch, head) slice per step).
+sample of the same workload (one strided block of query rows of one head per
+step).
 """
 
 from __future__ import annotations
@@ -123,11 +124,35 @@ class ClockSampler:
 # ------------------------------------------------------------- CPU oracle
 _CPU_INPUTS = {}
 
+# Largest score block (query rows x keys) the CPU sample materialises per step:
+# every row of a head for N <= 2048, a strided block of rows beyond.
+CPU_BLOCK_ENTRIES = 1 << 22
 
-def cpu_oracle_sample(w, seconds: float, max_heads: int | None = None):
-    """Time the fp64 oracle's forward+backward on (batch 0, head h) slices of
-    the workload until `seconds` of CPU work have been spent.  Returns
-    (TFLOPS, heads, elapsed seconds)."""
+
+def cpu_sample_rows(w, step: int):
+    """Query rows and head of CPU-sample step ``step``: head ``step % Hq`` of
+    batch 0, rows ``off, off + stride, ...`` with ``stride = N / R`` and the
+    offset rotating from step to step, R = min(N, CPU_BLOCK_ENTRIES / N)."""
+    import numpy as np
+    n_rows = max(1, min(w.N, CPU_BLOCK_ENTRIES // w.N))
+    stride = max(1, w.N // n_rows)
+    off = (step // w.Hq) % stride
+    return step % w.Hq, np.arange(off, w.N, stride)[:n_rows]
+
+
+def cpu_sample_flops(w, rows) -> float:
+    """FLOPs of the forward+backward share of the given query rows, in the
+    metric's convention: 3.5 x 4·d per visible (query, key) pair."""
+    import numpy as np
+    visible = float(np.sum(np.asarray(rows) + 1)) if w.causal else float(len(rows)) * w.N
+    return 3.5 * 4.0 * w.d * visible
+
+
+def cpu_oracle_sample(w, seconds: float, max_steps: int | None = None, first_step: int = 0):
+    """Time the fp64 oracle's forward+backward share (oracle.head_backward_rows)
+    of strided query-row blocks of single heads of the workload until
+    ``seconds`` of CPU work have been spent (or ``max_steps`` blocks).
+    Returns (TFLOPS, blocks, elapsed seconds, rows per block)."""
     import numpy as np
 
     import oracle
@@ -139,47 +164,47 @@ def cpu_oracle_sample(w, seconds: float, max_heads: int | None = None):
         _CPU_INPUTS[key] = make_inputs(w, "cpu")
     q, k, v, do = _CPU_INPUTS[key]
     G = w.G
-    heads, t_total = 0, 0.0
+    steps, t_total, flops, n_rows = 0, 0.0, 0.0, 0
     while True:
-        h = heads % w.Hq
-        sl = lambda t, hh: t[0:1, hh:hh + 1].float().numpy().astype(np.float64)  # noqa: E731
+        h, rows = cpu_sample_rows(w, first_step + steps)
+        n_rows = len(rows)
+        sl = lambda t, hh: t[0, hh].float().numpy().astype(np.float64)  # noqa: E731
         qs, dos = sl(q, h), sl(do, h)
         ks, vs = sl(k, h // G), sl(v, h // G)
         t0 = time.perf_counter()
-        oracle.attention_backward(qs, ks, vs, dos, w.scale, w.causal)
+        oracle.head_backward_rows(qs, ks, vs, dos, w.scale, w.causal, rows)
         t_total += time.perf_counter() - t0
-        heads += 1
-        if t_total >= seconds or (max_heads is not None and heads >= max_heads):
+        flops += cpu_sample_flops(w, rows)
+        steps += 1
+        if t_total >= seconds or (max_steps is not None and steps >= max_steps):
             break
-    flops_per_head = 3.5 * oracle.attention_flops(1, 1, w.N, w.d, w.causal)
-    return flops_per_head * heads / t_total / 1e12, heads, t_total
+    return flops / t_total / 1e12, steps, t_total, n_rows
 
 
 def run_reference(args, w, rank, world):
-    """The reference arm: the fp64 oracle on the host cores, one (b, h) slice
-    of the workload per step.  Rank 0 only."""
+    """The reference arm: the fp64 oracle on the host cores, one strided block
+    of query rows of one head of the workload per step.  Rank 0 only."""
     if rank != 0:
         return
-    import oracle
-
-    flops_per_step = 3.5 * oracle.attention_flops(1, 1, w.N, w.d, w.causal)
-    for _ in range(args.warmup):
-        cpu_oracle_sample(w, 0.0, max_heads=1)
-    times = []
-    for _ in range(args.steps):
-        _, _, t = cpu_oracle_sample(w, 0.0, max_heads=1)
-        times.append(t)
-    total = sum(times)
-    value = flops_per_step * args.steps / total / 1e12
+    for i in range(args.warmup):
+        cpu_oracle_sample(w, 0.0, max_steps=1, first_step=i)
+    total, flops, n_rows = 0.0, 0.0, 0
+    for i in range(args.steps):
+        h, rows = cpu_sample_rows(w, args.warmup + i)
+        _, _, t, n_rows = cpu_oracle_sample(w, 0.0, max_steps=1, first_step=args.warmup + i)
+        total += t
+        flops += cpu_sample_flops(w, rows)
+    value = flops / total / 1e12
     cores = _blas_threads()
+    sample = (f"per step: {n_rows} strided query rows of one head (batch 0) of {w.describe()}, their share "
+              "of the forward and backward (oracle.head_backward_rows) in fp64")
     line = {
         "impl": "reference", "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": args.gpus,
         "steps": args.steps, "warmup": args.warmup, "ms_per_step": 1e3 * total / args.steps,
         "higher_is_better": True, "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
         "config": {"workload": w.name, "B": w.B, "Hq": w.Hq, "Hkv": w.Hkv, "N": w.N, "d": w.d,
                    "causal": w.causal},
-        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle",
-                         "sample": f"one (batch 0, head h) slice of {w.describe()} per step, fwd+bwd in fp64"},
+        "cpu_baseline": {"value": value, "unit": "TFLOPS", "cores": cores, "kind": "oracle", "sample": sample},
         "e2e": {"value": value, "unit": "TFLOPS", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
     }
     print(json.dumps(line), flush=True)
@@ -594,9 +619,10 @@ def run_ours(args, w, rank, world, local_rank):
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
-        tflops, heads, secs = cpu_oracle_sample(w, args.cpu_seconds)
+        tflops, blocks, secs, n_rows = cpu_oracle_sample(w, args.cpu_seconds)
         cpu = {"value": tflops, "unit": "TFLOPS", "cores": _blas_threads(), "kind": "oracle",
-               "sample": f"{heads} (batch 0, head) slices of {w.describe()}, fwd+bwd in fp64, {secs:.1f} s"}
+               "sample": f"{blocks} blocks of {n_rows} strided query rows of one head (batch 0) of "
+                         f"{w.describe()}, their share of the forward and backward in fp64, {secs:.1f} s"}
 
     # dominant kernel: the backward dK/dV/dQ kernel (2.5x the forward FLOPs)
     bwd_main_flops = 2.5 * F

@@ -630,6 +630,15 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (st != FA_OK || empty) return st;
   const size_t need = fa_bwd_workspace_bytes(B, Hq, Hkv, N, d);
   if (need > (size_t)FA_NOALLOC_SCRATCH_BYTES) return FA_ERR_UNSUPPORTED;
+  // argument and device checks first, so that a bad pointer reports
+  // FA_ERR_INVALID_ARG and a non-sm_100 device FA_ERR_UNSUPPORTED before the
+  // scratch array's address is looked up
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv) return FA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)lse, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
   void* scratch = nullptr;
   st = noalloc_scratch(&scratch);
   if (st != FA_OK) return st;

@@ -50,8 +50,9 @@ class Workload:
                 f"{'causal' if self.causal else 'non-causal'} qk_std={self.qk_std:g}")
 
 
-# The five reference workloads (seed = 1000 + index).  C2 runs both causal and
-# non-causal; the non-causal variant is the benchmark workload.
+# The five reference workloads (seed = 1000 + index); C2 runs both causal and
+# non-causal.  The benchmark workload is the long causal sequence (N = 16384,
+# d = 128), the largest d = 128 problem.
 WORKLOADS = {
     "tiny_b1_h2_n128_d64": Workload("tiny_b1_h2_n128_d64", 1, 2, 2, 128, 64, False, 1.0, 1000),
     "train_b8_h16_n2048_d128": Workload("train_b8_h16_n2048_d128", 8, 16, 16, 2048, 128, False, 1.0, 1001),
@@ -69,7 +70,7 @@ WORKLOADS = {
                                                 1006),
 }
 
-BENCH_WORKLOAD = "train_b8_h16_n2048_d128"
+BENCH_WORKLOAD = "long_b1_h16_n16384_d128_causal"
 
 
 @dataclass(frozen=True)

@@ -27,8 +27,12 @@
  * past N are neither stored nor given any weight in the gradients.
  *
  * Ownership.  The caller allocates every buffer (device memory) and keeps it
- * alive until the work on `stream` has finished.  The library allocates no
- * memory.  `stream` is a cudaStream_t passed as void* (NULL = legacy default
+ * alive until the work on `stream` has finished.  No call allocates or frees
+ * memory.  The library's only device memory of its own is static: a 4-byte
+ * error word and the FA_NOALLOC_SCRATCH_BYTES (64 MiB) scratch array of
+ * fa_bwd_noalloc, both held by every device that loads the library, whether
+ * or not it ever calls fa_bwd_noalloc.
+ * `stream` is a cudaStream_t passed as void* (NULL = legacy default
  * stream).  Every call only enqueues work and returns; errors found on the
  * device are reported by fa_device_status().
  *

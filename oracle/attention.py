@@ -57,6 +57,7 @@ __all__ = [
     "attention_forward",
     "attention_backward",
     "head_forward_rows",
+    "head_backward_rows",
     "head_backward_sampled",
     "attention_forward_suffix",
     "attention_flops",
@@ -251,6 +252,35 @@ def attention_backward(q, k, v, do, scale, causal=False):
             dq[b, h] = scale * (ds @ k[b, g])
             dk[b, g] += scale * (ds.T @ q[b, h])
     return dq, dk, dv, o, lse
+
+
+def head_backward_rows(qh, kh, vh, doh, scale, causal, rows):
+    """The share of one block of query rows in the backward pass of one
+    (batch, query head).
+
+    Same formulas as :func:`attention_backward`, restricted to the query rows
+    ``rows`` (an index array): dQ of those rows is complete (it only involves
+    their own rows of P), while dK and dV are sums over query rows, so the
+    block contributes the partial sums  dV_part = P[rows]ᵀ dO[rows]  and
+    dK_part = s·dS[rows]ᵀ Q[rows].  Summing the partials of blocks that
+    partition all rows gives the head's dK and dV.
+
+    qh, doh: [N, d]; kh, vh: [N, d].  Returns (dq_rows [R, d], dk_part [N, d],
+    dv_part [N, d], o_rows [R, d], lse_rows [R])."""
+    qh = np.asarray(qh, np.float64)
+    kh = np.asarray(kh, np.float64)
+    vh = np.asarray(vh, np.float64)
+    doh = np.asarray(doh, np.float64)
+    rows = np.asarray(rows)
+    o_r, lse_r, p_r = head_forward_rows(qh, kh, vh, scale, causal, rows)
+    do_r = doh[rows]
+    dp_r = do_r @ vh.T
+    D_r = np.sum(do_r * o_r, axis=1, keepdims=True)
+    ds_r = p_r * (dp_r - D_r)
+    dq_r = scale * (ds_r @ kh)
+    dk_part = scale * (ds_r.T @ qh[rows])
+    dv_part = p_r.T @ do_r
+    return dq_r, dk_part, dv_part, o_r, lse_r
 
 
 def head_backward_sampled(q_heads, kh, vh, do_heads, scale, causal, q_rows, k_rows,

@@ -176,3 +176,33 @@ def _dec(lib, **kw):
 ])
 def test_decode_argument_validation(lib, kw, expect):
     assert _dec(lib, **kw) == expect
+
+
+def test_noalloc_scratch_size_matches_header():
+    # the binding's copy of FA_NOALLOC_SCRATCH_BYTES must equal the C #define
+    src = open(HEADER).read()
+    m = re.search(r"#define\s+FA_NOALLOC_SCRATCH_BYTES\s+\(([^)]*)\)", src)
+    assert m, "FA_NOALLOC_SCRATCH_BYTES not found in fa.h"
+    value = eval(m.group(1).replace("u", ""), {})  # e.g. "64u * 1024u * 1024u"
+    assert value == binding.FA_NOALLOC_SCRATCH_BYTES
+
+
+def _bwd_noalloc(lib, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5, do=FAKE * 6, dq=FAKE * 7, dk=FAKE * 8,
+             dv=FAKE * 9, B=1, Hq=2, Hkv=2, N=128, d=64, causal=0, scale=0.125)
+    a.update(kw)
+    return binding.fa_bwd_noalloc(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"], a["dv"],
+                                  a["B"], a["Hq"], a["Hkv"], a["N"], a["d"], a["causal"], a["scale"], 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), binding.FA_ERR_INVALID_ARG),                     # checked before the scratch lookup
+    (dict(dv=0), binding.FA_ERR_INVALID_ARG),
+    (dict(lse=FAKE * 5 + 4), binding.FA_ERR_INVALID_ARG),        # misaligned
+    (dict(Hq=3), binding.FA_ERR_INVALID_ARG),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(B=8, Hq=16, Hkv=16, N=2048, d=128), binding.FA_ERR_UNSUPPORTED),  # beyond the 64 MiB scratch
+    (dict(B=0), binding.FA_OK),
+])
+def test_noalloc_argument_validation(lib, kw, expect):
+    assert _bwd_noalloc(lib, **kw) == expect

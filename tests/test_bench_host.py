@@ -1,4 +1,5 @@
-"""Host-side helpers of bench.py (no GPU): the record of logit extremes."""
+"""Host-side helpers of bench.py (no GPU): the record of logit extremes and the
+bounded CPU-oracle sample."""
 
 import importlib.util
 import os
@@ -47,3 +48,30 @@ def test_logit_extremes_ignore_masked_pairs_and_other_heads():
 
 def test_single_rank_time_is_its_own_maximum():
     assert bench.reduce_max_over_ranks(2.5, 1, "cpu") == 2.5
+
+
+def test_cpu_sample_rows_are_bounded_strided_and_rotate():
+    from exact_attention_104_b200.workloads import WORKLOADS
+    w = WORKLOADS["long_b1_h16_n16384_d128_causal"]
+    seen = set()
+    for step in range(3 * w.Hq):
+        h, rows = bench.cpu_sample_rows(w, step)
+        assert h == step % w.Hq
+        assert len(rows) == bench.CPU_BLOCK_ENTRIES // w.N
+        assert rows.min() >= 0 and rows.max() < w.N
+        assert (rows[1:] - rows[:-1] == w.N // len(rows)).all()
+        seen.add(int(rows[0]))
+    assert seen == {0, 1, 2}
+    # a short sequence is sampled whole
+    h, rows = bench.cpu_sample_rows(WORKLOADS["train_b8_h16_n2048_d128"], 5)
+    assert h == 5 and list(rows) == list(range(2048))
+
+
+def test_cpu_sample_flops_count_visible_pairs():
+    import numpy as np
+    from exact_attention_104_b200.workloads import Workload
+    rows = np.array([0, 3, 9])
+    causal = Workload("c", 1, 1, 1, 10, 64, True)
+    full = Workload("f", 1, 1, 1, 10, 64, False)
+    assert bench.cpu_sample_flops(causal, rows) == 3.5 * 4 * 64 * (1 + 4 + 10)
+    assert bench.cpu_sample_flops(full, rows) == 3.5 * 4 * 64 * 3 * 10

@@ -288,6 +288,29 @@ def test_sampled_backward_equals_full(causal):
     np.testing.assert_allclose(dv_r, dv[0, 0][kr], rtol=1e-12, atol=1e-13)
 
 
+@pytest.mark.parametrize("causal", [False, True])
+def test_row_block_backward_partials_sum_to_full(causal):
+    # blocks of query rows (ragged sizes, one block strided) that partition all
+    # rows: dQ/O/LSE rows are the full ones, and the dK/dV partials add up to
+    # the full gradients of the head
+    N, d, s = 37, 5, 0.4
+    q, k, v, do = (_rand((1, 1, N, d), 40 + i) for i in range(4))
+    dq, dk, dv, o, lse = oracle.attention_backward(q, k, v, do, s, causal)
+    blocks = [np.arange(0, 37, 3), np.arange(1, 11, 3), np.setdiff1d(np.arange(N), np.concatenate(
+        [np.arange(0, 37, 3), np.arange(1, 11, 3)]))]
+    dk_sum, dv_sum = np.zeros((N, d)), np.zeros((N, d))
+    for rows in blocks:
+        dq_r, dk_p, dv_p, o_r, lse_r = oracle.head_backward_rows(q[0, 0], k[0, 0], v[0, 0], do[0, 0], s, causal,
+                                                                 rows)
+        np.testing.assert_allclose(dq_r, dq[0, 0][rows], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(o_r, o[0, 0][rows], rtol=1e-12, atol=1e-13)
+        np.testing.assert_allclose(lse_r, lse[0, 0][rows], rtol=1e-12, atol=1e-13)
+        dk_sum += dk_p
+        dv_sum += dv_p
+    np.testing.assert_allclose(dk_sum, dk[0, 0], rtol=1e-11, atol=1e-12)
+    np.testing.assert_allclose(dv_sum, dv[0, 0], rtol=1e-11, atol=1e-12)
+
+
 def test_flop_count():
     # 4·B·Hq·N²·d, halved when causal
     assert oracle.attention_flops(8, 16, 2048, 128, False) == 274877906944.0

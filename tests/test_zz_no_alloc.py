@@ -52,7 +52,7 @@ def test_noalloc_backward_matches_workspace_backward_on_two_calls(w):
 
 
 def test_noalloc_rejects_problems_larger_than_its_scratch():
-    w = Workload("na_big", 8, 16, 16, 2048, 128, False, 1.0, 64)  # needs 136 MiB of scratch
+    w = Workload("na_big", 8, 16, 16, 2048, 128, False, 1.0, 64)  # needs about 130 MiB (136 MB) of scratch
     assert binding.fa_bwd_workspace_bytes(w.B, w.Hq, w.Hkv, w.N, w.d) > binding.FA_NOALLOC_SCRATCH_BYTES
     shape_q = (w.B, w.Hq, w.N, w.d)
     t = lambda: torch.zeros(shape_q, dtype=torch.bfloat16, device="cuda")  # noqa: E731
