@@ -235,6 +235,13 @@ def decode_oracle_sample(w, seconds: float, max_batches: int | None = None):
     return w.fwd_flops() / w.B * done / t_total / 1e12, done, t_total
 
 
+def decode_split_kernel_name(w) -> str:
+    """The kernel fa_fwd_decode runs before its combine kernel: the CUDA-core
+    split kernel for at most 16 query rows per kv head (G·Nq), else the
+    tensor-core forward kernel in its decode mode."""
+    return "fa_decode_split_kernel" if w.G * w.Nq <= 16 else "fa_fwd_kernel (decode mode)"
+
+
 def run_decode(args, w, rank, world, local_rank):
     """One step = one fa_fwd_decode call over the whole decode workload (all
     batch entries and heads), K and V resident in HBM.  Reported in the same
@@ -343,7 +350,8 @@ def run_decode(args, w, rank, world, local_rank):
                    "causal": w.causal, "global_batch": w.B * world, "parallelism": f"dp{world}",
                    "l2": f"K/V {2 * w.B * w.Hkv * w.Nk * w.d * 2 / 2**20:.0f} MiB per step (> 126 MiB L2: no flush "
                          "needed)" if 4 * w.B * w.Hkv * w.Nk * w.d > 126 * 2**20 else "K/V fit in L2"},
-        "roofline": {"kernel": "fa_decode_split_kernel", "bound": "hbm", "achieved": gbs, "peak": peaks["hbm_gbs"],
+        "roofline": {"kernel": decode_split_kernel_name(w), "bound": "hbm", "achieved": gbs,
+                     "peak": peaks["hbm_gbs"],
                      "unit": "GB/s", "frac": gbs / peaks["hbm_gbs"],
                      "peak_source": peaks["source"] + " HBM copy (MEASURED_PEAKS.json)",
                      "bytes_per_launch": w.hbm_bytes(), "ms_per_launch": ms_split,
@@ -462,9 +470,9 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
 L2_BYTES = 126 * 2**20
 
 # dram__bytes_read.sum + dram__bytes_write.sum of one fa_bwd_kernel launch, from one ncu
-# capture of the current kernel (summarised under profiles/).  Must be reset
-# to None whenever fa_bwd_kernel changes.
-MEASURED_TRAFFIC = {"train_b8_h16_n2048_d128": 631.0e6}
+# capture of the current kernel (summarised under profiles/).  An entry must be
+# removed whenever fa_bwd_kernel changes.
+MEASURED_TRAFFIC = {"long_b1_h16_n16384_d128_causal": 628.1e6}
 
 # The same for one fa_decode_split_kernel launch (also summarised under profiles/);
 # reset to None whenever that kernel changes.

@@ -15,6 +15,12 @@ from .binding import (  # noqa: F401
     attention_forward,
     attention_backward,
     attention_decode,
+    attention_forward_varlen,
+    attention_backward_varlen,
+    fa_fwd_varlen,
+    fa_bwd_varlen,
+    fa_fwd_varlen_workspace_bytes,
+    fa_bwd_varlen_workspace_bytes,
     fa_fwd_decode,
     fa_decode_workspace_bytes,
     lib,

@@ -63,6 +63,14 @@ def lib() -> ctypes.CDLL:
     L.fa_decode_workspace_bytes.restype = z
     L.fa_fwd_decode.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, z, vp]
     L.fa_fwd_decode.restype = i
+    L.fa_fwd_varlen_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    L.fa_fwd_varlen_workspace_bytes.restype = z
+    L.fa_bwd_varlen_workspace_bytes.argtypes = [i, i, i, i, i, i]
+    L.fa_bwd_varlen_workspace_bytes.restype = z
+    L.fa_fwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, z, vp]
+    L.fa_fwd_varlen.restype = i
+    L.fa_bwd_varlen.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, i, f, vp, z, vp]
+    L.fa_bwd_varlen.restype = i
     _lib = L
     return L
 
@@ -147,6 +155,33 @@ def fa_fwd_decode(q, k, v, o, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, workspa
                                _stream_handle(stream))
 
 
+def fa_fwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d) -> int:
+    return int(lib().fa_fwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d))
+
+
+def fa_bwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d) -> int:
+    return int(lib().fa_bwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d))
+
+
+def fa_fwd_varlen(q, k, v, o, lse, cu_seqlens, nseq, Hq, Hkv, T, max_seqlen, d, causal, scale, workspace,
+                  workspace_bytes, stream=None) -> int:
+    """Raw C-ABI call of the packed variable-length forward pass (sequences
+    back to back along the token axis of [H, T, d] tensors, boundaries in the
+    device int32 tensor cu_seqlens).  Returns the status."""
+    return lib().fa_fwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(cu_seqlens), nseq, Hq, Hkv, T,
+                               max_seqlen, d, int(bool(causal)), float(scale), _ptr(workspace),
+                               int(workspace_bytes), _stream_handle(stream))
+
+
+def fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu_seqlens, nseq, Hq, Hkv, T, max_seqlen, d, causal, scale,
+                  workspace, workspace_bytes, stream=None) -> int:
+    """Raw C-ABI call of the packed variable-length backward pass.  Returns
+    the status."""
+    return lib().fa_bwd_varlen(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), _ptr(do), _ptr(dq), _ptr(dk),
+                               _ptr(dv), _ptr(cu_seqlens), nseq, Hq, Hkv, T, max_seqlen, d, int(bool(causal)),
+                               float(scale), _ptr(workspace), int(workspace_bytes), _stream_handle(stream))
+
+
 def fa_profile_next(start_event=None, stop_event=None) -> int:
     """Ask the next fa_fwd / fa_bwd call on this thread to record the given
     torch.cuda.Event objects around its attention kernel."""
@@ -226,3 +261,53 @@ def attention_decode(q, k, v, causal=False, scale=None, out=None, lse=None, work
     _check(fa_fwd_decode(q, k, v, out, lse, B, Hq, Hkv, Nq, Nk, d, causal, scale, workspace,
                          workspace.numel() * workspace.element_size(), stream), "fa_fwd_decode")
     return out, lse
+
+
+def _varlen_shapes(q, k, v, cu_seqlens):
+    if q.dim() != 3 or k.dim() != 3 or k.shape != v.shape:
+        raise FAError(FA_ERR_INVALID_ARG, "varlen: q must be [Hq, T, d] and k, v [Hkv, T, d]")
+    Hq, T, d = q.shape
+    if k.shape[1] != T or k.shape[2] != d:
+        raise FAError(FA_ERR_INVALID_ARG, "varlen: token or head dimension mismatch")
+    for t in (q, k, v):
+        if t.dtype != torch.bfloat16 or not t.is_cuda or not t.is_contiguous():
+            raise FAError(FA_ERR_INVALID_ARG, "varlen: q, k, v must be contiguous bf16 CUDA tensors")
+    if cu_seqlens.dtype != torch.int32 or not cu_seqlens.is_cuda or cu_seqlens.dim() != 1:
+        raise FAError(FA_ERR_INVALID_ARG, "varlen: cu_seqlens must be a 1-D int32 CUDA tensor")
+    return Hq, k.shape[0], T, d, cu_seqlens.numel() - 1
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, max_seqlen, causal=False, scale=None, out=None, lse=None,
+                             workspace=None, stream=None):
+    """O, LSE of a packed batch: q [Hq, T, d], k, v [Hkv, T, d] bf16 with the
+    sequences back to back along T (boundaries in the int32 CUDA tensor
+    cu_seqlens); each sequence attends only to itself.  max_seqlen bounds
+    every length.  Returns (o bf16 [Hq, T, d], lse fp32 [Hq, T])."""
+    Hq, Hkv, T, d, nseq = _varlen_shapes(q, k, v, cu_seqlens)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    if out is None:
+        out = torch.empty_like(q)
+    if lse is None:
+        lse = torch.empty(Hq, T, dtype=torch.float32, device=q.device)
+    need = fa_fwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(fa_fwd_varlen(q, k, v, out, lse, cu_seqlens, nseq, Hq, Hkv, T, max_seqlen, d, causal, scale, workspace,
+                         workspace.numel() * workspace.element_size(), stream), "fa_fwd_varlen")
+    return out, lse
+
+
+def attention_backward_varlen(q, k, v, o, lse, do, cu_seqlens, max_seqlen, causal=False, scale=None, dq=None,
+                              dk=None, dv=None, workspace=None, stream=None):
+    """dQ, dK, dV of a packed batch given the forward outputs and dO."""
+    Hq, Hkv, T, d, nseq = _varlen_shapes(q, k, v, cu_seqlens)
+    scale = 1.0 / math.sqrt(d) if scale is None else scale
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    need = fa_bwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d)
+    if workspace is None:
+        workspace = torch.empty(max(need, 256), dtype=torch.uint8, device=q.device)
+    _check(fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu_seqlens, nseq, Hq, Hkv, T, max_seqlen, d, causal,
+                         scale, workspace, workspace.numel() * workspace.element_size(), stream), "fa_bwd_varlen")
+    return dq, dk, dv

@@ -15,6 +15,7 @@
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 #include "fa_fwd_persistent.cuh"
+#include "fa_varlen.cuh"
 
 // Scratch of fa_bwd_noalloc: a fixed device array instead of a caller buffer.
 // Host code must not pass this symbol to a kernel (on the host it names a
@@ -174,14 +175,16 @@ bool reg_split_fits(Kern kern) {
   return r >= C::MIN_LAUNCH_REGS && r <= C::MAX_LAUNCH_REGS;
 }
 
-template <int D, bool CAUSAL, bool TAIL>
+// grid_units > 0 (VARLEN): a 1-D grid of that many CTAs instead of
+// (query tiles, Hq, B).
+template <int D, bool CAUSAL, bool TAIL, bool VARLEN = false>
 fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv, const fa::FwdParams& p,
-                     int B, int Hq, cudaStream_t stream) {
-  using C = fa::FwdCfg<D>;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, TAIL>;
+                     int B, int Hq, cudaStream_t stream, long long grid_units = 0) {
+  using C = fa::FwdCfg<D, 1>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, TAIL, VARLEN ? fa::kFwdVarlen : fa::kFwdDense>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
-  dim3 grid((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
+  const dim3 grid = VARLEN ? dim3((unsigned)grid_units) : dim3((p.n_qtiles + C::NQ - 1) / C::NQ, Hq, B);
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -189,15 +192,15 @@ fa_status launch_fwd(const CUtensorMap& tq, const CUtensorMap& tk, const CUtenso
 
 // Two query tiles per item (d = 64, 128): one persistent CTA per SM walks the
 // item list.  d = 256: one CTA per 128-row query tile (launch_fwd).
-template <int D, bool CAUSAL, bool TAIL>
+template <int D, bool CAUSAL, bool TAIL, bool VARLEN = false>
 fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                                 const fa::FwdParams& fp, int B, int Hq, int sms, cudaStream_t stream) {
   using C = fa::FwdPCfg<D>;
-  auto kern = fa::fa_fwd_persistent_kernel<D, CAUSAL, TAIL>;
+  auto kern = fa::fa_fwd_persistent_kernel<D, CAUSAL, TAIL, VARLEN>;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
   if (!reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
-  fa::FwdPParams p;
+  fa::FwdPParams p{};
   p.o = fp.o;
   p.lse = fp.lse;
   p.N = fp.N;
@@ -212,7 +215,12 @@ fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, co
   p.scale_log2 = fp.scale_log2;
   p.wait_cap = fp.wait_cap;
   p.err = fp.err;
-  const int grid = p.n_items < sms ? p.n_items : sms;
+  p.table = fp.table;
+  p.cu = fp.cu;
+  p.hdr = fp.hdr;
+  p.T = fp.T;
+  // VARLEN: the item count is only known on the device; one CTA per SM
+  const int grid = (!VARLEN && p.n_items < sms) ? p.n_items : sms;
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
@@ -224,24 +232,35 @@ fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, co
 #define FA_BWD_PERSISTENT 1
 #endif
 
-template <int D, bool CAUSAL, bool TAIL>
-fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
-                          const CUtensorMap& tdo, fa::BwdParams p, int B, int Hkv, int sms, cudaStream_t stream) {
+// dq_rows: rows of the fp32 dQ accumulator; units: work units, or (VARLEN)
+// an upper bound on them (the kernel reads the true count from the table).
+template <int D, bool CAUSAL, bool TAIL, bool VARLEN>
+fa_status launch_bwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                            const CUtensorMap& tdo, const fa::BwdParams& p, uint64_t dq_rows, long long units,
+                            int sms, cudaStream_t stream) {
   using C = fa::BwdCfg<D>;
-  auto kern = fa::fa_bwd_kernel<D, CAUSAL, TAIL>;
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL, TAIL, VARLEN>;
   if (C::REG_SPLIT && !reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
   CUtensorMap tdq;
-  if (!make_map_f32(&tdq, p.dqacc, (uint64_t)B * p.Hq * p.Np, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
+  if (!make_map_f32(&tdq, p.dqacc, dq_rows, D, C::DH, C::STG_ROWS)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
-  const long long units = (long long)((p.N + C::BC - 1) / C::BC) * C::NDH * Hkv * B;
-  if (units >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
-  p.n_units = (int)units;
   const bool persistent = FA_BWD_PERSISTENT && D <= 128;
   const dim3 grid((unsigned)(persistent && units > sms ? sms : units));
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, tdo, tdq, p);
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+template <int D, bool CAUSAL, bool TAIL>
+fa_status launch_bwd_main(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
+                          const CUtensorMap& tdo, fa::BwdParams p, int B, int Hkv, int sms, cudaStream_t stream) {
+  using C = fa::BwdCfg<D>;
+  const long long units = (long long)((p.N + C::BC - 1) / C::BC) * C::NDH * Hkv * B;
+  if (units >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  p.n_units = (int)units;
+  return launch_bwd_kernel<D, CAUSAL, TAIL, false>(tq, tk, tv, tdo, p, (uint64_t)B * p.Hq * p.Np, units, sms,
+                                                   stream);
 }
 
 template <int D>
@@ -283,6 +302,48 @@ fa_status noalloc_scratch(void** out) {
   return FA_OK;
 }
 
+// ----------------------------------------------------------------- varlen
+// Checks shared by the varlen entry points; *empty for nothing to compute.
+fa_status varlen_sizes(int nseq, int Hq, int Hkv, int T, int max_seqlen, int d, float scale, bool* empty) {
+  *empty = false;
+  if (nseq < 0 || T < 0 || Hq <= 0 || Hkv <= 0 || d <= 0) return FA_ERR_INVALID_ARG;
+  if (Hq % Hkv != 0) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !(scale > 0.f)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128 && d != 256) return FA_ERR_UNSUPPORTED;
+  if (nseq == 0 || T == 0) {
+    *empty = true;
+    return FA_OK;
+  }
+  if (max_seqlen < 1) return FA_ERR_INVALID_ARG;
+  if (max_seqlen > fa::kVarlenMaxSeqlen) return FA_ERR_UNSUPPORTED;
+  if (Hq > 65535) return FA_ERR_UNSUPPORTED;
+  if ((long long)Hq * fa::varlen_tp(nseq, T) >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  // work units (one per 128-row tile, at most T/128 + nseq) times heads
+  if (((long long)(T + 127) / 128 + nseq) * Hq * 2 >= (1LL << 31)) return FA_ERR_UNSUPPORTED;
+  return FA_OK;
+}
+
+// Upper bound on the work-table entries (one per 128-row tile of a sequence).
+long long varlen_max_entries(int nseq, int T) { return (long long)(T + 127) / 128 + nseq; }
+size_t varlen_table_bytes(int nseq, int T) { return round256(8 * (size_t)varlen_max_entries(nseq, T)); }
+
+// The first kernel of a varlen call: check cu_seqlens and write the work table
+// of (sequence, unit) pairs, heaviest first, behind the header.
+fa_status launch_varlen_plan(const int* cu, int nseq, int T, int max_seqlen, int tpu, bool bwd, bool causal,
+                             uint8_t* ws, int* err, cudaStream_t s) {
+  const int max_key = (max_seqlen + 127) / 128;
+  const size_t smem = 2 * (size_t)(max_key + 1) * sizeof(int);
+  if (smem > 48 * 1024 &&
+      cudaFuncSetAttribute(fa::fa_varlen_plan_kernel, cudaFuncAttributeMaxDynamicSharedMemorySize, (int)smem) !=
+          cudaSuccess)
+    return FA_ERR_CUDA;
+  int* hdr = reinterpret_cast<int*>(ws);
+  int2* table = reinterpret_cast<int2*>(ws + fa::kVarlenHdrBytes);
+  fa::fa_varlen_plan_kernel<<<1, fa::kPlanThreads, smem, s>>>(cu, nseq, T, max_seqlen, max_key, tpu, bwd ? 1 : 0,
+                                                              causal ? 1 : 0, table, hdr, err);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 }  // namespace
 
 namespace fa {
@@ -306,15 +367,23 @@ __global__ void selftest_exp2_kernel(const float* __restrict__ x, float* __restr
 }  // namespace fa
 
 // ------------------------------------------------------------------ decode
-// Split plan of a decode call: row groups of RMAX (4, 8 or 16) query rows,
-// and enough key splits for about kDecodeCtas CTAs in all (a pure function of
-// the sizes, so that fa_decode_workspace_bytes needs no device).
+// Split plan of a decode call (a pure function of the sizes, so that
+// fa_decode_workspace_bytes needs no device).
+//  * R = G·Nq <= 16 query rows per kv head: the CUDA-core kernel, row groups
+//    of RMAX (4, 8 or 16) rows, 64-key tiles, enough key splits for about
+//    kDecodeCtas CTAs in all;
+//  * R > 16: the tensor-core kernel (fa_fwd_kernel, decode mode), row tiles
+//    of 128 rows, 128-key tiles, and about one CTA per SM of a B200
+//    (kDecodeTcCtas) in all: every CTA streams its key range once at HBM
+//    speed, so one wave with few, long splits keeps the partial results small.
 #ifndef FA_DECODE_CTAS
 #define FA_DECODE_CTAS 1024
 #endif
 constexpr int kDecodeCtas = FA_DECODE_CTAS;
+constexpr int kDecodeTcCtas = 148;
 constexpr int kDecodeMaxSplit = 256;
 struct DecodePlan {
+  bool tc = false;  // tensor-core kernel
   int rmax = 4, n_rg = 1, n_split = 1, tiles_per_split = 1;
   size_t part_o_bytes = 0, part_ml_bytes = 0;
 };
@@ -340,11 +409,12 @@ fa_status decode_sizes(int B, int Hq, int Hkv, int Nq, int Nk, int d, float scal
 DecodePlan decode_plan(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
   DecodePlan pl;
   const long long R = (long long)(Hq / Hkv) * Nq;
-  pl.rmax = R <= 4 ? 4 : (R <= 8 ? 8 : 16);
+  pl.tc = R > 16;
+  pl.rmax = pl.tc ? 128 : (R <= 4 ? 4 : (R <= 8 ? 8 : 16));
   pl.n_rg = (int)((R + pl.rmax - 1) / pl.rmax);
   const long long units = (long long)B * Hkv * pl.n_rg;
-  const int n_tiles = (Nk + 63) / 64;
-  long long want = (kDecodeCtas + units - 1) / units;
+  const int n_tiles = pl.tc ? (Nk + 127) / 128 : (Nk + 63) / 64;
+  long long want = pl.tc ? kDecodeTcCtas / units : (kDecodeCtas + units - 1) / units;
   if (want < 1) want = 1;
   int n_split = (int)std::min<long long>({want, (long long)n_tiles, (long long)kDecodeMaxSplit});
   pl.tiles_per_split = (n_tiles + n_split - 1) / n_split;
@@ -366,16 +436,51 @@ fa_status launch_decode_split(const fa::DecodeParams& p, unsigned units, cudaStr
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
+// The tensor-core split kernel of a decode call with R > 16 rows per kv head.
+template <int D, bool CAUSAL>
+fa_status launch_decode_tc(const fa::DecodeParams& dp, const void* q, const void* k, const void* v, float scale,
+                           const DeviceInfo* di, unsigned units, cudaStream_t s) {
+  using C = fa::FwdCfg<D, 1>;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, true, fa::kFwdDecode>;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, (uint64_t)dp.B * dp.Hq * dp.Nq, D, 128) ||
+      !make_map(&tk, k, (uint64_t)dp.B * dp.Hkv * dp.Nk, D, 128) ||
+      !make_map(&tv, v, (uint64_t)dp.B * dp.Hkv * dp.Nk, D, 128))
+    return FA_ERR_CUDA;
+  fa::FwdParams p{};
+  p.Hq = dp.Hq;
+  p.Hkv = dp.Hkv;
+  p.G = dp.G;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.wait_cap = g_wait_cap.load(std::memory_order_relaxed);
+  p.err = di->err;
+  p.Nq = dp.Nq;
+  p.Nk = dp.Nk;
+  p.R = dp.R;
+  p.n_rt = dp.n_rg;
+  p.n_split = dp.n_split;
+  p.tiles_per_split = dp.tiles_per_split;
+  p.part_o = dp.part_o;
+  p.part_ml = dp.part_ml;
+  ProfileScope prof(s);
+  kern<<<dim3((unsigned)dp.n_split, units), C::THREADS, C::SMEM_BYTES, s>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
 template <int D>
 fa_status launch_decode(const fa::DecodeParams& p, int rmax, bool causal, unsigned units, cudaStream_t s) {
   fa_status st;
   switch (rmax) {
+    case 128: st = FA_OK; break;  // the tensor-core split kernel was launched by the caller
     case 4: st = causal ? launch_decode_split<D, 4, true>(p, units, s) : launch_decode_split<D, 4, false>(p, units, s); break;
     case 8: st = causal ? launch_decode_split<D, 8, true>(p, units, s) : launch_decode_split<D, 8, false>(p, units, s); break;
     default: st = causal ? launch_decode_split<D, 16, true>(p, units, s) : launch_decode_split<D, 16, false>(p, units, s); break;
   }
   if (st != FA_OK) return st;
   switch (rmax) {
+    case 128: fa::fa_decode_combine_kernel<D, 128><<<units, 256, 0, s>>>(p); break;
     case 4: fa::fa_decode_combine_kernel<D, 4><<<units, 256, 0, s>>>(p); break;
     case 8: fa::fa_decode_combine_kernel<D, 8><<<units, 256, 0, s>>>(p); break;
     default: fa::fa_decode_combine_kernel<D, 16><<<units, 256, 0, s>>>(p); break;
@@ -463,7 +568,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   const uint64_t qrows = (uint64_t)B * Hq * N, kvrows = (uint64_t)B * Hkv * N;
   if (!make_map(&tq, q, qrows, d, 128) || !make_map(&tk, k, kvrows, d, 128) || !make_map(&tv, v, kvrows, d, 128))
     return FA_ERR_CUDA;
-  fa::FwdParams p;
+  fa::FwdParams p{};
   p.o = static_cast<__nv_bfloat16*>(o);
   p.lse = lse;
   p.N = N;
@@ -549,7 +654,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
   if (!make_map(&tq, q, rows, d, 64) || !make_map(&tdo, dout, rows, d, 64) || !make_map(&tk, k, kvrows, d, 128) ||
       !make_map(&tv, v, kvrows, d, 128))
     return FA_ERR_CUDA;
-  fa::BwdParams p;
+  fa::BwdParams p{};
   p.lse2 = lse2;
   p.dvec = dvec;
   p.dqacc = dqacc;
@@ -619,7 +724,9 @@ fa_status fa_device_status(void* stream) {
   if (host != 0 && cudaMemcpy(di->err, &zero, sizeof(int), cudaMemcpyHostToDevice) != cudaSuccess)
     return FA_ERR_CUDA;
   if (host == 0) return FA_OK;
-  return (host & 0xff) == fa::kDevCheck ? FA_ERR_DEVICE_CHECK : FA_ERR_TIMEOUT;
+  if ((host & 0xff) == fa::kDevCheck) return FA_ERR_DEVICE_CHECK;
+  if ((host & 0xff) == fa::kDevBadSeqlens) return FA_ERR_INVALID_ARG;
+  return FA_ERR_TIMEOUT;
 }
 
 fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
@@ -644,6 +751,208 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
   if (st != FA_OK) return st;
   return fa_bwd(q, k, v, o, lse, dout, dq, dk, dv, B, Hq, Hkv, N, d, causal, scale, scratch,
                 (size_t)FA_NOALLOC_SCRATCH_BYTES, stream);
+}
+
+size_t fa_fwd_varlen_workspace_bytes(int nseq, int Hq, int Hkv, int T, int max_seqlen, int d) {
+  bool empty = false;
+  if (varlen_sizes(nseq, Hq, Hkv, T, max_seqlen, d, 1.f, &empty) != FA_OK) return 0;
+  if (empty) return fa::kVarlenHdrBytes;
+  return fa::kVarlenHdrBytes + varlen_table_bytes(nseq, T);
+}
+
+size_t fa_bwd_varlen_workspace_bytes(int nseq, int Hq, int Hkv, int T, int max_seqlen, int d) {
+  bool empty = false;
+  if (varlen_sizes(nseq, Hq, Hkv, T, max_seqlen, d, 1.f, &empty) != FA_OK) return 0;
+  if (empty) return fa::kVarlenHdrBytes;
+  const size_t rows_p = (size_t)Hq * fa::varlen_tp(nseq, T);
+  // header, work table, D and lse2 rows, fp32 dQ accumulator, unit counter
+  return fa::kVarlenHdrBytes + varlen_table_bytes(nseq, T) + 2 * round256(rows_p * 4) +
+         round256(rows_p * (size_t)d * 4) + 256;
+}
+
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int nseq, int Hq, int Hkv, int T, int max_seqlen, int d, int causal, float scale,
+                        void* workspace, size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status st = varlen_sizes(nseq, Hq, Hkv, T, max_seqlen, d, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !lse || !cu_seqlens || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_fwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d);
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)Hq * T * d * 2, kvbytes = (size_t)Hkv * T * d * 2;
+  const Range ins[4] = {span(q, qbytes), span(k, kvbytes), span(v, kvbytes), span(cu_seqlens, 4 * (size_t)(nseq + 1))};
+  const Range outs[3] = {span(o, qbytes), span(lse, (size_t)Hq * T * 4), span(workspace, need)};
+  for (int i = 0; i < 3; ++i) {
+    for (int j = 0; j < 4; ++j)
+      if (overlap(outs[i], ins[j])) return FA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 3; ++j)
+      if (overlap(outs[i], outs[j])) return FA_ERR_INVALID_ARG;
+  }
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  st = launch_varlen_plan(cu_seqlens, nseq, T, max_seqlen, d <= 128 ? 2 : 1, false, causal != 0, ws, di->err, s);
+  if (st != FA_OK) return st;
+  CUtensorMap tq, tk, tv;
+  if (!make_map(&tq, q, (uint64_t)Hq * T, d, 128) || !make_map(&tk, k, (uint64_t)Hkv * T, d, 128) ||
+      !make_map(&tv, v, (uint64_t)Hkv * T, d, 128))
+    return FA_ERR_CUDA;
+  fa::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = T;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = 0;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.wait_cap = g_wait_cap.load(std::memory_order_relaxed);
+  p.err = di->err;
+  p.table = reinterpret_cast<const int2*>(ws + fa::kVarlenHdrBytes);
+  p.cu = cu_seqlens;
+  p.hdr = reinterpret_cast<const int*>(ws);
+  p.T = T;
+  const long long grid_units = varlen_max_entries(nseq, T) * Hq;  // d = 256: one CTA per (tile, head)
+  auto dispatch = [&](auto dtag) -> fa_status {
+    constexpr int D = decltype(dtag)::value;
+    if constexpr (D <= 128) {
+      return causal ? launch_fwd_persistent<D, true, true, true>(tq, tk, tv, p, 1, Hq, di->sms, s)
+                    : launch_fwd_persistent<D, false, true, true>(tq, tk, tv, p, 1, Hq, di->sms, s);
+    } else {
+      return causal ? launch_fwd<D, true, true, true>(tq, tk, tv, p, 1, Hq, s, grid_units)
+                    : launch_fwd<D, false, true, true>(tq, tk, tv, p, 1, Hq, s, grid_units);
+    }
+  };
+  switch (d) {
+    case 64: return dispatch(std::integral_constant<int, 64>{});
+    case 128: return dispatch(std::integral_constant<int, 128>{});
+    default: return dispatch(std::integral_constant<int, 256>{});
+  }
+}
+
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv, const int* cu_seqlens, int nseq, int Hq,
+                        int Hkv, int T, int max_seqlen, int d, int causal, float scale, void* workspace,
+                        size_t workspace_bytes, void* stream) {
+  bool empty = false;
+  fa_status st = varlen_sizes(nseq, Hq, Hkv, T, max_seqlen, d, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (!q || !k || !v || !o || !lse || !dout || !dq || !dk || !dv || !cu_seqlens || !workspace)
+    return FA_ERR_INVALID_ARG;
+  for (const void* ptr : {q, k, v, o, (const void*)lse, dout, (const void*)dq, (const void*)dk, (const void*)dv})
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, max_seqlen, d);
+  if (workspace_bytes < need) return FA_ERR_INVALID_ARG;
+  const size_t rows = (size_t)Hq * T;
+  const size_t qbytes = rows * d * 2, kvbytes = (size_t)Hkv * T * d * 2;
+  const Range ins[7] = {span(q, qbytes),  span(k, kvbytes),    span(v, kvbytes),
+                        span(o, qbytes),  span(lse, rows * 4), span(dout, qbytes),
+                        span(cu_seqlens, 4 * (size_t)(nseq + 1))};
+  const Range outs[4] = {span(dq, qbytes), span(dk, kvbytes), span(dv, kvbytes), span(workspace, need)};
+  for (int i = 0; i < 4; ++i) {
+    for (int j = 0; j < 7; ++j)
+      if (overlap(outs[i], ins[j])) return FA_ERR_INVALID_ARG;
+    for (int j = i + 1; j < 4; ++j)
+      if (overlap(outs[i], outs[j])) return FA_ERR_INVALID_ARG;
+  }
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+
+  // workspace: header | work table | D | lse2 | fp32 dQ accumulator | unit counter
+  const int Tp = (int)fa::varlen_tp(nseq, T);
+  const size_t rows_p = (size_t)Hq * Tp;
+  uint8_t* ws = static_cast<uint8_t*>(workspace);
+  const size_t tb = varlen_table_bytes(nseq, T);
+  float* dvec = reinterpret_cast<float*>(ws + fa::kVarlenHdrBytes + tb);
+  float* lse2 = reinterpret_cast<float*>(ws + fa::kVarlenHdrBytes + tb + round256(rows_p * 4));
+  float* dqacc = reinterpret_cast<float*>(ws + fa::kVarlenHdrBytes + tb + 2 * round256(rows_p * 4));
+  int* unit_counter = reinterpret_cast<int*>(ws + fa::kVarlenHdrBytes + tb + 2 * round256(rows_p * 4) +
+                                             round256(rows_p * (size_t)d * 4));
+  const int* hdr = reinterpret_cast<const int*>(ws);
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+
+  st = launch_varlen_plan(cu_seqlens, nseq, T, max_seqlen, 1, true, causal != 0, ws, di->err, s);
+  if (st != FA_OK) return st;
+  {
+    const long long dq_vec4 = (long long)rows_p * d / 4;
+    long long want = (long long)rows_p * (d / 8);
+    if (dq_vec4 > want) want = dq_vec4;
+    long long blocks = (want + 255) / 256;
+    if (blocks > (long long)di->sms * 8) blocks = (long long)di->sms * 8;
+    if (blocks < 1) blocks = 1;
+    auto pre = [&](auto kern) {
+      kern<<<(unsigned)blocks, 256, 0, s>>>(static_cast<const __nv_bfloat16*>(o),
+                                            static_cast<const __nv_bfloat16*>(dout), lse, dvec, lse2, dqacc,
+                                            unit_counter, cu_seqlens, hdr, nseq, T, Tp, (long long)rows_p, dq_vec4);
+    };
+    switch (d) {
+      case 64: pre(fa::fa_bwd_pre_varlen_kernel<64>); break;
+      case 128: pre(fa::fa_bwd_pre_varlen_kernel<128>); break;
+      default: pre(fa::fa_bwd_pre_varlen_kernel<256>); break;
+    }
+    if (cudaGetLastError() != cudaSuccess) return FA_ERR_CUDA;
+  }
+
+  CUtensorMap tq, tk, tv, tdo;
+  const uint64_t kvrows = (uint64_t)Hkv * T;
+  if (!make_map(&tq, q, rows, d, 64) || !make_map(&tdo, dout, rows, d, 64) || !make_map(&tk, k, kvrows, d, 128) ||
+      !make_map(&tv, v, kvrows, d, 128))
+    return FA_ERR_CUDA;
+  fa::BwdParams p{};
+  p.lse2 = lse2;
+  p.dvec = dvec;
+  p.dqacc = dqacc;
+  p.dk = static_cast<__nv_bfloat16*>(dk);
+  p.dv = static_cast<__nv_bfloat16*>(dv);
+  p.N = T;
+  p.Np = Tp;
+  p.B = 1;
+  p.jt_band = 1;
+  p.n_units = 0;
+  p.unit_counter = unit_counter;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.scale = scale;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.wait_cap = g_wait_cap.load(std::memory_order_relaxed);
+  p.err = di->err;
+  p.table = reinterpret_cast<const int2*>(ws + fa::kVarlenHdrBytes);
+  p.cu = cu_seqlens;
+  p.hdr = hdr;
+  p.T = T;
+  p.Tp = Tp;
+  auto main_kernel = [&](auto dtag) -> fa_status {
+    constexpr int D = decltype(dtag)::value;
+    const long long units = varlen_max_entries(nseq, T) * Hkv * fa::BwdCfg<D>::NDH;  // upper bound
+    return causal ? launch_bwd_kernel<D, true, true, true>(tq, tk, tv, tdo, p, rows_p, units, di->sms, s)
+                  : launch_bwd_kernel<D, false, true, true>(tq, tk, tv, tdo, p, rows_p, units, di->sms, s);
+  };
+  switch (d) {
+    case 64: st = main_kernel(std::integral_constant<int, 64>{}); break;
+    case 128: st = main_kernel(std::integral_constant<int, 128>{}); break;
+    default: st = main_kernel(std::integral_constant<int, 256>{}); break;
+  }
+  if (st != FA_OK) return st;
+
+  long long blocks = ((long long)rows + 7) / 8;  // 8 warps (rows) per block
+  if (blocks > (long long)di->sms * 16) blocks = (long long)di->sms * 16;
+  __nv_bfloat16* dq16 = static_cast<__nv_bfloat16*>(dq);
+  switch (d) {
+    case 64: fa::fa_dq_convert_varlen_kernel<64><<<(unsigned)blocks, 256, 0, s>>>(dqacc, dq16, scale, cu_seqlens, hdr, nseq, T, Tp, (long long)rows); break;
+    case 128: fa::fa_dq_convert_varlen_kernel<128><<<(unsigned)blocks, 256, 0, s>>>(dqacc, dq16, scale, cu_seqlens, hdr, nseq, T, Tp, (long long)rows); break;
+    default: fa::fa_dq_convert_varlen_kernel<256><<<(unsigned)blocks, 256, 0, s>>>(dqacc, dq16, scale, cu_seqlens, hdr, nseq, T, Tp, (long long)rows); break;
+  }
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
 size_t fa_decode_workspace_bytes(int B, int Hq, int Hkv, int Nq, int Nk, int d) {
@@ -702,6 +1011,20 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
   if (n_units > 65535) return FA_ERR_UNSUPPORTED;  // grid.y of the split kernel
   const unsigned units = (unsigned)n_units;
   cudaStream_t s = static_cast<cudaStream_t>(stream);
+  if (pl.tc) {
+    if ((long long)B * Hq * Nq >= (1LL << 31) - 128) return FA_ERR_UNSUPPORTED;  // row index of the last Q box
+    auto tc = [&](auto dtag) -> fa_status {
+      constexpr int D = decltype(dtag)::value;
+      return causal ? launch_decode_tc<D, true>(p, q, k, v, scale, di, units, s)
+                    : launch_decode_tc<D, false>(p, q, k, v, scale, di, units, s);
+    };
+    switch (d) {
+      case 64: st = tc(std::integral_constant<int, 64>{}); break;
+      case 128: st = tc(std::integral_constant<int, 128>{}); break;
+      default: st = tc(std::integral_constant<int, 256>{}); break;
+    }
+    if (st != FA_OK) return st;
+  }
   switch (d) {
     case 64: return launch_decode<64>(p, pl.rmax, causal != 0, units, s);
     case 128: return launch_decode<128>(p, pl.rmax, causal != 0, units, s);

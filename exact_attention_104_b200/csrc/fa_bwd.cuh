@@ -26,6 +26,7 @@
 // and dPᵀ over the full head dimension.
 #pragma once
 
+#include "fa_varlen.cuh"
 #include "sm100.cuh"
 
 namespace fa {
@@ -194,6 +195,13 @@ struct BwdParams {
   float scale, scale_log2;
   long long wait_cap;
   int* err;
+  // VARLEN only: packed sequences of T tokens per head (Tp padded workspace
+  // rows per head), cu_seqlens, and the work table of (sequence, key tile)
+  // units with its header (hdr[0] units)
+  const int2* table;
+  const int* cu;
+  const int* hdr;
+  int T, Tp;
 };
 
 // One unit of backward work: a 128-key tile (and, at d = 256, one half of the
@@ -203,30 +211,73 @@ struct BwdParams {
 // p.jt_band, earliest band first, head by head inside a band: CTAs running at
 // the same time share Q/dO tiles in L2, and with a causal mask the heavy bands
 // (early key tiles, more query steps) run first.
+// len: the sequence's length; qrow(head) / qprow(head) / kvrow: rows of its
+// first token in the Q/dO (and dQ output), padded workspace and K/V tensors.
 struct BwdUnit {
-  int jt, dh, hkv, b, i_start, per_head, n;
+  int jt, dh, hkv, i_start, per_head, n;
+  int len, start, pstart, b;
 };
 
-template <int D, bool CAUSAL>
-__device__ __forceinline__ BwdUnit bwd_unit(int idx, const BwdParams& p) {
+// A packed batch's units (VARLEN; ne = hdr[0] table entries): causal units
+// heaviest first across kv heads, non-causal ones kv head by kv head, the
+// d-halves of a key tile adjacent.
+template <int D, bool CAUSAL, bool VARLEN>
+__device__ __forceinline__ BwdUnit bwd_unit(int idx, const BwdParams& p, int ne) {
   using C = BwdCfg<D>;
-  const int n_kt = (p.N + C::BC - 1) / C::BC;
-  const int U = C::NDH * p.Hkv * p.B;  // units per key tile
-  const int bi = idx / (p.jt_band * U);
-  const int wb = min(p.jt_band, n_kt - bi * p.jt_band);  // key tiles in this band
-  const int rb = idx - bi * p.jt_band * U;
-  const int bh = rb / (wb * C::NDH);
-  const int rem = rb - bh * (wb * C::NDH);
   BwdUnit u;
-  u.jt = bi * p.jt_band + rem / C::NDH;
-  u.dh = rem % C::NDH;
-  u.hkv = bh % p.Hkv;
-  u.b = bh / p.Hkv;
-  const int nqt = (p.N + C::BR - 1) / C::BR;
+  if (VARLEN) {
+    u.dh = idx % C::NDH;
+    const int rest = idx / C::NDH;
+    int e;
+    if (CAUSAL) {
+      e = rest / p.Hkv;
+      u.hkv = rest % p.Hkv;
+    } else {
+      u.hkv = rest / ne;
+      e = rest % ne;
+    }
+    const int2 ent = p.table[e];
+    u.b = ent.x;
+    u.jt = ent.y;
+    u.start = p.cu[ent.x];
+    u.len = p.cu[ent.x + 1] - u.start;
+    u.pstart = varlen_pstart(ent.x, u.start);
+  } else {
+    const int n_kt = (p.N + C::BC - 1) / C::BC;
+    const int U = C::NDH * p.Hkv * p.B;  // units per key tile
+    const int bi = idx / (p.jt_band * U);
+    const int wb = min(p.jt_band, n_kt - bi * p.jt_band);  // key tiles in this band
+    const int rb = idx - bi * p.jt_band * U;
+    const int bh = rb / (wb * C::NDH);
+    const int rem = rb - bh * (wb * C::NDH);
+    u.jt = bi * p.jt_band + rem / C::NDH;
+    u.dh = rem % C::NDH;
+    u.hkv = bh % p.Hkv;
+    u.b = bh / p.Hkv;
+    u.len = p.N;
+    u.start = 0;
+    u.pstart = 0;
+  }
+  const int nqt = (u.len + C::BR - 1) / C::BR;
   u.i_start = CAUSAL ? (u.jt * C::BC) / C::BR : 0;
   u.per_head = nqt - u.i_start;
   u.n = p.G * u.per_head;  // query steps
   return u;
+}
+
+// Row of query row 0 of query head `head` in Q / dO / dQ, and in the padded
+// workspace arrays; row of key 0 of the unit's kv head in K / V / dK / dV.
+template <bool VARLEN>
+__device__ __forceinline__ int bwd_qrow(const BwdUnit& u, int head, const BwdParams& p) {
+  return VARLEN ? head * p.T + u.start : (u.b * p.Hq + head) * p.N;
+}
+template <bool VARLEN>
+__device__ __forceinline__ int bwd_qprow(const BwdUnit& u, int head, const BwdParams& p) {
+  return VARLEN ? head * p.Tp + u.pstart : (u.b * p.Hq + head) * p.Np;
+}
+template <bool VARLEN>
+__device__ __forceinline__ int bwd_kvrow(const BwdUnit& u, const BwdParams& p) {
+  return VARLEN ? u.hkv * p.T + u.start : (u.b * p.Hkv + u.hkv) * p.N;
 }
 
 // TAIL: N is not a multiple of 128 (keys and queries past N get P = 0, rows past
@@ -243,18 +294,23 @@ __device__ __forceinline__ BwdUnit bwd_unit(int idx, const BwdParams& p) {
 // dV / dK products wait until the previous unit's accumulators have been read
 // out of TMEM (b_dvfree / b_dkfree), so its epilogue overlaps the next unit's
 // first loads and products.
-template <int D, bool CAUSAL, bool TAIL>
+// VARLEN: a packed batch of sequences (always with TAIL); units come from
+// the work table, each with its own length and row bases.
+template <int D, bool CAUSAL, bool TAIL, bool VARLEN = false>
 __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmDO,
                   const __grid_constant__ CUtensorMap tmDQ, const BwdParams p) {
   using C = BwdCfg<D>;
+  static_assert(!VARLEN || TAIL, "packed sequences have ragged ends");
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
   auto BAR = [&](int i) -> uint32_t { return sbase + C::BAR_OFF + 8 * i; };
   uint32_t* tmem_holder = reinterpret_cast<uint32_t*>(smem + C::MISC_OFF);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::MISC_OFF + 4);
+  const int ne = VARLEN ? p.hdr[0] : 0;
+  const int n_units = VARLEN ? ne * p.Hkv * C::NDH : p.n_units;
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
@@ -327,15 +383,15 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (uc >= 2 && !mbar_wait(BAR(C::B_UNITEMPTY + (uc & 1)), ((uc >> 1) - 1) & 1, wc, 27)) break;
         unit_slot[uc & 1] = idx;
         mbar_arrive(BAR(C::B_UNITFULL + (uc & 1)));
-        if (idx >= p.n_units) break;
-        const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+        if (idx >= n_units) break;
+        const BwdUnit u = bwd_unit<D, CAUSAL, VARLEN>(idx, p, ne);
         // Q, dO, lse2, D of step s of this unit into its stage
         auto load_q = [&](int s) -> bool {
           const int g = gs + s;
           const int st = g % C::NSTAGE;
           if (!mbar_wait(BAR(C::B_QEMPTY + st), ((g / C::NSTAGE) & 1) ^ 1, wc, 11)) return false;
-          const int q_row = (u.b * p.Hq + step_head(u, s)) * p.N + step_q0(u, s);
-          const int q_row_p = (u.b * p.Hq + step_head(u, s)) * p.Np + step_q0(u, s);
+          const int q_row = bwd_qrow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);
+          const int q_row_p = bwd_qprow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);
           const uint32_t bar = BAR(C::B_QFULL + st);
           mbar_expect_tx(bar, 2 * C::Q_BYTES + 512);
 #pragma unroll
@@ -353,7 +409,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int s = 0; s < pre && ok; ++s) ok = load_q(s);
         if (!ok) break;
         if (uc > 0 && !mbar_wait(BAR(C::B_KVEMPTY), (uc - 1) & 1, wc, 18)) break;
-        const int kv_row = (u.b * p.Hkv + u.hkv) * p.N + u.jt * C::BC;
+        const int kv_row = bwd_kvrow<VARLEN>(u, p) + u.jt * C::BC;
         mbar_expect_tx(BAR(C::B_KVFULL), 2 * C::KV_BYTES);
 #pragma unroll
         for (int pn = 0; pn < D / 64; ++pn) {
@@ -402,8 +458,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       for (int uc = 0; ok; ++uc) {
         const int idx = next_unit(uc);
         if (idx < 0) { ok = false; break; }
-        if (idx >= p.n_units) break;
-        const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+        if (idx >= n_units) break;
+        const BwdUnit u = bwd_unit<D, CAUSAL, VARLEN>(idx, p, ne);
         const int n = u.n;
         const uint64_t dQ_mn = sdesc_sw128(sbase + C::Q_OFF + (u.dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
         const uint64_t dDO_mn = sdesc_sw128(sbase + C::DO_OFF + (u.dh * C::DH / 64) * C::Q_PANEL, C::Q_PANEL, 1024);
@@ -480,8 +536,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     for (int uc = 0; ok; ++uc) {
       const int idx = next_unit(uc);
       if (idx < 0) { ok = false; break; }
-      if (idx >= p.n_units) break;
-      const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+      if (idx >= n_units) break;
+      const BwdUnit u = bwd_unit<D, CAUSAL, VARLEN>(idx, p, ne);
       const int key = u.jt * C::BC + r;
       for (int s = 0; s < u.n; ++s) {
         const int g = gs + s;
@@ -512,10 +568,10 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
             if (key > q0 + c) pr[c] = 0.f;
         }
         // ragged N: keys and queries past the end of the sequence contribute nothing
-        if (TAIL && (key >= p.N || q0 + C::BR > p.N)) {
+        if (TAIL && (key >= u.len || q0 + C::BR > u.len)) {
 #pragma unroll
           for (int c = 0; c < 64; ++c)
-            if (key >= p.N || q0 + c >= p.N) pr[c] = 0.f;
+            if (key >= u.len || q0 + c >= u.len) pr[c] = 0.f;
         }
         uint32_t pk[32];
 #pragma unroll
@@ -565,7 +621,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // loads, only rows < N are stored
       if (!mbar_wait_warp(BAR(C::B_ACC), uc & 1, wc, 25)) { ok = false; break; }
       tc_fence_after();
-      __nv_bfloat16* dst = p.dk + ((size_t)(u.b * p.Hkv + u.hkv) * p.N + key) * D + u.dh * C::DH;
+      __nv_bfloat16* dst = p.dk + ((size_t)bwd_kvrow<VARLEN>(u, p) + key) * D + u.dh * C::DH;
 #pragma unroll
       for (int oc = 0; oc < C::DH / 32; ++oc) {
         uint32_t v[32];
@@ -583,7 +639,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         for (int c = 0; c < 16; ++c)
           w[c] = pack_bf16(__uint_as_float(v[2 * c]) * p.scale, __uint_as_float(v[2 * c + 1]) * p.scale);
         uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
-        if (!TAIL || key < p.N) {
+        if (!TAIL || key < u.len) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
         }
@@ -606,8 +662,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     for (int uc = 0; ok; ++uc) {
       const int idx = next_unit(uc);
       if (idx < 0) { ok = false; break; }
-      if (idx >= p.n_units) break;
-      const BwdUnit u = bwd_unit<D, CAUSAL>(idx, p);
+      if (idx >= n_units) break;
+      const BwdUnit u = bwd_unit<D, CAUSAL, VARLEN>(idx, p, ne);
       for (int s = 0; s < u.n && ok; ++s) {
         const int g = gs + s;
         if (!mbar_wait_warp(BAR(C::B_DQFULL), g & 1, wc, 31)) { ok = false; break; }
@@ -621,7 +677,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         tc_fence_before();
         __syncwarp();
         if (lane == 0) mbar_arrive(BAR(C::B_DQEMPTY));
-        const int q_row = (u.b * p.Hq + step_head(u, s)) * p.Np + step_q0(u, s);  // padded accumulator row
+        const int q_row = bwd_qprow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);  // padded accumulator row
 #pragma unroll
         for (int sub = 0; sub < 64 / C::STG_ROWS; ++sub) {
           // the previous reduce must have finished reading the staging tile
@@ -651,7 +707,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       // dV epilogue
       if (!mbar_wait_warp(BAR(C::B_ACC), uc & 1, wc, 32)) { ok = false; break; }
       tc_fence_after();
-      __nv_bfloat16* dst = p.dv + ((size_t)(u.b * p.Hkv + u.hkv) * p.N + u.jt * C::BC + r) * D + u.dh * C::DH;
+      __nv_bfloat16* dst = p.dv + ((size_t)bwd_kvrow<VARLEN>(u, p) + u.jt * C::BC + r) * D + u.dh * C::DH;
 #pragma unroll
       for (int oc = 0; oc < C::DH / 32; ++oc) {
         uint32_t v[32];
@@ -668,7 +724,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
 #pragma unroll
         for (int c = 0; c < 16; ++c) w[c] = pack_bf16(__uint_as_float(v[2 * c]), __uint_as_float(v[2 * c + 1]));
         uint4* d4 = reinterpret_cast<uint4*>(dst + oc * 32);
-        if (!TAIL || u.jt * C::BC + r < p.N) {
+        if (!TAIL || u.jt * C::BC + r < u.len) {
 #pragma unroll
           for (int c = 0; c < 4; ++c) d4[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
         }

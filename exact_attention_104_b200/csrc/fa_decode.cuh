@@ -78,10 +78,6 @@ template <int N>
 __device__ __forceinline__ void cp_async_wait() {
   asm volatile("cp.async.wait_group %0;" ::"n"(N) : "memory");
 }
-// two bf16 in one 32-bit word -> two floats (exact)
-__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
-__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
-__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t x) { return f2_make(bf_lo(x), bf_hi(x)); }
 
 // Query row r of row group rg -> (head within the group g, query index i).
 __device__ __forceinline__ void dec_row(const DecodeParams& p, int rg, int r, int RMAX, int& g, int& i) {

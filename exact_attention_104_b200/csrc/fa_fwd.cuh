@@ -28,11 +28,13 @@ namespace fa {
 
 constexpr float kRescaleTau = 8.0f;
 
-template <int D>
+// NQ_: query tiles per CTA (two in the persistent kernel for d = 64, 128;
+// one in fa_fwd_kernel).
+template <int D, int NQ_ = (D <= 128) ? 2 : 1>
 struct FwdCfg {
   static constexpr int BM = 128;                 // query rows per tile (MMA M)
   static constexpr int BN = 128;                 // keys per K/V tile (MMA N of QKᵀ)
-  static constexpr int NQ = (D <= 128) ? 2 : 1;  // query tiles per CTA
+  static constexpr int NQ = NQ_;                 // query tiles per CTA
   static constexpr int THREADS = 128 + 128 * NQ;
   static constexpr int CH = D < 128 ? D : 128;   // K/V chunk width in columns
   static constexpr int NCH = D / CH;             // chunks per K or V tile
@@ -71,7 +73,23 @@ struct FwdParams {
   float scale_log2;
   long long wait_cap;
   int* err;
+  // VARLEN only: packed sequences of T tokens per head, cu_seqlens, and the
+  // work table of (sequence, query tile) units with its header (hdr[0] units)
+  const int2* table;
+  const int* cu;
+  const int* hdr;
+  int T;
+  // DECODE only: Nq query rows per head against Nk keys; the G·Nq rows of a
+  // kv head's query group (R of them) in n_rt tiles of 128; the key axis in
+  // n_split splits of tiles_per_split 128-key tiles; partial results
+  int Nq, Nk, R, n_rt, n_split, tiles_per_split;
+  float* part_o;   // [n_split][B·Hkv·n_rt][128][d]
+  float* part_ml;  // [n_split][B·Hkv·n_rt][128][2]: m (log2 units), l
 };
+
+// fa_fwd_kernel modes: one (batch, head, query tile) per CTA; a packed batch
+// of sequences; decoding (a kv head's query group against one key split).
+enum : int { kFwdDense = 0, kFwdVarlen = 1, kFwdDecode = 2 };
 
 // Load order of the K/V tiles ("units"; each unit is NCH chunks) of the
 // one-tile kernel: it keeps two S tiles in flight, so the MMA warp first uses
@@ -103,13 +121,69 @@ __device__ __forceinline__ float row_max128(const float (&s)[128]) {
 }
 
 // TAIL: N is not a multiple of 128 (keys past N masked, rows past N not stored).
-template <int D, bool CAUSAL, bool TAIL>
-__global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
+// MODE kFwdVarlen: a packed batch of sequences (always with TAIL): a 1-D grid
+// of at least table-entries × Hq CTAs; CTA i takes unit i (causal: heaviest
+// first across heads, else head by head) and CTAs past the last unit exit at
+// once.
+// MODE kFwdDecode: grid (n_split, B·Hkv·n_rt); a CTA multiplies one 128-row
+// tile of a kv head's query group (row r = g·Nq + i: query i of head
+// hkv·G + g, at sequence position Nk − Nq + i) by the 128-key tiles of one
+// key split, with a per-row position mask, and writes the split's
+// unnormalised O with its reference max m and normaliser l for the combine
+// kernel.  The group's rows are contiguous in q ([B, Hq, Nq, d], heads of a
+// group adjacent), so one 128-row box loads them; every row of a K/V tile
+// serves up to 128 query rows (the CUDA-core decode kernel serves 16).
+template <int D, bool CAUSAL, bool TAIL, int MODE = kFwdDense>
+__global__ void __launch_bounds__(FwdCfg<D, 1>::THREADS, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
-  using C = FwdCfg<D>;
+  using C = FwdCfg<D, 1>;
   using Ord = KVOrder;
-  static_assert(C::NQ == 1, "one query tile per CTA (d = 64 and 128 use fa_fwd_persistent_kernel)");
+  constexpr bool VARLEN = MODE == kFwdVarlen;
+  constexpr bool DECODE = MODE == kFwdDecode;
+  static_assert(!VARLEN || TAIL, "packed sequences have ragged ends");
+  int h = 0, qt = 0, len = 0, q_base = 0, kv_base = 0, n = 0;
+  int t0 = 0, rt = 0, rows_valid = C::BM;  // DECODE: first key tile, row tile, real rows of the tile
+  if (DECODE) {
+    const int unit = blockIdx.y;
+    rt = unit % p.n_rt;
+    const int hkv = (unit / p.n_rt) % p.Hkv;
+    const int b = unit / (p.n_rt * p.Hkv);
+    q_base = (b * p.Hq + hkv * p.G) * p.Nq + rt * C::BM;
+    t0 = blockIdx.x * p.tiles_per_split;
+    const int n_tiles = (p.Nk + C::BN - 1) / C::BN;
+    n = min(n_tiles, t0 + p.tiles_per_split) - t0;
+    kv_base = (b * p.Hkv + hkv) * p.Nk + t0 * C::BN;
+    rows_valid = min(C::BM, p.R - rt * C::BM);
+    len = p.Nk;
+  } else if (VARLEN) {
+    const int ne = p.hdr[0];
+    const int idx = blockIdx.x;
+    if (idx >= ne * p.Hq) return;  // no unit for this CTA (nothing shared has been touched)
+    int e;
+    if (CAUSAL) {
+      e = idx / p.Hq;
+      h = idx % p.Hq;
+    } else {
+      h = idx / ne;
+      e = idx % ne;
+    }
+    const int2 ent = p.table[e];
+    qt = ent.y;
+    const int start = p.cu[ent.x];
+    len = p.cu[ent.x + 1] - start;
+    q_base = h * p.T + start;
+    kv_base = (h / p.G) * p.T + start;
+  } else {
+    h = blockIdx.y;
+    const int b = blockIdx.z;
+    // causal: heaviest query tiles first so the tail of the grid is short
+    qt = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
+    len = p.N;
+    q_base = (b * p.Hq + h) * p.N;
+    kv_base = (b * p.Hkv + h / p.G) * p.N;
+  }
+  if (!DECODE) n = CAUSAL ? qt + 1 : (len + C::BN - 1) / C::BN;  // K/V tiles this query tile sees
   extern __shared__ uint8_t smem_raw[];
   uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
   const uint32_t sbase = smem_u32(smem);
@@ -119,12 +193,6 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
-  const int h = blockIdx.y;
-  const int b = blockIdx.z;
-  const int hkv = h / p.G;
-  // causal: heaviest query tiles first so the tail of the grid is short
-  const int qt = CAUSAL ? (int)(gridDim.x - 1 - blockIdx.x) : (int)blockIdx.x;
-  const int n = CAUSAL ? qt + 1 : p.n_qtiles;  // K/V tiles this query tile sees
 
   if (threadIdx.x == 0) {
     mbar_init(BAR(C::B_QFULL), 1);
@@ -160,8 +228,8 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&tmV);
       const uint64_t pol_kv = policy_evict_last();
       const uint64_t pol_q = policy_evict_first();
-      const int q_row_base = (b * p.Hq + h) * p.N;
-      const int kv_row_base = (b * p.Hkv + hkv) * p.N;
+      const int q_row_base = q_base;
+      const int kv_row_base = kv_base;
       mbar_expect_tx(BAR(C::B_QFULL), C::Q_BYTES);
 #pragma unroll
       for (int pn = 0; pn < D / 64; ++pn)
@@ -299,8 +367,11 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
       const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
       const float sl2 = p.scale_log2;
       const int ocol = C::O_COL;
+      // DECODE: last key this row may see (absolute key index)
+      const int row_last = DECODE ? (CAUSAL ? p.Nk - p.Nq + (rt * C::BM + row) % p.Nq : p.Nk - 1) : 0;
       float m_ref = -INFINITY;
-      float l = 0.f;
+      float l = 0.f;    // Σ P in fp32: the normaliser of the LSE
+      float l_o = 0.f;  // Σ of the bf16-rounded P that the PV product used: the normaliser of O
       bool ok = true;
       // Completion of PV(j) is signalled on o_done[j & 1]: S(j+1) is issued
       // before PV(j), so a single barrier could run two phases ahead of a
@@ -331,15 +402,23 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           s[64 + c] = __uint_as_float(r2[c]);
           s[96 + c] = __uint_as_float(r3[c]);
         }
-        if (CAUSAL && j == qt) {
+        if (DECODE) {
+          const int key0 = (t0 + j) * C::BN;
+          if (key0 + C::BN - 1 > row_last) {
+#pragma unroll
+            for (int c = 0; c < 128; ++c)
+              if (key0 + c > row_last) s[c] = -INFINITY;
+          }
+        }
+        if (!DECODE && CAUSAL && j == qt) {
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c > row) s[c] = -INFINITY;
         }
         // ragged N: keys past the end of the sequence (the causal mask already
         // excludes them for every row < N)
-        if (TAIL && !CAUSAL && (j + 1) * C::BN > p.N) {
-          const int lim = p.N - j * C::BN;
+        if (!DECODE && TAIL && !CAUSAL && (j + 1) * C::BN > len) {
+          const int lim = len - j * C::BN;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= lim) s[c] = -INFINITY;
@@ -359,15 +438,22 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             alpha = ex2(m_ref - m_new);
             m_ref = m_new;
             l *= alpha;
+            l_o *= alpha;
           }
         }
         // P = 2^(s·scale·log2e − m_ref), rounded to bf16 and written over the
         // first 64 columns of S.  Keys 0..63 are handed to the MMA warp before
         // keys 64..127 are exponentiated, so the first half of the PV product
         // overlaps the second half of the exponentials.  Scale/shift and row
-        // sums use packed fp32x2 instructions.
-        const float neg_m = -m_ref;
+        // sums use packed fp32x2 instructions.  O is divided by the sum of the
+        // rounded P, so that the weights it applies to V sum to one exactly:
+        // with the very peaked rows of large logits the rounding of the
+        // dominant P otherwise scales the whole row of O by up to 2^-9.
+        // (a decoding row can see no key of this split at all: its reference
+        // stays -inf and every P is 0)
+        const float neg_m = (DECODE && m_ref == -INFINITY) ? 0.f : -m_ref;
         uint64_t rs2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
+        uint64_t ro2[2] = {f2_make(0.f, 0.f), f2_make(0.f, 0.f)};
         auto exp_half = [&](int base, uint32_t (&pk)[32]) {
 #pragma unroll
           for (int c = 0; c < 32; ++c) {
@@ -378,6 +464,7 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
             const float a1 = ex2(x1);
             rs2[c & 1] = f2_add(rs2[c & 1], f2_make(a0, a1));
             pk[c] = pack_bf16(a0, a1);
+            ro2[c & 1] = f2_add(ro2[c & 1], bf2_to_f2(pk[c]));
           }
         };
         {
@@ -418,12 +505,37 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
         f2_split(rs2[0], a, b2);
         f2_split(rs2[1], c2, d2);
         l += (a + b2) + (c2 + d2);
+        f2_split(ro2[0], a, b2);
+        f2_split(ro2[1], c2, d2);
+        l_o += (a + b2) + (c2 + d2);
       }
       if (ok) ok = mbar_wait_warp(BAR(C::B_ODONE + odone_idx(n - 1)), odone_par(n - 1), wc, 7);
-      if (ok) {
+      if (ok && DECODE) {
+        // this split's partial result: O scaled so that O / l is the average
+        // under the rounded weights the PV product used, m and l in log2 units
         tc_fence_after();
-        const float inv_l = 1.f / l;
-        __nv_bfloat16* orow = p.o + ((size_t)(b * p.Hq + h) * p.N + q_row) * D;
+        const size_t slot = ((size_t)blockIdx.x * gridDim.y + blockIdx.y) * C::BM + row;
+        const float f = l_o > 0.f ? l / l_o : 0.f;
+        float* po = p.part_o + slot * D;
+#pragma unroll
+        for (int oc = 0; oc < D / 32; ++oc) {
+          uint32_t ov[32];
+          tmem_ld32(tl + ocol + oc * 32, ov);
+          tmem_ld_wait();
+          reg_fence(ov);
+          if (row < rows_valid) {
+            float4* dst = reinterpret_cast<float4*>(po + oc * 32);
+#pragma unroll
+            for (int c = 0; c < 8; ++c)
+              dst[c] = make_float4(__uint_as_float(ov[4 * c]) * f, __uint_as_float(ov[4 * c + 1]) * f,
+                                   __uint_as_float(ov[4 * c + 2]) * f, __uint_as_float(ov[4 * c + 3]) * f);
+          }
+        }
+        if (row < rows_valid) *reinterpret_cast<float2*>(p.part_ml + slot * 2) = make_float2(m_ref, l);
+      } else if (ok) {
+        tc_fence_after();
+        const float inv_l = 1.f / l_o;
+        __nv_bfloat16* orow = p.o + ((size_t)q_base + q_row) * D;
 #pragma unroll
         for (int oc = 0; oc < D / 32; ++oc) {
           uint32_t ov[32];
@@ -435,14 +547,14 @@ __global__ void __launch_bounds__(FwdCfg<D>::THREADS, 1)
           for (int c = 0; c < 16; ++c)
             w[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
           uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
-          if (!TAIL || q_row < p.N) {  // rows past a ragged end are computed, not stored
+          if (!TAIL || q_row < len) {  // rows past a ragged end are computed, not stored
 #pragma unroll
             for (int c = 0; c < 4; ++c) dst[c] = make_uint4(w[4 * c], w[4 * c + 1], w[4 * c + 2], w[4 * c + 3]);
           }
         }
         float lg;
         asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-        if (!TAIL || q_row < p.N) p.lse[(size_t)(b * p.Hq + h) * p.N + q_row] = (m_ref + lg) * kLn2;
+        if (!TAIL || q_row < len) p.lse[(size_t)q_base + q_row] = (m_ref + lg) * kLn2;
       }
       tc_fence_before();
     }

@@ -78,39 +78,75 @@ struct FwdPParams {
   int N, Hq, G, n_qtiles;
   int n_units;  // query-tile pairs per (batch, head)
   int BH;       // batch · query heads
-  int n_items;  // n_units · BH
+  int n_items;  // n_units · BH (VARLEN: from the work table, see below)
   float scale_log2;
   long long wait_cap;
   int* err;
+  // VARLEN only: packed sequences of T tokens per head, cu_seqlens, and the
+  // work table of (sequence, tile pair) units with its header (hdr[0] units)
+  const int2* table;
+  const int* cu;
+  const int* hdr;
+  int T;
 };
 
 // One work item: query tiles qt0 (tile 0) and qt0 + 1 (tile 1, absent when
-// qt0 is the last tile).  Iteration jj of the item multiplies by K/V block
-// kv_block(jj); tile 0 takes part from iteration skew on, tile 1 in all.
+// qt0 is the last tile) of one (batch or sequence, head).  Iteration jj of
+// the item multiplies by K/V block kv_block(jj); tile 0 takes part from
+// iteration skew on, tile 1 in all.  qbase / kvbase are the rows of the
+// sequence's first token in the Q (and O, LSE) and K/V tensors, len its
+// length.
 struct FwdItem {
-  int b, h, qt0, n0, n1, skew, nit;
+  int h, qt0, n0, n1, skew, nit;
+  int qbase, kvbase, len;
   __device__ int kv_block(int jj) const { return (skew && jj == 0) ? qt0 + 1 : jj - skew; }
   __device__ int first(int t) const { return t == 0 ? skew : 0; }
   __device__ bool has(int t) const { return t == 0 || n1 > 0; }
 };
 
-template <bool CAUSAL>
-__device__ __forceinline__ FwdItem fwd_item(int idx, const FwdPParams& p) {
-  int unit, bh;
-  if (CAUSAL) {
-    unit = p.n_units - 1 - idx / p.BH;  // heaviest (latest) query tiles first
-    bh = idx % p.BH;
-  } else {
-    bh = idx / p.n_units;
-    unit = idx % p.n_units;
-  }
+// ne: VARLEN work-table entries (hdr[0]).  Causal items go heaviest first
+// across all heads; non-causal items head by head, so that CTAs running at
+// the same time share a head's K/V tiles in L2.
+template <bool CAUSAL, bool VARLEN>
+__device__ __forceinline__ FwdItem fwd_item(int idx, const FwdPParams& p, int ne) {
   FwdItem w;
-  w.b = bh / p.Hq;
-  w.h = bh % p.Hq;
+  int unit, n_qtiles;
+  if (VARLEN) {
+    int e;
+    if (CAUSAL) {
+      e = idx / p.Hq;
+      w.h = idx % p.Hq;
+    } else {
+      w.h = idx / ne;
+      e = idx % ne;
+    }
+    const int2 ent = p.table[e];
+    unit = ent.y;
+    const int start = p.cu[ent.x];
+    w.len = p.cu[ent.x + 1] - start;
+    w.qbase = w.h * p.T + start;
+    w.kvbase = (w.h / p.G) * p.T + start;
+    n_qtiles = (w.len + 127) / 128;
+  } else {
+    int bh;
+    if (CAUSAL) {
+      unit = p.n_units - 1 - idx / p.BH;  // heaviest (latest) query tiles first
+      bh = idx % p.BH;
+    } else {
+      bh = idx / p.n_units;
+      unit = idx % p.n_units;
+    }
+    const int b = bh / p.Hq;
+    w.h = bh % p.Hq;
+    w.len = p.N;
+    w.qbase = bh * p.N;
+    w.kvbase = (b * (p.Hq / p.G) + w.h / p.G) * p.N;
+    n_qtiles = p.n_qtiles;
+  }
   w.qt0 = 2 * unit;
-  const bool has1 = w.qt0 + 1 < p.n_qtiles;
-  w.n0 = CAUSAL ? w.qt0 + 1 : p.n_qtiles;
-  w.n1 = has1 ? (CAUSAL ? w.qt0 + 2 : p.n_qtiles) : 0;
+  const bool has1 = w.qt0 + 1 < n_qtiles;
+  w.n0 = CAUSAL ? w.qt0 + 1 : n_qtiles;
+  w.n1 = has1 ? (CAUSAL ? w.qt0 + 2 : n_qtiles) : 0;
   w.skew = (CAUSAL && has1) ? 1 : 0;
   w.nit = w.n0 + w.skew;
   return w;
@@ -125,7 +161,9 @@ __device__ __forceinline__ int fwd_item_index(int k, int c, int G) {
 }
 
 // TAIL: N is not a multiple of 128 (keys past N masked, rows past N not stored).
-template <int D, bool CAUSAL, bool TAIL>
+// VARLEN: a packed batch of sequences (always with TAIL); items come from the
+// work table, each with its own length and row bases.
+template <int D, bool CAUSAL, bool TAIL, bool VARLEN = false>
 __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
     fa_fwd_persistent_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                              const __grid_constant__ CUtensorMap tmV, const FwdPParams p) {
@@ -139,9 +177,12 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
 
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
+  static_assert(!VARLEN || TAIL, "packed sequences have ragged ends");
   const int G = gridDim.x;
   const int cta = blockIdx.x;
-  const int n_rounds = (p.n_items + G - 1) / G;
+  const int ne = VARLEN ? p.hdr[0] : 0;
+  const int n_items = VARLEN ? ne * p.Hq : p.n_items;
+  const int n_rounds = (n_items + G - 1) / G;
 
   if (threadIdx.x == 0) {
     for (int t = 0; t < 2; ++t) {
@@ -184,11 +225,10 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       bool ok = true;
       for (int k = 0; k < n_rounds && ok; ++k) {
         const int idx = fwd_item_index<CAUSAL>(k, cta, G);
-        if (idx >= p.n_items) continue;
-        const FwdItem w = fwd_item<CAUSAL>(idx, p);
-        const int hkv = w.h / p.G;
-        const int q_row_base = (w.b * p.Hq + w.h) * p.N;
-        const int kv_row_base = (w.b * (p.Hq / p.G) + hkv) * p.N;
+        if (idx >= n_items) continue;
+        const FwdItem w = fwd_item<CAUSAL, VARLEN>(idx, p, ne);
+        const int q_row_base = w.qbase;
+        const int kv_row_base = w.kvbase;
         for (int t = 0; t < 2 && ok; ++t) {
           if (!w.has(t)) continue;
           // the previous item's last QKᵀ of this tile must be done reading the buffer
@@ -284,18 +324,18 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
     };
 
     int k = 0;
-    while (k < n_rounds && fwd_item_index<CAUSAL>(k, cta, G) >= p.n_items) ++k;
+    while (k < n_rounds && fwd_item_index<CAUSAL>(k, cta, G) >= n_items) ++k;
     if (k < n_rounds) {
-      FwdItem w = fwd_item<CAUSAL>(fwd_item_index<CAUSAL>(k, cta, G), p);
+      FwdItem w = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k, cta, G), p, ne);
       int base = 0;
       for (int t = 0; t < 2 && ok; ++t)
         if (w.has(t)) ok = issue_s(t, w, base, w.first(t));
       while (ok) {
         int k2 = k + 1;
-        while (k2 < n_rounds && fwd_item_index<CAUSAL>(k2, cta, G) >= p.n_items) ++k2;
+        while (k2 < n_rounds && fwd_item_index<CAUSAL>(k2, cta, G) >= n_items) ++k2;
         const bool has_next = k2 < n_rounds;
         FwdItem w2 = w;
-        if (has_next) w2 = fwd_item<CAUSAL>(fwd_item_index<CAUSAL>(k2, cta, G), p);
+        if (has_next) w2 = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k2, cta, G), p, ne);
         const int base2 = base + 2 * w.nit;
         for (int jj = 0; jj < w.nit && ok; ++jj) {
           for (int t = 0; t < 2; ++t) {
@@ -348,8 +388,8 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
     bool ok = true;
     for (int k = 0; k < n_rounds && ok; ++k) {
       const int idx = fwd_item_index<CAUSAL>(k, cta, G);
-      if (idx >= p.n_items) continue;
-      const FwdItem w = fwd_item<CAUSAL>(idx, p);
+      if (idx >= n_items) continue;
+      const FwdItem w = fwd_item<CAUSAL, VARLEN>(idx, p, ne);
       if (!w.has(t)) continue;
       const int n = t == 0 ? w.n0 : w.n1;
       const int qt = w.qt0 + t;
@@ -385,8 +425,8 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         }
         // ragged N: keys past the end of the sequence (the causal mask already
         // excludes them for every row < N)
-        if (TAIL && !CAUSAL && (kb + 1) * C::BN > p.N) {
-          const int lim = p.N - kb * C::BN;
+        if (TAIL && !CAUSAL && (kb + 1) * C::BN > w.len) {
+          const int lim = w.len - kb * C::BN;
 #pragma unroll
           for (int c = 0; c < 128; ++c)
             if (c >= lim) s[c] = -INFINITY;
@@ -470,7 +510,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       tc_fence_after();
       const int q_row = qt * C::BM + row;
       const float inv_l = 1.f / l;
-      __nv_bfloat16* orow = p.o + ((size_t)(w.b * p.Hq + w.h) * p.N + q_row) * D;
+      __nv_bfloat16* orow = p.o + ((size_t)w.qbase + q_row) * D;
 #pragma unroll
       for (int oc = 0; oc < D / 32; ++oc) {
         uint32_t ov[32];
@@ -482,14 +522,14 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         for (int c = 0; c < 16; ++c)
           wv[c] = pack_bf16(__uint_as_float(ov[2 * c]) * inv_l, __uint_as_float(ov[2 * c + 1]) * inv_l);
         uint4* dst = reinterpret_cast<uint4*>(orow + oc * 32);
-        if (!TAIL || q_row < p.N) {  // rows past a ragged end are computed, not stored
+        if (!TAIL || q_row < w.len) {  // rows past a ragged end are computed, not stored
 #pragma unroll
           for (int c = 0; c < 4; ++c) dst[c] = make_uint4(wv[4 * c], wv[4 * c + 1], wv[4 * c + 2], wv[4 * c + 3]);
         }
       }
       float lg;
       asm("lg2.approx.ftz.f32 %0, %1;" : "=f"(lg) : "f"(l));
-      if (!TAIL || q_row < p.N) p.lse[(size_t)(w.b * p.Hq + w.h) * p.N + q_row] = (m_ref + lg) * kLn2;
+      if (!TAIL || q_row < w.len) p.lse[(size_t)w.qbase + q_row] = (m_ref + lg) * kLn2;
       done += n;
     }
     tc_fence_before();

@@ -20,7 +20,9 @@ constexpr float kLog2e = 1.4426950408889634f;
 constexpr float kLn2 = 0.6931471805599453f;
 
 // Device error word values (the failing site goes in bits 8..15).
-enum : int { kDevOk = 0, kDevTimeout = 4, kDevCheck = 5 };
+// kDevBadSeqlens: a varlen call's cu_seqlens broke its rules (the call
+// computed nothing).
+enum : int { kDevOk = 0, kDevTimeout = 4, kDevCheck = 5, kDevBadSeqlens = 6 };
 
 __device__ __forceinline__ uint32_t smem_u32(const void* p) {
   return static_cast<uint32_t>(__cvta_generic_to_shared(p));
@@ -399,6 +401,11 @@ __device__ __forceinline__ uint32_t pack_bf16(float lo, float hi) {
   asm("cvt.rn.bf16x2.f32 %0, %1, %2;" : "=r"(r) : "f"(hi), "f"(lo));
   return r;
 }
+
+// two bf16 in one 32-bit word -> two floats (exact)
+__device__ __forceinline__ float bf_lo(uint32_t x) { return __uint_as_float(x << 16); }
+__device__ __forceinline__ float bf_hi(uint32_t x) { return __uint_as_float(x & 0xffff0000u); }
+__device__ __forceinline__ uint64_t bf2_to_f2(uint32_t x) { return f2_make(bf_lo(x), bf_hi(x)); }
 
 // Per-warpgroup register reallocation (the whole warpgroup executes it).
 template <int N>

@@ -120,6 +120,10 @@ DECODE_WORKLOADS = {
     # one decoding step of a batch of 8 sequences with a 32k-token cache, GQA 4:1
     "decode_b8_hq32_hkv8_nk32768_d128": DecodeWorkload("decode_b8_hq32_hkv8_nk32768_d128", 8, 32, 8, 1, 32768, 128,
                                                       True, 1007),
+    # 32 queries per head (a speculative or chunked decoding step): 128 query
+    # rows per kv head share every K/V tile
+    "decode_b8_hq32_hkv8_nq32_nk32768_d128": DecodeWorkload("decode_b8_hq32_hkv8_nq32_nk32768_d128", 8, 32, 8, 32,
+                                                           32768, 128, True, 1008),
 }
 
 
@@ -159,3 +163,75 @@ def shard_units(B: int, Hkv: int, rank: int, world: int):
     start = rank * base + min(rank, extra)
     count = base + (1 if rank < extra else 0)
     return [(u // Hkv, u % Hkv) for u in range(start, start + count)]
+
+
+@dataclass(frozen=True)
+class VarlenWorkload:
+    """A packed batch of sequences with the given lengths (sequences back to
+    back along the token axis of [H, T, d] tensors)."""
+    name: str
+    lengths: tuple
+    Hq: int
+    Hkv: int
+    d: int
+    causal: bool
+    seed: int
+    qk_std: float = 1.0
+
+    @property
+    def scale(self) -> float:
+        return 1.0 / math.sqrt(self.d)
+
+    @property
+    def G(self) -> int:
+        return self.Hq // self.Hkv
+
+    @property
+    def T(self) -> int:
+        return int(sum(self.lengths))
+
+    @property
+    def max_seqlen(self) -> int:
+        return max(1, max(self.lengths))
+
+    def cu_seqlens(self):
+        out = [0]
+        for n in self.lengths:
+            out.append(out[-1] + int(n))
+        return out
+
+    def fwd_flops(self) -> float:
+        """4·d FLOPs per visible (query, key) pair and query head (the fixed-
+        length count, summed over the sequences)."""
+        pairs = sum((n * (n + 1)) // 2 if self.causal else n * n for n in self.lengths)
+        return 4.0 * self.Hq * self.d * pairs
+
+    def describe(self) -> str:
+        return (f"{len(self.lengths)} sequences, T={self.T}, max len {self.max_seqlen}, Hq={self.Hq} "
+                f"Hkv={self.Hkv} d={self.d} {'causal' if self.causal else 'non-causal'}")
+
+
+def varlen_lengths(nseq: int, lo: int, hi: int, seed: int, include=()):
+    """nseq sequence lengths drawn uniformly from [lo, hi] (seeded), with the
+    values in ``include`` placed first."""
+    g = torch.Generator("cpu").manual_seed(seed)
+    extra = torch.randint(lo, hi + 1, (max(0, nseq - len(include)),), generator=g).tolist()
+    return tuple(list(include) + extra)
+
+
+def make_varlen_inputs(w: VarlenWorkload, device="cpu"):
+    """Draw (q, k, v, do, cu_seqlens): q, do bf16 [Hq, T, d], k, v bf16
+    [Hkv, T, d] (standard normals in the order q, k, v, do; q and k times
+    qk_std) and cu_seqlens int32 [nseq + 1]."""
+    g = torch.Generator("cpu").manual_seed(w.seed)
+    T = w.T
+    q = torch.randn(w.Hq, T, w.d, generator=g, dtype=torch.float32)
+    k = torch.randn(w.Hkv, T, w.d, generator=g, dtype=torch.float32)
+    v = torch.randn(w.Hkv, T, w.d, generator=g, dtype=torch.float32)
+    do = torch.randn(w.Hq, T, w.d, generator=g, dtype=torch.float32)
+    if w.qk_std != 1.0:
+        q.mul_(w.qk_std)
+        k.mul_(w.qk_std)
+    out = [t.to(torch.bfloat16).to(device) for t in (q, k, v, do)]
+    cu = torch.tensor(w.cu_seqlens(), dtype=torch.int32, device=device)
+    return (*out, cu)

@@ -162,6 +162,57 @@ fa_status fa_fwd_decode(const void* q, const void* k, const void* v, void* o, fl
                         int B, int Hq, int Hkv, int Nq, int Nk, int d, int causal, float scale,
                         void* workspace, size_t workspace_bytes, void* stream);
 
+/* ------------------------------------------------------------------------
+ * Packed batches of sequences with different lengths ("varlen").
+ *
+ * `nseq` independent sequences are stored back to back along the token axis
+ * of every head: sequence b owns tokens cu_seqlens[b] .. cu_seqlens[b+1] - 1,
+ * and T = cu_seqlens[nseq] tokens in all.  Each sequence attends only to its
+ * own keys (with `causal` != 0, key j of the sequence is masked for query i
+ * of the sequence when j > i, positions counted from the sequence's first
+ * token), so the result for every sequence is exactly that of one fa_fwd /
+ * fa_bwd call on its own tokens.  Ragged batches are the case the
+ * "Flash-Attention" concept page names under "Design space and trade-offs"
+ * (they change which tiles are legal and how work balances) and "Known
+ * limits" (continuous batching).
+ *
+ * Layouts (head-major: [B, H, N, d] with B = 1, N = T and the sequences
+ * concatenated along N):
+ *   q, o, dout, dq : bf16 [Hq,  T, d]
+ *   k, v, dk, dv   : bf16 [Hkv, T, d]
+ *   lse            : fp32 [Hq,  T]
+ *   cu_seqlens     : int32 [nseq + 1] in DEVICE memory: cu_seqlens[0] = 0,
+ *                    non-decreasing, cu_seqlens[nseq] = T (empty sequences
+ *                    are allowed)
+ * `max_seqlen` (host) must bound every sequence length, 1 <= max_seqlen <=
+ * 2^20.  Because cu_seqlens lives on the device it is checked by the
+ * library's first kernel: if it breaks any rule above, no attention kernel
+ * computes anything, the outputs are left untouched and fa_device_status()
+ * reports FA_ERR_INVALID_ARG.
+ *
+ * Scheduling: the first kernel of each call turns cu_seqlens into a table of
+ * (sequence, tile) work units in the workspace, heaviest first, which the
+ * attention kernels deal out.  Units of equal weight may come in any order,
+ * so the backward's dQ, like fa_bwd's, is not bitwise reproducible.
+ *
+ * Workspace: device, 256-byte aligned, at least the size the matching
+ * *_workspace_bytes function returns (0 for invalid sizes); it is in use
+ * until the call's kernels have finished.  Other errors as for fa_fwd and
+ * fa_bwd; T == 0 (or nseq == 0) is an empty problem.
+ * fa_fwd_varlen enqueues two kernels, fa_bwd_varlen four. */
+size_t fa_fwd_varlen_workspace_bytes(int nseq, int Hq, int Hkv, int T, int max_seqlen, int d);
+fa_status fa_fwd_varlen(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens, int nseq, int Hq, int Hkv, int T, int max_seqlen,
+                        int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
+size_t fa_bwd_varlen_workspace_bytes(int nseq, int Hq, int Hkv, int T, int max_seqlen, int d);
+fa_status fa_bwd_varlen(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dout, void* dq, void* dk, void* dv,
+                        const int* cu_seqlens, int nseq, int Hq, int Hkv, int T, int max_seqlen,
+                        int d, int causal, float scale, void* workspace, size_t workspace_bytes,
+                        void* stream);
+
 /* Size in bytes of the fixed device scratch array used by fa_bwd_noalloc. */
 #define FA_NOALLOC_SCRATCH_BYTES (64u * 1024u * 1024u)
 

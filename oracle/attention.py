@@ -60,6 +60,8 @@ __all__ = [
     "head_backward_rows",
     "head_backward_sampled",
     "attention_forward_suffix",
+    "attention_forward_varlen",
+    "attention_backward_varlen",
     "attention_flops",
 ]
 
@@ -363,6 +365,69 @@ def attention_forward_suffix(q, k, v, scale, causal=False):
             o[b, h] = (e / l) @ v[b, g]
             lse[b, h] = (m + np.log(l))[:, 0]
     return o, lse
+
+
+# ---------------------------------------------------------------------------
+# Packed batches of sequences with different lengths
+# ---------------------------------------------------------------------------
+
+def _varlen_bounds(cu_seqlens, T):
+    cu = [int(c) for c in cu_seqlens]
+    assert cu[0] == 0 and cu[-1] == T and all(a <= b for a, b in zip(cu, cu[1:])), cu
+    return cu
+
+
+def attention_forward_varlen(q, k, v, cu_seqlens, scale, causal=False):
+    """Attention over a packed batch of independent sequences of different
+    lengths ("Flash-Attention" concept page, "Design space and trade-offs":
+    ragged batches change which tiles are legal and how work balances).
+
+    Sequence b holds tokens cu_seqlens[b] .. cu_seqlens[b+1]-1 of the packed
+    token axis; its queries see only its own keys (causal: key j of the
+    sequence is masked for query i of the sequence when j > i, positions
+    counted from the sequence's first token).  So every sequence is exactly one
+    call of :func:`attention_forward` on its own tokens.
+
+    q: [Hq, T, d]; k, v: [Hkv, T, d] (heads first, sequences back to back along
+    the token axis); cu_seqlens: nseq + 1 non-decreasing offsets from 0 to T.
+    Returns O [Hq, T, d] and LSE [Hq, T] (natural log), float64."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    Hq, T, d = q.shape
+    cu = _varlen_bounds(cu_seqlens, T)
+    o = np.zeros_like(q)
+    lse = np.zeros((Hq, T))
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        if hi == lo:
+            continue
+        ob, lb = attention_forward(q[None, :, lo:hi], k[None, :, lo:hi], v[None, :, lo:hi], scale, causal)
+        o[:, lo:hi], lse[:, lo:hi] = ob[0], lb[0]
+    return o, lse
+
+
+def attention_backward_varlen(q, k, v, do, cu_seqlens, scale, causal=False):
+    """Gradients of :func:`attention_forward_varlen`: each sequence is one
+    call of :func:`attention_backward` on its own tokens (the sequences share
+    no keys, so nothing couples their gradients).  Layouts as in the forward;
+    do: [Hq, T, d].  Returns (dq, dk, dv, o, lse) in float64."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    do = np.asarray(do, np.float64)
+    Hq, T, d = q.shape
+    cu = _varlen_bounds(cu_seqlens, T)
+    dq, dk, dv, o = np.zeros_like(q), np.zeros_like(k), np.zeros_like(v), np.zeros_like(q)
+    lse = np.zeros((Hq, T))
+    for b in range(len(cu) - 1):
+        lo, hi = cu[b], cu[b + 1]
+        if hi == lo:
+            continue
+        r = attention_backward(q[None, :, lo:hi], k[None, :, lo:hi], v[None, :, lo:hi], do[None, :, lo:hi],
+                               scale, causal)
+        dq[:, lo:hi], dk[:, lo:hi], dv[:, lo:hi], o[:, lo:hi], lse[:, lo:hi] = (x[0] for x in r)
+    return dq, dk, dv, o, lse
 
 
 def attention_flops(B, Hq, N, d, causal):

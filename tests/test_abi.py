@@ -148,6 +148,11 @@ def test_decode_workspace_bytes(lib):
     assert ws(1, 2, 2, 1, 100, 96) == 0       # unsupported d
     assert ws(1, 2, 2, 1, 0, 64) == 0         # queries with no key
     assert ws(0, 2, 2, 1, 100, 64) == 0       # empty problem needs nothing
+    # more than 16 query rows per kv head: 128-row tiles, 128-key tiles, about
+    # one CTA per SM in all (64 units of B8 x Hkv8 -> 2 splits of 128 tiles)
+    assert ws(8, 32, 8, 32, 32768, 128) == 2 * 64 * 128 * 128 * 4 + 2 * 64 * 128 * 2 * 4
+    # 512 rows -> 4 row tiles; Nk = 300 -> 3 key tiles, one split each at most
+    assert ws(1, 4, 2, 256, 300, 128) == 3 * 8 * 128 * 128 * 4 + 3 * 8 * 128 * 2 * 4
 
 
 def _dec(lib, **kw):
@@ -206,3 +211,77 @@ def _bwd_noalloc(lib, **kw):
 ])
 def test_noalloc_argument_validation(lib, kw, expect):
     assert _bwd_noalloc(lib, **kw) == expect
+
+
+def test_varlen_workspace_bytes(lib):
+    # header + work table (one int2 per 128-row tile, T/128 + nseq bound); the
+    # backward adds D and lse2 rows, the fp32 dQ accumulator over padded rows
+    # Tp = ceil64(T + 256·nseq) per head, and the unit counter
+    r256 = lambda x: (x + 255) // 256 * 256  # noqa: E731
+    nseq, Hq, Hkv, T, d = 3, 4, 2, 1000, 128
+    table = r256(8 * ((T + 127) // 128 + nseq))
+    assert binding.fa_fwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, 600, d) == 256 + table
+    Tp = (T + 256 * nseq + 63) // 64 * 64
+    rows_p = Hq * Tp
+    assert binding.fa_bwd_varlen_workspace_bytes(nseq, Hq, Hkv, T, 600, d) == \
+        256 + table + 2 * r256(rows_p * 4) + r256(rows_p * d * 4) + 256
+    assert binding.fa_fwd_varlen_workspace_bytes(3, 3, 2, 1000, 600, 128) == 0      # Hq % Hkv
+    assert binding.fa_fwd_varlen_workspace_bytes(3, 4, 2, 1000, 600, 96) == 0       # unsupported d
+    assert binding.fa_bwd_varlen_workspace_bytes(3, 4, 2, 1000, 0, 128) == 0        # max_seqlen < 1
+    assert binding.fa_bwd_varlen_workspace_bytes(3, 4, 2, 1000, (1 << 20) + 1, 128) == 0
+    assert binding.fa_fwd_varlen_workspace_bytes(0, 4, 2, 0, 1, 128) == 256         # empty problem
+
+
+def _fwd_varlen(lib, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5, cu=FAKE * 6, nseq=3, Hq=4, Hkv=2, T=1000,
+             max_seqlen=600, d=128, causal=1, scale=0.088, ws=FAKE * 7, wsb=1 << 20)
+    a.update(kw)
+    return binding.fa_fwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["cu"], a["nseq"], a["Hq"], a["Hkv"],
+                                 a["T"], a["max_seqlen"], a["d"], a["causal"], a["scale"], a["ws"], a["wsb"], 0)
+
+
+def _bwd_varlen(lib, **kw):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5, do=FAKE * 6, dq=FAKE * 7, dk=FAKE * 8,
+             dv=FAKE * 9, cu=FAKE * 10, nseq=3, Hq=4, Hkv=2, T=1000, max_seqlen=600, d=128, causal=0, scale=0.088,
+             ws=FAKE * 11, wsb=1 << 24)
+    a.update(kw)
+    return binding.fa_bwd_varlen(a["q"], a["k"], a["v"], a["o"], a["lse"], a["do"], a["dq"], a["dk"], a["dv"],
+                                 a["cu"], a["nseq"], a["Hq"], a["Hkv"], a["T"], a["max_seqlen"], a["d"],
+                                 a["causal"], a["scale"], a["ws"], a["wsb"], 0)
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(q=0), binding.FA_ERR_INVALID_ARG),
+    (dict(cu=0), binding.FA_ERR_INVALID_ARG),
+    (dict(cu=FAKE * 6 + 2), binding.FA_ERR_INVALID_ARG),         # cu_seqlens not 4-byte aligned
+    (dict(o=FAKE * 4 + 8), binding.FA_ERR_INVALID_ARG),          # misaligned
+    (dict(ws=FAKE * 7 + 16), binding.FA_ERR_INVALID_ARG),        # workspace not 256-aligned
+    (dict(wsb=100), binding.FA_ERR_INVALID_ARG),                 # workspace too small
+    (dict(o=FAKE), binding.FA_ERR_INVALID_ARG),                  # output aliases q
+    (dict(ws=FAKE * 6), binding.FA_ERR_INVALID_ARG),             # workspace aliases cu_seqlens
+    (dict(Hq=3), binding.FA_ERR_INVALID_ARG),                    # Hq % Hkv
+    (dict(nseq=-1), binding.FA_ERR_INVALID_ARG),
+    (dict(max_seqlen=0), binding.FA_ERR_INVALID_ARG),
+    (dict(max_seqlen=(1 << 20) + 1), binding.FA_ERR_UNSUPPORTED),
+    (dict(d=96), binding.FA_ERR_UNSUPPORTED),
+    (dict(scale=float("nan")), binding.FA_ERR_INVALID_ARG),
+    (dict(T=0), binding.FA_OK),                                  # empty problem: nothing to do
+    (dict(nseq=0, T=0), binding.FA_OK),
+])
+def test_fwd_varlen_argument_validation(lib, kw, expect):
+    assert _fwd_varlen(lib, **kw) == expect
+
+
+@pytest.mark.parametrize("kw,expect", [
+    (dict(do=0), binding.FA_ERR_INVALID_ARG),
+    (dict(cu=0), binding.FA_ERR_INVALID_ARG),
+    (dict(wsb=1000), binding.FA_ERR_INVALID_ARG),                # workspace too small
+    (dict(dk=FAKE * 7), binding.FA_ERR_INVALID_ARG),             # dk aliases dq
+    (dict(dq=FAKE * 10), binding.FA_ERR_INVALID_ARG),            # dq overlaps cu_seqlens
+    (dict(Hq=1), binding.FA_ERR_INVALID_ARG),                    # Hq % Hkv
+    (dict(d=32), binding.FA_ERR_UNSUPPORTED),
+    (dict(Hq=4096, Hkv=2, T=1 << 19, nseq=1), binding.FA_ERR_UNSUPPORTED),  # padded rows reach 2^31
+    (dict(T=0, nseq=0), binding.FA_OK),
+])
+def test_bwd_varlen_argument_validation(lib, kw, expect):
+    assert _bwd_varlen(lib, **kw) == expect

@@ -37,8 +37,18 @@ def _check(w):
 
 # (B, Hq, Hkv, Nq, Nk, d, causal): single key; GQA groups of 4 and 8 rows;
 # Nk ragged against the 64-key tiles; Nq = Nk (a whole square problem);
-# G·Nq = 128 rows (eight row groups); d = 64, 128, 256
+# d = 64, 128, 256.  With more than 16 rows per kv head (G·Nq) the
+# tensor-core kernel runs: 40, 64, 128 rows (one 128-row tile, partly
+# filled), 160 and 512 rows (two and four tiles), Nk ragged against its
+# 128-key tiles, shorter than one tile, and square (Nq = Nk, causal)
 CASES = [
+    (1, 8, 2, 16, 1000, 128, True),
+    (2, 16, 2, 5, 777, 64, False),
+    (1, 4, 2, 256, 300, 128, True),
+    (1, 2, 1, 200, 200, 256, True),
+    (1, 32, 8, 32, 4096, 128, True),
+    (2, 8, 1, 20, 20000, 128, False),
+    (1, 4, 1, 30, 100, 256, False),
     (1, 1, 1, 1, 1, 128, True),
     (1, 4, 1, 1, 100, 128, True),
     (2, 8, 2, 3, 1000, 64, True),
@@ -64,6 +74,15 @@ def test_decode_bench_workload_matches_oracle(name):
 
 def test_decode_is_deterministic():
     w = DecodeWorkload("det", 2, 8, 2, 2, 2000, 128, True, 91)
+    q, k, v = make_decode_inputs(w, "cuda")
+    a = attention_decode(q, k, v, causal=True)
+    b = attention_decode(q, k, v, causal=True)
+    torch.cuda.synchronize()
+    assert torch.equal(a[0], b[0]) and torch.equal(a[1], b[1])
+
+
+def test_decode_tensor_core_path_is_deterministic():
+    w = DecodeWorkload("det_tc", 2, 8, 2, 32, 3000, 128, True, 92)
     q, k, v = make_decode_inputs(w, "cuda")
     a = attention_decode(q, k, v, causal=True)
     b = attention_decode(q, k, v, causal=True)

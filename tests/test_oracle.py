@@ -311,6 +311,93 @@ def test_row_block_backward_partials_sum_to_full(causal):
     np.testing.assert_allclose(dv_sum, dv[0, 0], rtol=1e-11, atol=1e-12)
 
 
+# ---------------------------------------------------------------------------
+# Packed variable-length batches
+# ---------------------------------------------------------------------------
+
+VARLEN_CASES = [
+    # (lengths, Hq, Hkv): ragged lengths, a length-1 sequence, an empty one, GQA
+    ([5, 1, 0, 17, 9], 4, 2),
+    ([3, 12], 2, 2),
+    ([1], 1, 1),
+]
+
+
+def _sdpa_block_diagonal(q, k, v, lengths, scale, causal):
+    """torch fp64 SDPA over the whole packed token axis with a boolean mask
+    that lets token i see token j only inside its own sequence (and, causal,
+    only j <= i) -- an independent route to the same definition."""
+    T = q.shape[1]
+    seq = np.repeat(np.arange(len(lengths)), lengths)
+    pos = np.concatenate([np.arange(n) for n in lengths]) if T else np.zeros(0, int)
+    allowed = seq[:, None] == seq[None, :]
+    if causal:
+        allowed &= pos[None, :] <= pos[:, None]
+    G = q.shape[0] // k.shape[0]
+    tq = torch.tensor(q[None], requires_grad=True)
+    tk = torch.tensor(k[None], requires_grad=True)
+    tv = torch.tensor(v[None], requires_grad=True)
+    out = torch.nn.functional.scaled_dot_product_attention(
+        tq, tk.repeat_interleave(G, 1), tv.repeat_interleave(G, 1), attn_mask=torch.tensor(allowed), scale=scale)
+    return tq, tk, tv, out
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("lengths,Hq,Hkv", VARLEN_CASES)
+def test_varlen_matches_block_diagonal_sdpa(lengths, Hq, Hkv, causal):
+    T, d, s = sum(lengths), 6, 0.45
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    q, do = _rand((Hq, T, d), 70), _rand((Hq, T, d), 71)
+    k, v = _rand((Hkv, T, d), 72), _rand((Hkv, T, d), 73)
+    dq, dk, dv, o, lse = oracle.attention_backward_varlen(q, k, v, do, cu, s, causal)
+    o_f, lse_f = oracle.attention_forward_varlen(q, k, v, cu, s, causal)
+    np.testing.assert_array_equal(o, o_f)
+    np.testing.assert_array_equal(lse, lse_f)
+    tq, tk, tv, out = _sdpa_block_diagonal(q, k, v, lengths, s, causal)
+    out.backward(torch.tensor(do[None]))
+    np.testing.assert_allclose(o, out.detach().numpy()[0], rtol=1e-12, atol=1e-13)
+    for mine, ref in ((dq, tq.grad), (dk, tk.grad), (dv, tv.grad)):
+        np.testing.assert_allclose(mine, ref.numpy()[0], rtol=1e-10, atol=1e-12)
+    # LSE from its definition, row by row
+    for b in range(len(lengths)):
+        for i in range(lengths[b]):
+            t = cu[b] + i
+            keys = np.arange(cu[b], cu[b] + (i + 1 if causal else lengths[b]))
+            for h in range(Hq):
+                sc = s * (k[h // (Hq // Hkv), keys] @ q[h, t])
+                assert abs(lse[h, t] - (sc.max() + np.log(np.exp(sc - sc.max()).sum()))) < 1e-12
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_zero_queries_give_sequence_means(causal):
+    lengths = [4, 1, 7]
+    cu = np.concatenate([[0], np.cumsum(lengths)])
+    T, d = sum(lengths), 3
+    v = _rand((1, T, d), 74)
+    o, lse = oracle.attention_forward_varlen(np.zeros((2, T, d)), _rand((1, T, d), 75), v, cu, 0.5, causal)
+    for b, n in enumerate(lengths):
+        for i in range(n):
+            t = cu[b] + i
+            seen = v[0, cu[b]:cu[b] + (i + 1 if causal else n)]
+            np.testing.assert_allclose(o[:, t], np.broadcast_to(seen.mean(axis=0), (2, d)), rtol=1e-13, atol=1e-14)
+            np.testing.assert_allclose(lse[:, t], math.log(len(seen)), rtol=1e-13)
+
+
+def test_varlen_boundary_mistake_is_caught(monkeypatch):
+    # plant a mistake in the oracle: every sequence boundary moved one token
+    # early, so the first token of each sequence joins the previous one
+    orig = oa._varlen_bounds
+
+    def shifted(cu_seqlens, T):
+        cu = orig(cu_seqlens, T)
+        return [0] + [max(0, c - 1) for c in cu[1:-1]] + [cu[-1]]
+
+    monkeypatch.setattr(oa, "_varlen_bounds", shifted)
+    for causal in (False, True):
+        with pytest.raises(AssertionError):
+            test_varlen_matches_block_diagonal_sdpa([5, 1, 0, 17, 9], 4, 2, causal)
+
+
 def test_flop_count():
     # 4·B·Hq·N²·d, halved when causal
     assert oracle.attention_flops(8, 16, 2048, 128, False) == 274877906944.0
