@@ -476,7 +476,8 @@ MEASURED_TRAFFIC = {"long_b1_h16_n16384_d128_causal": 628.1e6}
 
 # The same for one fa_decode_split_kernel launch (also summarised under profiles/);
 # reset to None whenever that kernel changes.
-MEASURED_DECODE_TRAFFIC = {"decode_b8_hq32_hkv8_nk32768_d128": 1079.4e6}
+MEASURED_DECODE_TRAFFIC = {"decode_b8_hq32_hkv8_nk32768_d128": 1079.4e6,
+                           "decode_b8_hq32_hkv8_nq32_nk32768_d128": 1079.0e6}
 
 
 def _l2_note(*tensors) -> str:

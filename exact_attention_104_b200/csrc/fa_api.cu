@@ -14,6 +14,7 @@
 #include "fa_bwd.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_pair.cuh"
 #include "fa_fwd_persistent.cuh"
 #include "fa_varlen.cuh"
 
@@ -223,6 +224,42 @@ fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, co
   const int grid = (!VARLEN && p.n_items < sms) ? p.n_items : sms;
   ProfileScope prof(stream);
   kern<<<grid, C::THREADS, C::SMEM_BYTES, stream>>>(tq, tk, tv, p);
+  return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+// d = 128 on CTA pairs (cta_group::2): clusters of two CTAs, each CTA one
+// 128-row query tile, each K/V tile split between the two.
+#ifndef FA_FWD_PAIR
+#define FA_FWD_PAIR 0
+#endif
+
+template <bool CAUSAL, bool TAIL>
+fa_status launch_fwd_pair(const void* k, const CUtensorMap& tq, const CUtensorMap& tv, const fa::FwdParams& p,
+                          int B, int Hq, uint64_t kvrows, cudaStream_t stream) {
+  using C = fa::FwdPairCfg;
+  auto kern = fa::fa_fwd_pair_kernel<CAUSAL, TAIL>;
+  CUtensorMap tk_half;  // K halves: 64-key boxes
+  if (!make_map(&tk_half, k, kvrows, C::D, 64)) return FA_ERR_CUDA;
+  if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
+    return FA_ERR_CUDA;
+  const int pairs = (p.n_qtiles + 1) / 2;
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = dim3(2u * (unsigned)pairs, (unsigned)Hq, (unsigned)B);
+  cfg.blockDim = dim3(C::THREADS);
+  cfg.dynamicSmemBytes = C::SMEM_BYTES;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeClusterDimension;
+  attr[0].val.clusterDim.x = 2;
+  attr[0].val.clusterDim.y = 1;
+  attr[0].val.clusterDim.z = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  ProfileScope prof(stream);
+  if (cudaLaunchKernelEx(&cfg, kern, tq, tk_half, tv, p) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
@@ -479,11 +516,12 @@ fa_status launch_decode(const fa::DecodeParams& p, int rmax, bool causal, unsign
     default: st = causal ? launch_decode_split<D, 16, true>(p, units, s) : launch_decode_split<D, 16, false>(p, units, s); break;
   }
   if (st != FA_OK) return st;
+  const dim3 cgrid(units, (unsigned)((rmax + fa::kCombineRows - 1) / fa::kCombineRows));
   switch (rmax) {
-    case 128: fa::fa_decode_combine_kernel<D, 128><<<units, 256, 0, s>>>(p); break;
-    case 4: fa::fa_decode_combine_kernel<D, 4><<<units, 256, 0, s>>>(p); break;
-    case 8: fa::fa_decode_combine_kernel<D, 8><<<units, 256, 0, s>>>(p); break;
-    default: fa::fa_decode_combine_kernel<D, 16><<<units, 256, 0, s>>>(p); break;
+    case 128: fa::fa_decode_combine_kernel<D, 128><<<cgrid, 256, 0, s>>>(p); break;
+    case 4: fa::fa_decode_combine_kernel<D, 4><<<cgrid, 256, 0, s>>>(p); break;
+    case 8: fa::fa_decode_combine_kernel<D, 8><<<cgrid, 256, 0, s>>>(p); break;
+    default: fa::fa_decode_combine_kernel<D, 16><<<cgrid, 256, 0, s>>>(p); break;
   }
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
@@ -584,7 +622,12 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   // one kernel instance per (d, causal, ragged tail)
   auto dispatch = [&](auto dtag) -> fa_status {
     constexpr int D = decltype(dtag)::value;
-    if constexpr (D <= 128) {
+    if constexpr (D == 128 && FA_FWD_PAIR) {
+      if (causal) return tail ? launch_fwd_pair<true, true>(k, tq, tv, p, B, Hq, kvrows, s)
+                              : launch_fwd_pair<true, false>(k, tq, tv, p, B, Hq, kvrows, s);
+      return tail ? launch_fwd_pair<false, true>(k, tq, tv, p, B, Hq, kvrows, s)
+                  : launch_fwd_pair<false, false>(k, tq, tv, p, B, Hq, kvrows, s);
+    } else if constexpr (D <= 128) {
       if (causal) return tail ? launch_fwd_persistent<D, true, true>(tq, tk, tv, p, B, Hq, di->sms, s)
                               : launch_fwd_persistent<D, true, false>(tq, tk, tv, p, B, Hq, di->sms, s);
       return tail ? launch_fwd_persistent<D, false, true>(tq, tk, tv, p, B, Hq, di->sms, s)

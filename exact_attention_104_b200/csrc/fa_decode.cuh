@@ -312,17 +312,23 @@ __global__ void __launch_bounds__(DecCfg<D, RMAX>::THREADS)
   }
 }
 
-// One CTA per (batch, kv head, row group); thread = (row, column pair).
+// Rows of a combine CTA: a row group of up to 16 rows is one CTA, the
+// 128-row groups of the tensor-core path are spread over 8 CTAs.
+constexpr int kCombineRows = 16;
+
+// One CTA per (batch, kv head, row group, chunk of kCombineRows rows);
+// thread = (row, column pair).
 template <int D, int RMAX>
 __global__ void __launch_bounds__(256) fa_decode_combine_kernel(const DecodeParams p) {
   const int unit = blockIdx.x;
   const int rg = unit % p.n_rg;
   const int hkv = (unit / p.n_rg) % p.Hkv;
   const int b = unit / (p.n_rg * p.Hkv);
-  const int rows = min(RMAX, p.R - rg * RMAX);
+  const int r0 = blockIdx.y * kCombineRows;
+  const int rows = min(RMAX, p.R - rg * RMAX) - r0;  // rows of this chunk (may be <= 0)
   const size_t units = (size_t)p.B * p.Hkv * p.n_rg;
-  for (int item = threadIdx.x; item < rows * (D / 2); item += blockDim.x) {
-    const int r = item / (D / 2), cp = item - r * (D / 2);
+  for (int item = threadIdx.x; item < min(rows, kCombineRows) * (D / 2); item += blockDim.x) {
+    const int r = r0 + item / (D / 2), cp = item % (D / 2);
     float M = -INFINITY;
     for (int s = 0; s < p.n_split; ++s) M = fmaxf(M, p.part_ml[(((size_t)s * units + unit) * RMAX + r) * 2]);
     float L = 0.f, o0 = 0.f, o1 = 0.f;

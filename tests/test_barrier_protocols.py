@@ -526,281 +526,153 @@ def test_forward_model_catches_a_missing_wait():
     assert caught > 0
 
 
-# --------------------------------------------- forward, three S buffers (planned)
-def simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=3, n_slot=8, ring=4, mistake=None):
-    """The schedule planned for the d = 64 forward, where TMEM has room for a
-    third S buffer: QKᵀ number n (in today's issue order) goes to buffer
-    n mod nbuf, and after every PV (and in the prologue) the MMA warp issues as
-    many next QKᵀs as are allowed, a buffer being reusable once the PV that read
-    its previous occupant has been issued.  S-full and P-full barriers are per
-    (tile, buffer); each softmax warpgroup waits for its previous PV, in order,
-    after its exponentials and before it releases P.  The softmax warpgroups
-    learn each QKᵀ's sequence number from a per-tile ring of ``ring`` slots in
-    shared memory, which the MMA warp fills before it issues the product
-    (one full-barrier per slot, no empty-barrier: the MMA warp runs at most
-    nbuf QKᵀs ahead of the PVs).  Q tiles and K/V units are
-    loaded as in simulate_fwd (K and V of each iteration through ``n_slot``
-    slots, units waited in load order, released by their last reader).  The
-    kernel still uses the two-buffer schedule of simulate_fwd; this model checks
-    the planned one (nbuf = 2 is the same schedule with two buffers).  Since
-    QKᵀs are issued earlier, the K/V ring must be deeper: with three buffers
-    the model deadlocks at 5 slots and runs at 6 (two buffers: 3 and 4); the
-    d = 64 kernel has 8."""
+# ------------------------------------------------------------ forward, CTA pair
+def _kv_order(n):
+    """Load order of fa_fwd_kernel / fa_fwd_pair_kernel's K/V units with two S
+    tiles in flight: K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1)."""
+    unit_k = lambda j: 0 if j == 0 else 2 * j - 1          # noqa: E731
+    unit_v = lambda j: 2 * n - 1 if j == n - 1 else 2 * j + 2  # noqa: E731
+    return unit_k, unit_v
+
+
+def simulate_fwd_pair(n, n_slot, seed, mistake=None):
+    """fa_fwd_pair_kernel: one cluster of two CTAs over ``n`` K/V tiles.  Both
+    CTAs' producers load their halves of every unit and of Q, counted on the
+    leader's barriers (which the leader's producer arms); the leader's MMA
+    warp issues every product on one tensor pipe and commits to the barrier of
+    the same name in both CTAs; the softmax warps of both CTAs (four each,
+    modelled as one role per CTA) arrive on the leader's P barriers."""
     rnd = random.Random(seed)
-    n_pairs = (n_qtiles + 1) // 2
-    n_items = n_pairs * BH
-    done = {"S": [], "PV": []}
+    unit_k, unit_v = _kv_order(n)
+    bars = {}
+    for r in range(2):
+        for s in range(n_slot):
+            bars[r, "KVEMPTY", s] = _Bar(1)
+        for x in range(2):
+            bars[r, "SFULL", x] = _Bar(1)
+            bars[r, "ODONE", x] = _Bar(1)
+        bars[r, "DRAIN"] = _Bar(1)
+    bars[0, "QFULL"] = _Bar(3)           # the leader's arming arrival + two Q loads
+    for s in range(n_slot):
+        bars[0, "KVFULL", s] = _Bar(3)   # the leader's arming arrival + two halves
+    for x in range(2):
+        bars[0, "PFULL", x] = _Bar(8)
+        bars[0, "PFULL2", x] = _Bar(8)
+    wait = _waiter(bars)
+    tc, tma = [], {0: [], 1: []}
+    halves = {}                 # unit -> halves landed
+    slot_unit = {}              # (cta, slot) -> unit
+    read_done = set()           # units whose last reading product has completed
+    p_phase_tiles = {}          # (name, x, phase) -> tiles of the arrivals
+    p_count = {}
+    issued = []
 
-    def item(idx):
-        if causal:
-            pair, bh = n_pairs - 1 - idx // BH, idx % BH
-        else:
-            bh, pair = idx // n_pairs, idx % n_pairs
-        qt0 = 2 * pair
-        has1 = qt0 + 1 < n_qtiles
-        n0 = qt0 + 1 if causal else n_qtiles
-        n1 = (qt0 + 2 if causal else n_qtiles) if has1 else 0
-        skew = 1 if (causal and has1) else 0
-        return dict(qt0=qt0, n0=n0, n1=n1, skew=skew, nit=n0 + skew)
+    def producer(r):
+        if r == 0:
+            bars[0, "QFULL"].arrive()
+        tma[r].append(((0, "QFULL"), None))
+        for u in range(2 * n):
+            s = u % n_slot
+            if u >= n_slot and mistake != "no_kvempty_wait":
+                yield from wait((r, "KVEMPTY", s), u // n_slot - 1)
+            if (r, s) in slot_unit:
+                assert slot_unit[r, s] in read_done, f"cta {r} slot {s} refilled while unit {slot_unit[r, s]} is read"
+            slot_unit[r, s] = u
+            if r == 0:
+                bars[0, "KVFULL", s].arrive()
+            tma[r].append(((0, "KVFULL", s), u))
+            yield
 
-    def kvb(w, jj):
-        return w["qt0"] + 1 if (w["skew"] and jj == 0) else jj - w["skew"]
+    def mma():
+        yield from wait((0, "QFULL"), 0)
+        ready = {"k": -1, "v": -1}
 
-    def first(w, t):
-        return w["skew"] if t == 0 else 0
+        def need(kind, j):
+            if j <= ready[kind]:
+                return
+            ready[kind] = j
+            u = unit_k(j) if kind == "k" else unit_v(j)
+            yield from wait((0, "KVFULL", u % n_slot), u // n_slot)
+            assert halves.get(u) == 2, f"unit {u} used with {halves.get(u)} halves"
 
-    def has(w, t):
-        return t == 0 or w["n1"] > 0
+        def s_tile(j):
+            yield from need("k", j)
+            issued.append(("S", j))
+            tc.append(("commit", "SFULL", j & 1))
+            tc.append(("release", unit_k(j)))
 
-    def deal(k, c):
-        return k * n_ctas + ((n_ctas - 1 - c) if (causal and (k & 1)) else c)
+        yield from s_tile(0)
+        if n > 1:
+            yield from s_tile(1)
+        for j in range(n):
+            x = j & 1
+            yield from wait((0, "PFULL", x), j >> 1)
+            assert p_phase_tiles[("PFULL", x, j >> 1)] == {j}, "P barrier phase mixes tiles"
+            yield from need("v", j)
+            yield from wait((0, "PFULL2", x), j >> 1)
+            assert p_phase_tiles[("PFULL2", x, j >> 1)] == {j}, "P barrier phase mixes tiles"
+            issued.append(("PV", j))
+            tc.append(("commit", "ODONE", x))
+            tc.append(("release", unit_v(j)))
+            if j + 2 < n:
+                yield from s_tile(j + 2)
+        tc.append(("commit", "DRAIN", None))
+        yield from wait((0, "DRAIN"), 0)
 
-    n_rounds = (n_items + n_ctas - 1) // n_ctas
-    gens, engines = {}, {}
-
-    def make_cta(c):
-        items = [deal(k, c) for k in range(n_rounds) if deal(k, c) < n_items]
-        base_of = {}
-        acc = 0
-        for idx in items:
-            base_of[idx] = acc
-            acc += 2 * item(idx)["nit"]
-        # the QKᵀ sequence in today's issue order, and the PV order
-        seq, pv_order = [], []
-        if items:
-            w0 = item(items[0])
-            for t in range(2):
-                if has(w0, t):
-                    seq.append((items[0], t, first(w0, t)))
-            for pos, idx in enumerate(items):
-                w = item(idx)
-                nxt = items[pos + 1] if pos + 1 < len(items) else None
-                w2 = item(nxt) if nxt is not None else None
-                for jj in range(w["nit"]):
-                    for t in range(2):
-                        if not has(w, t) or jj < first(w, t):
-                            continue
-                        pv_order.append((idx, t, jj))
-                        if jj + 1 < w["nit"]:
-                            seq.append((idx, t, jj + 1))
-                        elif nxt is not None and has(w2, t):
-                            seq.append((nxt, t, first(w2, t)))
-                if nxt is not None and not has(w, 1) and has(w2, 1):
-                    seq.append((nxt, 1, 0))
-        seq_no = {e: n for n, e in enumerate(seq)}
-        assert len(seq_no) == len(seq) == len(pv_order)
-        # phase index of QKᵀ n on its (tile, buffer) barriers: how many earlier
-        # QKᵀs of the same tile went to the same buffer
-        phase = {}
-        cnt = {}
-        for n, e in enumerate(seq):
-            key = (e[1], n % nbuf)
-            phase[n] = cnt.get(key, 0)
-            cnt[key] = phase[n] + 1
-        bars = {}
-        for t in range(2):
-            for b in range(nbuf):
-                bars["SFULL", t, b] = _Bar(1)   # per (tile, buffer)
-                bars["PFULL", t, b] = _Bar(4)
-            bars["ODONE", t] = _Bar(1)
-            bars["QFULL", t] = _Bar(1)
-            bars["QEMPTY", t] = _Bar(1)
-            for r in range(ring):
-                bars["NFULL", t, r] = _Bar(1)
-        for sl in range(n_slot):
-            bars["KVFULL", sl] = _Bar(1)
-            bars["KVEMPTY", sl] = _Bar(1)
-        wait = _waiter(bars)
-        tc, tma = [], []
-        buf_owner = {}        # buffer -> QKᵀ number written last
-        pv_issued = set()     # QKᵀ numbers whose PV has been issued
-        p_written = set()
-        q_tile = {0: None, 1: None}
-        ring_slot = {}                   # (tile, slot) -> sequence number written last
-        ring_read = set()                # (tile, tile QKᵀ count) entries read
-        issued_per_tile = [0, 0]
-        slot_unit, released, loaded = {}, set(), set()
-
-        def producer():
-            useq = 0
-            q_loads = [0, 0]
-            for idx in items:
-                w = item(idx)
-                for t in range(2):
-                    if not has(w, t):
-                        continue
-                    if q_loads[t] > 0:
-                        yield from wait(("QEMPTY", t), q_loads[t] - 1)
-                    q_tile[t] = idx
-                    tma.append((("QFULL", t), None))
-                    q_loads[t] += 1
-                for u in range(2 * w["nit"]):
-                    U = useq + u
-                    sl = U % n_slot
-                    if U >= n_slot:
-                        yield from wait(("KVEMPTY", sl), U // n_slot - 1)
-                    if sl in slot_unit:
-                        assert slot_unit[sl] in released, f"slot {sl} refilled while unit {slot_unit[sl]} is read"
-                    slot_unit[sl] = U
-                    tma.append((("KVFULL", sl), U))
-                useq += 2 * w["nit"]
-
-        def mma():
-            nxt = [0]
-            waited = [-1]
-            q_seen = [0, 0]
-
-            def wait_upto(U):
-                while waited[0] < U:
-                    waited[0] += 1
-                    yield from wait(("KVFULL", waited[0] % n_slot), waited[0] // n_slot)
-                    assert waited[0] in loaded
-
-            def release(U):
-                assert U not in released
-                released.add(U)
-                tc.append(("commit", ("KVEMPTY", U % n_slot)))
-
-            def try_issue():
-                while nxt[0] < len(seq):
-                    n = nxt[0]
-                    b = n % nbuf
-                    if n >= nbuf and (n - nbuf) not in pv_issued and mistake != "no_buffer_rule":
-                        return
-                    idx, t, jj = seq[n]
-                    w = item(idx)
-                    if jj == first(w, t):
-                        yield from wait(("QFULL", t), q_seen[t])
-                        q_seen[t] += 1
-                    assert q_tile[t] == idx, "Q tile overwritten"
-                    U = base_of[idx] + 2 * jj
-                    yield from wait_upto(U)
-                    if b in buf_owner:
-                        assert buf_owner[b] in pv_issued, "S overwrites an unconsumed P"
-                    buf_owner[b] = n
-                    g = issued_per_tile[t]
-                    if g >= ring:
-                        assert (t, g - ring) in ring_read, "ring slot overwritten before it was read"
-                    ring_slot[t, g % ring] = n
-                    bars["NFULL", t, g % ring].arrive()
-                    issued_per_tile[t] = g + 1
-                    done["S"].append(seq[n])
-                    tc.append(("commit", ("SFULL", t, b)))
-                    if jj == w["nit"] - 1:
-                        tc.append(("commit", ("QEMPTY", t)))
-                    if t == 1 or w["n1"] == 0:
-                        release(U)
-                    nxt[0] += 1
-            yield from try_issue()
-            for (idx, t, jj) in pv_order:
-                n = seq_no[(idx, t, jj)]
-                w = item(idx)
-                yield from wait(("PFULL", t, n % nbuf), phase[n])
-                Uv = base_of[idx] + 2 * jj + 1
-                yield from wait_upto(Uv)
-                assert n in p_written and n not in pv_issued and Uv not in released
-                pv_issued.add(n)
-                done["PV"].append((idx, t, jj))
-                tc.append(("commit", ("ODONE", t)))
-                if t == 1 or w["n1"] == 0:
-                    release(Uv)
-                yield
-                yield from try_issue()
-            assert nxt[0] == len(seq), "QKᵀs left unissued"
-
-        def softmax(t):
-            mine = [n for n, e in enumerate(seq) if e[1] == t]
-            seen = [-1]
-
-            def odone_upto(k):
-                # PV completions are waited in order, never skipping one
-                while seen[0] < k:
-                    seen[0] += 1
-                    yield from wait(("ODONE", t), seen[0])
-            for j, n in enumerate(mine):
-                yield from wait(("NFULL", t, j % ring), j // ring)
-                assert ring_slot[t, j % ring] == n, "wrong sequence number in the ring"
-                ring_read.add((t, j))
-                yield from wait(("SFULL", t, n % nbuf), phase[n])
-                yield                                   # S load, row max, exponentials
-                # the previous PV must be done before O is rescaled (rare) and
-                # before this P is released; PV(j) cannot have started yet, so
-                # at most one ODONE phase is outstanding here
-                if j > 0:
-                    yield from odone_upto(j - 1)
-                yield                                   # rescale of O, P store
-                assert buf_owner[n % nbuf] == n, "S overwritten before its softmax finished"
-                p_written.add(n)
+    def softmax(r):
+        for j in range(n):
+            x = j & 1
+            yield from wait((r, "SFULL", x), j >> 1)
+            if j > 0 and rnd.random() < 0.3:      # conditional rescale of O
+                yield from wait((r, "ODONE", (j - 1) & 1), (j - 1) >> 1)
+            for name in ("PFULL", "PFULL2"):
+                key = (name, x)
+                ph = p_count.get(key, 0) // 8
+                p_phase_tiles.setdefault((name, x, ph), set()).add(j)
                 for _ in range(4):
-                    bars["PFULL", t, n % nbuf].arrive()
-            if mine:
-                yield from odone_upto(len(mine) - 1)
+                    p_count[key] = p_count.get(key, 0) + 1
+                    bars[0, name, x].arrive()
+                yield
+        yield from wait((r, "ODONE", (n - 1) & 1), (n - 1) >> 1)
 
-        def tc_done(entry):
-            bars[entry[1]].arrive()
+    def tc_done(entry):
+        kind = entry[0]
+        if kind == "commit":
+            _, name, x = entry
+            for r in range(2):                    # multicast to both CTAs
+                bars[(r, name) if x is None else (r, name, x)].arrive()
+        else:
+            u = entry[1]
+            read_done.add(u)
+            for r in range(2):
+                bars[r, "KVEMPTY", u % n_slot].arrive()
 
-        def tma_done(entry):
-            bar, unit = entry
-            if unit is not None:
-                loaded.add(unit)
-            bars[bar].arrive()
+    def tma_done(entry):
+        bar, unit = entry
+        if unit is not None:
+            halves[unit] = halves.get(unit, 0) + 1
+        bars[bar].arrive()
 
-        gens[c, "producer"] = producer()
-        gens[c, "mma"] = mma()
-        gens[c, "sm", 0] = softmax(0)
-        gens[c, "sm", 1] = softmax(1)
-        engines[c, "tc"] = (tc, tc_done)
-        engines[c, "tma"] = (tma, tma_done)
-
-    for c in range(n_ctas):
-        make_cta(c)
+    gens = {"producer0": producer(0), "producer1": producer(1), "mma": mma(),
+            "softmax0": softmax(0), "softmax1": softmax(1)}
+    engines = {"tc": (tc, tc_done), "tma0": (tma[0], tma_done), "tma1": (tma[1], tma_done)}
     _run(gens, engines, rnd)
-    for kind in ("S", "PV"):
-        got = sorted((i, t, kvb(item(i), jj)) for (i, t, jj) in done[kind])
-        want = []
-        for idx in range(n_items):
-            w = item(idx)
-            for t in range(2):
-                if has(w, t):
-                    qt = w["qt0"] + t
-                    want += [(idx, t, j) for j in (range(qt + 1) if causal else range(n_qtiles))]
-        assert got == sorted(want), kind
+    assert [k for k in issued if k[0] == "PV"] == [("PV", j) for j in range(n)]
+    assert sorted(j for k, j in issued if k == "S") == list(range(n))
 
 
-@pytest.mark.parametrize("nbuf,n_slot", [(3, 8), (2, 5)])
-@pytest.mark.parametrize("causal", [False, True])
-def test_three_buffer_forward_schedule(causal, nbuf, n_slot):
-    for n_qtiles in (1, 2, 3, 5, 8):
-        for BH, n_ctas in ((1, 1), (3, 2), (5, 3)):
-            for seed in range(3):
-                simulate_fwd_three_buffers(n_qtiles, BH, causal, n_ctas, seed, nbuf=nbuf, n_slot=n_slot)
+@pytest.mark.parametrize("n_slot", [10, 4])
+def test_forward_pair_protocol(n_slot):
+    for n in (1, 2, 3, 7, 16):
+        for seed in range(6):
+            simulate_fwd_pair(n, n_slot, seed=seed * 31 + n)
 
 
-def test_three_buffer_model_catches_a_buffer_reused_too_early():
+def test_forward_pair_model_catches_a_missing_wait():
     caught = 0
-    for seed in range(10):
+    for seed in range(30):
         try:
-            simulate_fwd_three_buffers(5, 3, True, 2, seed, mistake="no_buffer_rule")
+            simulate_fwd_pair(12, 4, seed, mistake="no_kvempty_wait")
         except AssertionError:
             caught += 1
     assert caught > 0
