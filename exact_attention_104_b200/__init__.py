@@ -7,6 +7,7 @@ ABI declared in ``include/fa.h``); this package only marshals arguments.
 from .binding import (  # noqa: F401
     FAError,
     fa_fwd,
+    fa_fwd_pair,
     fa_bwd,
     fa_bwd_workspace_bytes,
     fa_device_status,

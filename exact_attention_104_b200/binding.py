@@ -41,6 +41,8 @@ def lib() -> ctypes.CDLL:
     vp, i, f, z = ctypes.c_void_p, ctypes.c_int, ctypes.c_float, ctypes.c_size_t
     L.fa_fwd.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
     L.fa_fwd.restype = i
+    L.fa_fwd_pair.argtypes = [vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp]
+    L.fa_fwd_pair.restype = i
     L.fa_bwd_workspace_bytes.argtypes = [i, i, i, i, i]
     L.fa_bwd_workspace_bytes.restype = z
     L.fa_bwd.argtypes = [vp, vp, vp, vp, vp, vp, vp, vp, vp, i, i, i, i, i, i, f, vp, z, vp]
@@ -108,6 +110,13 @@ def fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream=None) -> int
     """Raw C-ABI call; tensors or integer device pointers.  Returns the status."""
     return lib().fa_fwd(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
                         int(bool(causal)), float(scale), _stream_handle(stream))
+
+
+def fa_fwd_pair(q, k, v, o, lse, B, Hq, Hkv, N, d, causal, scale, stream=None) -> int:
+    """Raw C-ABI call of the forward pass on CTA pairs (d = 128).  Returns the
+    status."""
+    return lib().fa_fwd_pair(_ptr(q), _ptr(k), _ptr(v), _ptr(o), _ptr(lse), B, Hq, Hkv, N, d,
+                             int(bool(causal)), float(scale), _stream_handle(stream))
 
 
 def fa_bwd_workspace_bytes(B, Hq, Hkv, N, d) -> int:

@@ -227,24 +227,22 @@ fa_status launch_fwd_persistent(const CUtensorMap& tq, const CUtensorMap& tk, co
   return cudaGetLastError() == cudaSuccess ? FA_OK : FA_ERR_CUDA;
 }
 
-// d = 128 on CTA pairs (cta_group::2): clusters of two CTAs, each CTA one
-// 128-row query tile, each K/V tile split between the two.
-#ifndef FA_FWD_PAIR
-#define FA_FWD_PAIR 0
-#endif
+// d = 128 on CTA pairs (cta_group::2): clusters of two CTAs, each CTA two
+// 128-row query tiles, each K/V block split between the two (fa_fwd_pair).
 
 template <bool CAUSAL, bool TAIL>
 fa_status launch_fwd_pair(const void* k, const CUtensorMap& tq, const CUtensorMap& tv, const fa::FwdParams& p,
                           int B, int Hq, uint64_t kvrows, cudaStream_t stream) {
   using C = fa::FwdPairCfg;
   auto kern = fa::fa_fwd_pair_kernel<CAUSAL, TAIL>;
+  if (!reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
   CUtensorMap tk_half;  // K halves: 64-key boxes
   if (!make_map(&tk_half, k, kvrows, C::D, 64)) return FA_ERR_CUDA;
   if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, C::SMEM_BYTES) != cudaSuccess)
     return FA_ERR_CUDA;
-  const int pairs = (p.n_qtiles + 1) / 2;
+  const int items = (p.n_qtiles + 3) / 4;  // four query tiles per cluster
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(2u * (unsigned)pairs, (unsigned)Hq, (unsigned)B);
+  cfg.gridDim = dim3(2u * (unsigned)items, (unsigned)Hq, (unsigned)B);
   cfg.blockDim = dim3(C::THREADS);
   cfg.dynamicSmemBytes = C::SMEM_BYTES;
   cfg.stream = stream;
@@ -622,12 +620,7 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
   // one kernel instance per (d, causal, ragged tail)
   auto dispatch = [&](auto dtag) -> fa_status {
     constexpr int D = decltype(dtag)::value;
-    if constexpr (D == 128 && FA_FWD_PAIR) {
-      if (causal) return tail ? launch_fwd_pair<true, true>(k, tq, tv, p, B, Hq, kvrows, s)
-                              : launch_fwd_pair<true, false>(k, tq, tv, p, B, Hq, kvrows, s);
-      return tail ? launch_fwd_pair<false, true>(k, tq, tv, p, B, Hq, kvrows, s)
-                  : launch_fwd_pair<false, false>(k, tq, tv, p, B, Hq, kvrows, s);
-    } else if constexpr (D <= 128) {
+    if constexpr (D <= 128) {
       if (causal) return tail ? launch_fwd_persistent<D, true, true>(tq, tk, tv, p, B, Hq, di->sms, s)
                               : launch_fwd_persistent<D, true, false>(tq, tk, tv, p, B, Hq, di->sms, s);
       return tail ? launch_fwd_persistent<D, false, true>(tq, tk, tv, p, B, Hq, di->sms, s)
@@ -644,6 +637,48 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
     case 256: return dispatch(std::integral_constant<int, 256>{});
   }
   return FA_ERR_UNSUPPORTED;
+}
+
+fa_status fa_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse, int B, int Hq, int Hkv,
+                      int N, int d, int causal, float scale, void* stream) {
+  bool empty = false;
+  fa_status st = check_sizes(B, Hq, Hkv, N, d, scale, &empty);
+  if (st != FA_OK || empty) return st;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  const size_t qbytes = (size_t)B * Hq * N * d * 2, kvbytes = (size_t)B * Hkv * N * d * 2;
+  const Range rq = span(q, qbytes), rk = span(k, kvbytes), rv = span(v, kvbytes);
+  const Range ro = span(o, qbytes), rl = span(lse, (size_t)B * Hq * N * 4);
+  for (Range out : {ro, rl})
+    for (Range in : {rq, rk, rv})
+      if (overlap(out, in)) return FA_ERR_INVALID_ARG;
+  if (overlap(ro, rl)) return FA_ERR_INVALID_ARG;
+  DeviceInfo* di = nullptr;
+  st = current_device(&di);
+  if (st != FA_OK) return st;
+  const uint64_t qrows = (uint64_t)B * Hq * N, kvrows = (uint64_t)B * Hkv * N;
+  // the item of the last query tiles reads up to three tiles past N
+  if (qrows + 3 * 128 >= (1ULL << 31)) return FA_ERR_UNSUPPORTED;
+  CUtensorMap tq, tv;
+  if (!make_map(&tq, q, qrows, d, 128) || !make_map(&tv, v, kvrows, d, 128)) return FA_ERR_CUDA;
+  fa::FwdParams p{};
+  p.o = static_cast<__nv_bfloat16*>(o);
+  p.lse = lse;
+  p.N = N;
+  p.Hq = Hq;
+  p.Hkv = Hkv;
+  p.G = Hq / Hkv;
+  p.n_qtiles = (N + 127) / 128;
+  p.scale_log2 = scale * fa::kLog2e;
+  p.wait_cap = g_wait_cap.load(std::memory_order_relaxed);
+  p.err = di->err;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  const bool tail = (N % 128) != 0;
+  if (causal) return tail ? launch_fwd_pair<true, true>(k, tq, tv, p, B, Hq, kvrows, s)
+                          : launch_fwd_pair<true, false>(k, tq, tv, p, B, Hq, kvrows, s);
+  return tail ? launch_fwd_pair<false, true>(k, tq, tv, p, B, Hq, kvrows, s)
+              : launch_fwd_pair<false, false>(k, tq, tv, p, B, Hq, kvrows, s);
 }
 
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dout,

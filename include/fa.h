@@ -81,6 +81,17 @@ fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* ls
                  int B, int Hq, int Hkv, int N, int d, int causal, float scale,
                  void* stream);
 
+/* The same forward pass (same arguments, layouts, results within the same
+ * rounding) computed on pairs of CTAs that share every tensor-core product
+ * (tcgen05 cta_group::2, the "2-CTA MMA" of FA4 in the version table of the
+ * handbook page "FlashAttention"): a cluster of two CTAs takes four query
+ * tiles of 128 rows, each CTA two of them, and each CTA loads only half of
+ * every K/V block.  d = 128 only (other d: FA_ERR_UNSUPPORTED).  On B200 it
+ * measured 12-26 % slower than fa_fwd, which therefore does not use it. */
+fa_status fa_fwd_pair(const void* q, const void* k, const void* v, void* o, float* lse,
+                      int B, int Hq, int Hkv, int N, int d, int causal, float scale,
+                      void* stream);
+
 /* Bytes of device workspace fa_bwd needs: two fp32 [B,Hq,Np] row vectors
  * (D = rowsum(dO∘O) and LSE·log2 e) and an fp32 [B,Hq,Np,d] dQ accumulator,
  * each rounded up to 256 bytes, where Np = N rounded up to a multiple of 128

@@ -285,3 +285,16 @@ def test_fwd_varlen_argument_validation(lib, kw, expect):
 ])
 def test_bwd_varlen_argument_validation(lib, kw, expect):
     assert _bwd_varlen(lib, **kw) == expect
+
+
+def test_pair_forward_argument_validation(lib):
+    a = dict(q=FAKE, k=FAKE * 2, v=FAKE * 3, o=FAKE * 4, lse=FAKE * 5, B=1, Hq=2, Hkv=2, N=256, d=128, causal=0,
+             scale=0.088)
+    call = lambda **kw: binding.fa_fwd_pair(*[{**a, **kw}[n] for n in ("q", "k", "v", "o", "lse", "B", "Hq", "Hkv",  # noqa: E731
+                                                                       "N", "d", "causal", "scale")], 0)
+    assert call(d=64) == binding.FA_ERR_UNSUPPORTED
+    assert call(d=256) == binding.FA_ERR_UNSUPPORTED
+    assert call(q=0) == binding.FA_ERR_INVALID_ARG
+    assert call(o=FAKE) == binding.FA_ERR_INVALID_ARG       # output aliases q
+    assert call(Hq=3) == binding.FA_ERR_INVALID_ARG
+    assert call(N=0) == binding.FA_OK

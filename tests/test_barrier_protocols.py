@@ -527,43 +527,39 @@ def test_forward_model_catches_a_missing_wait():
 
 
 # ------------------------------------------------------------ forward, CTA pair
-def _kv_order(n):
-    """Load order of fa_fwd_kernel / fa_fwd_pair_kernel's K/V units with two S
-    tiles in flight: K0, K1, V0, K2, V1, ..., K(n-1), V(n-2), V(n-1)."""
-    unit_k = lambda j: 0 if j == 0 else 2 * j - 1          # noqa: E731
-    unit_v = lambda j: 2 * n - 1 if j == n - 1 else 2 * j + 2  # noqa: E731
-    return unit_k, unit_v
-
-
-def simulate_fwd_pair(n, n_slot, seed, mistake=None):
-    """fa_fwd_pair_kernel: one cluster of two CTAs over ``n`` K/V tiles.  Both
-    CTAs' producers load their halves of every unit and of Q, counted on the
-    leader's barriers (which the leader's producer arms); the leader's MMA
-    warp issues every product on one tensor pipe and commits to the barrier of
-    the same name in both CTAs; the softmax warps of both CTAs (four each,
-    modelled as one role per CTA) arrive on the leader's P barriers."""
+def simulate_fwd_pair(n0, n1, n_slot, seed, mistake=None, max_steps=20_000_000):
+    """fa_fwd_pair_kernel: one cluster of two CTAs, each with two query tiles;
+    tile pair t (one tile in each CTA) multiplies K/V blocks 0 .. n_t - 1,
+    n0 <= n1.  Both CTAs' producers load their Q tiles and their halves of
+    every K/V unit (K(0), V(0), K(1), V(1), ...), counted on the leader's
+    barriers, which the leader's producer arms; the leader's MMA warp issues
+    every product on one tensor pipe and commits to the barrier of the same
+    name in both CTAs; the softmax warps of tile pair t in both CTAs (four per
+    CTA, modelled as one role per CTA) arrive on the leader's P barriers of
+    tile pair t."""
+    assert 1 <= n0 <= n1
     rnd = random.Random(seed)
-    unit_k, unit_v = _kv_order(n)
+    n_of = (n0, n1)
     bars = {}
     for r in range(2):
         for s in range(n_slot):
             bars[r, "KVEMPTY", s] = _Bar(1)
-        for x in range(2):
-            bars[r, "SFULL", x] = _Bar(1)
-            bars[r, "ODONE", x] = _Bar(1)
+        for t in range(2):
+            bars[r, "SFULL", t] = _Bar(1)
+            bars[r, "ODONE", t] = _Bar(1)
         bars[r, "DRAIN"] = _Bar(1)
-    bars[0, "QFULL"] = _Bar(3)           # the leader's arming arrival + two Q loads
+    bars[0, "QFULL"] = _Bar(3)           # the leader's arming arrival + both CTAs' Q loads
     for s in range(n_slot):
         bars[0, "KVFULL", s] = _Bar(3)   # the leader's arming arrival + two halves
-    for x in range(2):
-        bars[0, "PFULL", x] = _Bar(8)
-        bars[0, "PFULL2", x] = _Bar(8)
+    for t in range(2):
+        bars[0, "PFULL", t] = _Bar(8)
+        bars[0, "PFULL2", t] = _Bar(8)
     wait = _waiter(bars)
     tc, tma = [], {0: [], 1: []}
     halves = {}                 # unit -> halves landed
     slot_unit = {}              # (cta, slot) -> unit
     read_done = set()           # units whose last reading product has completed
-    p_phase_tiles = {}          # (name, x, phase) -> tiles of the arrivals
+    p_phase_blocks = {}         # (name, t, phase) -> blocks of the arrivals
     p_count = {}
     issued = []
 
@@ -571,7 +567,7 @@ def simulate_fwd_pair(n, n_slot, seed, mistake=None):
         if r == 0:
             bars[0, "QFULL"].arrive()
         tma[r].append(((0, "QFULL"), None))
-        for u in range(2 * n):
+        for u in range(2 * n1):
             s = u % n_slot
             if u >= n_slot and mistake != "no_kvempty_wait":
                 yield from wait((r, "KVEMPTY", s), u // n_slot - 1)
@@ -585,62 +581,67 @@ def simulate_fwd_pair(n, n_slot, seed, mistake=None):
 
     def mma():
         yield from wait((0, "QFULL"), 0)
-        ready = {"k": -1, "v": -1}
+        waited = [-1]
 
-        def need(kind, j):
-            if j <= ready[kind]:
-                return
-            ready[kind] = j
-            u = unit_k(j) if kind == "k" else unit_v(j)
-            yield from wait((0, "KVFULL", u % n_slot), u // n_slot)
-            assert halves.get(u) == 2, f"unit {u} used with {halves.get(u)} halves"
+        def wait_upto(u):
+            while waited[0] < u:
+                waited[0] += 1
+                yield from wait((0, "KVFULL", waited[0] % n_slot), waited[0] // n_slot)
+                assert halves.get(waited[0]) == 2
 
-        def s_tile(j):
-            yield from need("k", j)
-            issued.append(("S", j))
-            tc.append(("commit", "SFULL", j & 1))
-            tc.append(("release", unit_k(j)))
+        def issue_s(t, j):
+            yield from wait_upto(2 * j)
+            assert 2 * j not in read_done
+            issued.append(("S", t, j))
+            tc.append(("commit", "SFULL", t))
+            if t == 1 and mistake != "release_k_early":
+                tc.append(("release", 2 * j))
+            if t == 0 and mistake == "release_k_early":
+                tc.append(("release", 2 * j))
 
-        yield from s_tile(0)
-        if n > 1:
-            yield from s_tile(1)
-        for j in range(n):
-            x = j & 1
-            yield from wait((0, "PFULL", x), j >> 1)
-            assert p_phase_tiles[("PFULL", x, j >> 1)] == {j}, "P barrier phase mixes tiles"
-            yield from need("v", j)
-            yield from wait((0, "PFULL2", x), j >> 1)
-            assert p_phase_tiles[("PFULL2", x, j >> 1)] == {j}, "P barrier phase mixes tiles"
-            issued.append(("PV", j))
-            tc.append(("commit", "ODONE", x))
-            tc.append(("release", unit_v(j)))
-            if j + 2 < n:
-                yield from s_tile(j + 2)
+        yield from issue_s(0, 0)
+        yield from issue_s(1, 0)
+        for j in range(n1):
+            for t in range(2):
+                if j >= n_of[t]:
+                    continue
+                yield from wait((0, "PFULL", t), j)
+                assert p_phase_blocks[("PFULL", t, j)] == {j}, "P barrier phase mixes blocks"
+                yield from wait_upto(2 * j + 1)
+                assert 2 * j + 1 not in read_done
+                yield from wait((0, "PFULL2", t), j)
+                assert p_phase_blocks[("PFULL2", t, j)] == {j}, "P barrier phase mixes blocks"
+                issued.append(("PV", t, j))
+                tc.append(("commit", "ODONE", t))
+                if t == 1:
+                    tc.append(("release", 2 * j + 1))
+                if j + 1 < n_of[t]:
+                    yield from issue_s(t, j + 1)
         tc.append(("commit", "DRAIN", None))
         yield from wait((0, "DRAIN"), 0)
 
-    def softmax(r):
+    def softmax(r, t):
+        n = n_of[t]
         for j in range(n):
-            x = j & 1
-            yield from wait((r, "SFULL", x), j >> 1)
-            if j > 0 and rnd.random() < 0.3:      # conditional rescale of O
-                yield from wait((r, "ODONE", (j - 1) & 1), (j - 1) >> 1)
+            yield from wait((r, "SFULL", t), j)
+            if j > 0 and rnd.random() < 0.3:      # conditional rescale of O_t
+                yield from wait((r, "ODONE", t), j - 1)
             for name in ("PFULL", "PFULL2"):
-                key = (name, x)
+                key = (name, t)
                 ph = p_count.get(key, 0) // 8
-                p_phase_tiles.setdefault((name, x, ph), set()).add(j)
+                p_phase_blocks.setdefault((name, t, ph), set()).add(j)
                 for _ in range(4):
                     p_count[key] = p_count.get(key, 0) + 1
-                    bars[0, name, x].arrive()
+                    bars[0, name, t].arrive()
                 yield
-        yield from wait((r, "ODONE", (n - 1) & 1), (n - 1) >> 1)
+        yield from wait((r, "ODONE", t), n - 1)
 
     def tc_done(entry):
         kind = entry[0]
         if kind == "commit":
-            _, name, x = entry
+            _, name, t = entry
             for r in range(2):                    # multicast to both CTAs
-                bars[(r, name) if x is None else (r, name, x)].arrive()
+                bars[(r, name) if t is None else (r, name, t)].arrive()
         else:
             u = entry[1]
             read_done.add(u)
@@ -653,26 +654,31 @@ def simulate_fwd_pair(n, n_slot, seed, mistake=None):
             halves[unit] = halves.get(unit, 0) + 1
         bars[bar].arrive()
 
-    gens = {"producer0": producer(0), "producer1": producer(1), "mma": mma(),
-            "softmax0": softmax(0), "softmax1": softmax(1)}
+    gens = {"producer0": producer(0), "producer1": producer(1), "mma": mma()}
+    for r in range(2):
+        for t in range(2):
+            gens[f"softmax{r}{t}"] = softmax(r, t)
     engines = {"tc": (tc, tc_done), "tma0": (tma[0], tma_done), "tma1": (tma[1], tma_done)}
-    _run(gens, engines, rnd)
-    assert [k for k in issued if k[0] == "PV"] == [("PV", j) for j in range(n)]
-    assert sorted(j for k, j in issued if k == "S") == list(range(n))
+    _run(gens, engines, rnd, max_steps)
+    for t in range(2):
+        assert [x for x in issued if x[:2] == ("PV", t)] == [("PV", t, j) for j in range(n_of[t])]
+        assert [x for x in issued if x[:2] == ("S", t)] == [("S", t, j) for j in range(n_of[t])]
 
 
-@pytest.mark.parametrize("n_slot", [10, 4])
+@pytest.mark.parametrize("n_slot", [9, 3])
 def test_forward_pair_protocol(n_slot):
-    for n in (1, 2, 3, 7, 16):
-        for seed in range(6):
-            simulate_fwd_pair(n, n_slot, seed=seed * 31 + n)
+    for n0, n1 in ((1, 1), (1, 3), (2, 4), (6, 6)):
+        for seed in range(3):
+            simulate_fwd_pair(n0, n1, n_slot, seed=seed * 31 + n1)
 
 
-def test_forward_pair_model_catches_a_missing_wait():
+@pytest.mark.parametrize("mistake", ["no_kvempty_wait", "release_k_early"])
+def test_forward_pair_model_catches_a_mistake(mistake):
     caught = 0
-    for seed in range(30):
+    for seed in range(12):
         try:
-            simulate_fwd_pair(12, 4, seed, mistake="no_kvempty_wait")
+            simulate_fwd_pair(3, 5, 3, seed, mistake=mistake, max_steps=200_000)
         except AssertionError:
             caught += 1
+            break
     assert caught > 0
