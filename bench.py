@@ -390,6 +390,135 @@ def run_decode_reference(args, w, rank):
     print(json.dumps(line), flush=True)
 
 
+# ----------------------------------------------------------------- varlen
+def run_varlen(args, w, rank, world, local_rank):
+    """One step = fa_fwd_varlen + fa_bwd_varlen over a packed batch of
+    sequences of different lengths ([H, T, d] tensors), inputs resident in
+    HBM.  FLOPs: 4·d per visible (query, key) pair of each sequence and query
+    head, 3.5x for forward + backward (the fixed-length convention)."""
+    import torch
+    import torch.distributed as dist
+
+    from exact_attention_104_b200 import binding
+    from exact_attention_104_b200.workloads import make_varlen_inputs
+
+    dev = torch.device("cuda", local_rank)
+    torch.cuda.set_device(dev)
+    binding.lib()
+    stream = torch.cuda.current_stream()
+    q, k, v, do, cu = make_varlen_inputs(w, dev)
+    nseq, T = len(w.lengths), w.T
+    o = torch.empty_like(q)
+    lse = torch.empty(w.Hq, T, dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(q), torch.empty_like(k), torch.empty_like(v)
+    fws = binding.fa_fwd_varlen_workspace_bytes(nseq, w.Hq, w.Hkv, T, w.max_seqlen, w.d)
+    bws = binding.fa_bwd_varlen_workspace_bytes(nseq, w.Hq, w.Hkv, T, w.max_seqlen, w.d)
+    fw = torch.empty(fws, dtype=torch.uint8, device=dev)
+    bw = torch.empty(bws, dtype=torch.uint8, device=dev)
+
+    def step(fprof=None, bprof=None):
+        if fprof is not None:
+            binding.fa_profile_next(*fprof)
+        st = binding.fa_fwd_varlen(q, k, v, o, lse, cu, nseq, w.Hq, w.Hkv, T, w.max_seqlen, w.d, w.causal, w.scale,
+                                   fw, fws, stream)
+        if st:
+            raise binding.FAError(st, "fa_fwd_varlen")
+        if bprof is not None:
+            binding.fa_profile_next(*bprof)
+        st = binding.fa_bwd_varlen(q, k, v, o, lse, do, dq, dk, dv, cu, nseq, w.Hq, w.Hkv, T, w.max_seqlen, w.d,
+                                   w.causal, w.scale, bw, bws, stream)
+        if st:
+            raise binding.FAError(st, "fa_bwd_varlen")
+
+    def barrier():
+        if world > 1:
+            dist.barrier()
+        torch.cuda.synchronize()
+
+    for _ in range(args.warmup):
+        step()
+    torch.cuda.synchronize()
+    if binding.fa_device_status(stream) != 0:
+        raise RuntimeError("device error during warm-up")
+    K = args.steps
+    ev = lambda: torch.cuda.Event(enable_timing=True)  # noqa: E731
+    f_ev = [(ev(), ev()) for _ in range(K)]
+    b_ev = [(ev(), ev()) for _ in range(K)]
+    start, stop = ev(), ev()
+    for e in [x for pair in f_ev + b_ev for x in pair] + [start, stop]:
+        e.record(stream)
+    torch.cuda.synchronize()
+    with ClockSampler(local_rank) as clk:
+        barrier()
+        start.record(stream)
+        for i in range(K):
+            step(f_ev[i], b_ev[i])
+        stop.record(stream)
+        barrier()
+    clocks = clk.summary()
+    if binding.fa_device_status(stream) != 0:
+        raise RuntimeError("device error in the timed region")
+    mo = lambda x: reduce_max_over_ranks(x, world, dev)  # noqa: E731
+    ms_step = mo(start.elapsed_time(stop)) / K
+    ms_fwd = mo(sum(a.elapsed_time(b) for a, b in f_ev) / K)
+    ms_bwd = mo(sum(a.elapsed_time(b) for a, b in b_ev) / K)
+    F = w.fwd_flops()
+    value = 3.5 * F * world / (ms_step * 1e-3) / 1e12
+    peaks = _peaks()
+    bwd_tflops = 2.5 * F / (ms_bwd * 1e-3) / 1e12
+
+    e2e = None
+    if not args.no_e2e:
+        host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
+        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
+        host_cu = cu.cpu().pin_memory()
+
+        def e2e_step():
+            for hsrc, ddst in zip(host_in, (q, k, v, do)):
+                ddst.copy_(hsrc, non_blocking=True)
+            cu.copy_(host_cu, non_blocking=True)
+            step()
+            for hdst, dsrc in zip(host_out, (o, lse, dq, dk, dv)):
+                hdst.copy_(dsrc, non_blocking=True)
+
+        e2e_step()
+        ke = max(3, min(K, 20))
+        barrier()
+        a, b = ev(), ev()
+        a.record(stream)
+        for _ in range(ke):
+            e2e_step()
+        b.record(stream)
+        barrier()
+        ms_e2e = mo(a.elapsed_time(b)) / ke
+        e2e = {"value": 3.5 * F * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
+               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in) + host_cu.numel() * 4,
+               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out), "steps": ke,
+               "overlap": "none: copies and kernels of a step in order on one stream"}
+    line = {
+        "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": w.name, "sequences": len(w.lengths), "T": T, "max_seqlen": w.max_seqlen,
+                   "lengths": list(w.lengths), "Hq": w.Hq, "Hkv": w.Hkv, "d": w.d, "causal": w.causal,
+                   "parallelism": f"dp{world}",
+                   "l2": _l2_note(q, k, v, o, do)},
+        "fwd_tflops": F / (ms_fwd * 1e-3) / 1e12,
+        "bwd_tflops": bwd_tflops,
+        "ms": {"fwd_kernel": ms_fwd, "bwd_main_kernel": ms_bwd},
+        "roofline": {"kernel": "fa_bwd_kernel (packed-batch mode)", "bound": "tensor", "achieved": bwd_tflops,
+                     "peak": peaks["bf16_tflops"], "unit": "TFLOP/s", "frac": bwd_tflops / peaks["bf16_tflops"],
+                     "peak_source": peaks["source"] + " bf16 burst (MEASURED_PEAKS.json)",
+                     "flops_per_launch": 2.5 * F, "ms_per_launch": ms_bwd, "traffic": None},
+        "cpu_baseline": None,
+        "e2e": e2e,
+        "gpu_launches": 6 * K,
+        "clocks": clocks,
+    }
+    if rank == 0:
+        print(json.dumps(line), flush=True)
+
+
 # ------------------------------------------------------------------- e2e
 def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ranks, K):
     """The step through the public C ABI with its data on the host: every step
@@ -691,9 +820,10 @@ def main():
     if args.warmup < 3:
         args.warmup = 3
 
-    from exact_attention_104_b200.workloads import BENCH_WORKLOAD, DECODE_WORKLOADS, WORKLOADS
+    from exact_attention_104_b200.workloads import BENCH_WORKLOAD, DECODE_WORKLOADS, VARLEN_WORKLOADS, WORKLOADS
 
-    names = list(WORKLOADS) + list(DECODE_WORKLOADS) if args.workload == "all" else [args.workload or BENCH_WORKLOAD]
+    names = (list(WORKLOADS) + list(DECODE_WORKLOADS) + list(VARLEN_WORKLOADS) if args.workload == "all"
+             else [args.workload or BENCH_WORKLOAD])
     rank = int(os.environ.get("RANK", "0"))
     world = int(os.environ.get("WORLD_SIZE", "1"))
     local_rank = int(os.environ.get("LOCAL_RANK", "0"))
@@ -702,6 +832,10 @@ def main():
         for name in names:
             if name in DECODE_WORKLOADS:
                 run_decode_reference(args, DECODE_WORKLOADS[name], rank)
+            elif name in VARLEN_WORKLOADS:
+                if rank == 0:
+                    print(json.dumps({"impl": "reference", "workload": name,
+                                      "unavailable": "the reference arm times fixed-length workloads"}), flush=True)
             else:
                 run_reference(args, WORKLOADS[name], rank, world)
         return
@@ -719,6 +853,8 @@ def main():
         for name in names:
             if name in DECODE_WORKLOADS:
                 run_decode(args, DECODE_WORKLOADS[name], rank, world, local_rank)
+            elif name in VARLEN_WORKLOADS:
+                run_varlen(args, VARLEN_WORKLOADS[name], rank, world, local_rank)
             else:
                 run_ours(args, WORKLOADS[name], rank, world, local_rank)
     finally:

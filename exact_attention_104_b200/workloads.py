@@ -235,3 +235,11 @@ def make_varlen_inputs(w: VarlenWorkload, device="cpu"):
     out = [t.to(torch.bfloat16).to(device) for t in (q, k, v, do)]
     cu = torch.tensor(w.cu_seqlens(), dtype=torch.int32, device=device)
     return (*out, cu)
+
+
+# A packed batch for the benchmark: 16 causal sequences of 256 .. 4096 tokens
+# (seeded), 16 heads, d = 128 -- a training batch of documents of mixed length.
+VARLEN_WORKLOADS = {
+    "varlen_16seq_256to4096_h16_d128_causal": VarlenWorkload(
+        "varlen_16seq_256to4096_h16_d128_causal", varlen_lengths(16, 256, 4096, 1009), 16, 16, 128, True, 1009),
+}

@@ -8,8 +8,9 @@ fa_bwd_varlen) on the GPU, through the C ABI.
   a varlen unit runs the same per-tile arithmetic in the same order as the
   fixed-length kernels on that sequence, so O, LSE, dK and dV are identical
   bit for bit; dQ differs only in the order of its fp32 reduce-adds.
-* Lengths from 1 to 5000 (GQA 4:1, d = 128), sampled rows of every sequence
-  against the oracle.
+* Lengths from 1 to 5000 (GQA 4:1, d = 128), and the benchmark's packed
+  batch (16 causal sequences of 256 to 4096 tokens, 16 heads), sampled rows
+  of every sequence against the oracle.
 * cu_seqlens that breaks its rules: the call computes nothing, leaves the
   outputs untouched and fa_device_status reports FA_ERR_INVALID_ARG."""
 
@@ -20,7 +21,7 @@ import torch
 import oracle
 from exact_attention_104_b200 import (attention_backward, attention_backward_varlen, attention_forward,
                                       attention_forward_varlen, binding)
-from exact_attention_104_b200.workloads import VarlenWorkload, make_varlen_inputs, varlen_lengths
+from exact_attention_104_b200.workloads import VARLEN_WORKLOADS, VarlenWorkload, make_varlen_inputs, varlen_lengths
 
 from _parity import GRAD_REL_FRO, assert_within_tolerance, f64, rel_fro
 
@@ -82,28 +83,31 @@ def test_varlen_equals_one_call_per_sequence(d, causal):
         assert rel_fro(f64(dq[0]), f64(g["dq"][:, lo:hi])) <= 1e-3, (b, "dq")
 
 
-@pytest.mark.parametrize("causal", [False, True])
-def test_varlen_lengths_1_to_5000_sampled(causal):
-    lengths = varlen_lengths(10, 1, 5000, 77 + causal, include=(1, 5000, 129))
-    w = VarlenWorkload("mixed_1_5000", lengths, 8, 2, 128, causal, 3100 + causal)
-    g = _run(w)
+def _sampled_errors(w, g, seed, rows_per_seq=12):
+    """Sampled rows of every sequence (its first and last rows, the rows
+    around the first tile edge, the last tile's first row and random ones),
+    on the first and last kv head and all their query heads, against the
+    oracle's row-wise forward and sampled backward."""
     cu = w.cu_seqlens()
-    rng = np.random.default_rng(5 + causal)
+    rng = np.random.default_rng(seed)
     o_abs, lse_abs, dq_p, dk_p, dv_p = [], [], [], [], []
-    for b, n in enumerate(lengths):
+    for b, n in enumerate(w.lengths):
+        if n == 0:
+            continue
         lo = cu[b]
         fixed = {0, n - 1, 127, 128, (n - 1) // 128 * 128}
-        rows = np.array(sorted({r for r in fixed if 0 <= r < n} | set(rng.choice(n, min(n, 12), replace=False))))
+        rows = np.array(sorted({r for r in fixed if 0 <= r < n} |
+                               set(rng.choice(n, min(n, rows_per_seq), replace=False))))
         for g_kv in sorted({0, w.Hkv - 1}):
             kh, vh = f64(g["k"][g_kv, lo:lo + n]), f64(g["v"][g_kv, lo:lo + n])
             heads = range(g_kv * w.G, (g_kv + 1) * w.G)
             qh = np.stack([f64(g["q"][h, lo:lo + n]) for h in heads])
             doh = np.stack([f64(g["do"][h, lo:lo + n]) for h in heads])
             for i, h in enumerate(heads):
-                o_r, lse_r, _ = oracle.head_forward_rows(qh[i], kh, vh, w.scale, causal, rows)
+                o_r, lse_r, _ = oracle.head_forward_rows(qh[i], kh, vh, w.scale, w.causal, rows)
                 o_abs.append(np.abs(f64(g["o"][h, lo:lo + n][rows]) - o_r))
                 lse_abs.append(np.abs(f64(g["lse"][h, lo:lo + n][rows]) - lse_r))
-            dq_r, dk_r, dv_r = oracle.head_backward_sampled(qh, kh, vh, doh, w.scale, causal, rows, rows)
+            dq_r, dk_r, dv_r = oracle.head_backward_sampled(qh, kh, vh, doh, w.scale, w.causal, rows, rows)
             for i, h in enumerate(heads):
                 dq_p.append((f64(g["dq"][h, lo:lo + n][rows]), dq_r[i]))
             dk_p.append((f64(g["dk"][g_kv, lo:lo + n][rows]), dk_r))
@@ -114,7 +118,24 @@ def test_varlen_lengths_1_to_5000_sampled(causal):
     for name, pairs in (("dq", dq_p), ("dk", dk_p), ("dv", dv_p)):
         err[name] = rel_fro(np.concatenate([p[0].ravel() for p in pairs]),
                             np.concatenate([p[1].ravel() for p in pairs]))
+    return err
+
+
+@pytest.mark.parametrize("causal", [False, True])
+def test_varlen_lengths_1_to_5000_sampled(causal):
+    lengths = varlen_lengths(10, 1, 5000, 77 + causal, include=(1, 5000, 129))
+    w = VarlenWorkload("mixed_1_5000", lengths, 8, 2, 128, causal, 3100 + causal)
+    err = _sampled_errors(w, _run(w), 5 + causal)
     print(lengths, err)
+    assert_within_tolerance(err)
+
+
+@pytest.mark.parametrize("name", list(VARLEN_WORKLOADS))
+def test_varlen_bench_workload_sampled(name):
+    """The packed batch the benchmark times, in the same call sequence."""
+    w = VARLEN_WORKLOADS[name]
+    err = _sampled_errors(w, _run(w), 11, rows_per_seq=6)
+    print(w.name, err)
     assert_within_tolerance(err)
 
 
