@@ -44,6 +44,13 @@ struct BwdCfg {
   static constexpr int Q_BYTES = BR * D * 2;
   static constexpr int NSTAGE = (D == 64) ? 4 : (D == 128 ? 3 : 1);
   static constexpr int LA = NSTAGE >= 2 ? 2 : 1;  // Sᵀ lookahead in steps
+  // d = 256 (one stage): a step's Q and dO tiles load in two halves.  Half A
+  // is the two 64-column panels outside the CTA's own output columns (read
+  // only by Sᵀ and dPᵀ, so it is free once dPᵀ is done); half B is the CTA's
+  // own two panels and the row statistics (read until the dK product).  The
+  // next step's half A loads while this step's softmax and gradient products
+  // run, and Sᵀ / dPᵀ consume half A before half B.
+  static constexpr bool HALVES = (NSTAGE == 1 && D == 256);
   static constexpr int K_OFF = 0;
   static constexpr int V_OFF = KV_BYTES;
   static constexpr int DS_OFF = 2 * KV_BYTES;   // dSᵀ: 128 key rows x 64 queries (bf16), 16 KB
@@ -73,7 +80,12 @@ struct BwdCfg {
   static constexpr int B_UNITFULL = B_DVFREE + 1;   // + {0,1}: next unit index published
   static constexpr int B_UNITEMPTY = B_UNITFULL + 2; // + {0,1}: read by all nine consumer warps
   static constexpr int B_DRAIN = B_UNITEMPTY + 2;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_HAFULL = B_DRAIN + 1;    // half A of a step's Q and dO loaded
+  static constexpr int B_HAEMPTY = B_HAFULL + 1;  // half A read by Sᵀ and dPᵀ
+  static constexpr int B_QBFULL = B_HAEMPTY + 1;  // half B of Q and the row statistics loaded
+  static constexpr int B_DOBFULL = B_QBFULL + 1;  // half B of dO loaded
+  static constexpr int B_HBEMPTY = B_DOBFULL + 1; // half B read by the dV and dK products
+  static constexpr int NBAR = B_HBEMPTY + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int UNIT_OFF = MISC_OFF + 16;   // two unit-index slots
   static constexpr int SMEM_BYTES = UNIT_OFF + 16 + 1024;
@@ -340,6 +352,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       mbar_init(BAR(C::B_UNITEMPTY + i), 9);  // MMA warp, four compute warps, four drain warps
     }
     mbar_init(BAR(C::B_DRAIN), 1);
+    for (int i = C::B_HAFULL; i <= C::B_HBEMPTY; ++i) mbar_init(BAR(i), 1);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -388,6 +401,35 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // Q, dO, lse2, D of step s of this unit into its stage
         auto load_q = [&](int s) -> bool {
           const int g = gs + s;
+          if constexpr (C::HALVES) {
+            const int q_row = bwd_qrow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);
+            const int q_row_p = bwd_qprow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);
+            const int own = 2 * u.dh, oth = 2 - own;
+            if (!mbar_wait(BAR(C::B_HAEMPTY), (g & 1) ^ 1, wc, 40)) return false;
+            // a unit's first step: the previous step (another unit, perhaps with
+            // the other output half) may still read these panels as its half B
+            if (s == 0 && !mbar_wait(BAR(C::B_HBEMPTY), (g & 1) ^ 1, wc, 45)) return false;
+            mbar_expect_tx(BAR(C::B_HAFULL), 4 * C::Q_PANEL);
+#pragma unroll
+            for (int j = 0; j < 2; ++j) {
+              const int pn = oth + j;
+              tma_load_2d(sbase + C::Q_OFF + pn * C::Q_PANEL, &tmQ, BAR(C::B_HAFULL), pn * 64, q_row);
+              tma_load_2d(sbase + C::DO_OFF + pn * C::Q_PANEL, &tmDO, BAR(C::B_HAFULL), pn * 64, q_row);
+            }
+            if (!mbar_wait(BAR(C::B_HBEMPTY), (g & 1) ^ 1, wc, 41)) return false;
+            mbar_expect_tx(BAR(C::B_QBFULL), 2 * C::Q_PANEL + 512);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d(sbase + C::Q_OFF + (own + j) * C::Q_PANEL, &tmQ, BAR(C::B_QBFULL), (own + j) * 64, q_row);
+            bulk_load(sbase + C::LS_OFF, p.lse2 + q_row_p, 256, BAR(C::B_QBFULL));
+            bulk_load(sbase + C::LS_OFF + 256, p.dvec + q_row_p, 256, BAR(C::B_QBFULL));
+            mbar_expect_tx(BAR(C::B_DOBFULL), 2 * C::Q_PANEL);
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+              tma_load_2d(sbase + C::DO_OFF + (own + j) * C::Q_PANEL, &tmDO, BAR(C::B_DOBFULL), (own + j) * 64,
+                          q_row);
+            return true;
+          }
           const int st = g % C::NSTAGE;
           if (!mbar_wait(BAR(C::B_QEMPTY + st), ((g / C::NSTAGE) & 1) ^ 1, wc, 11)) return false;
           const int q_row = bwd_qrow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);
@@ -473,44 +515,90 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         };
         if (!mbar_wait_warp(BAR(C::B_KVFULL), uc & 1, wc, 12)) { ok = false; break; }
         tc_fence_after();
-        for (int k = 0; k < C::LA && k < n && ok; ++k) {
-          ok = wait_q(gs + k);
-          if (!ok) break;
-          issue_xt(dK_k, q_off(gs + k), tbase + C::ST_COL + 64 * ((gs + k) & 1));
-          tc_commit_w(BAR(C::B_SFULL + ((gs + k) & 1)));
-        }
-        if (!ok) break;
-        issue_xt(dV_k, do_off(gs), tbase + C::DP_COL);
-        tc_commit_w(BAR(C::B_DPFULL));
-        for (int s = 0; s < n && ok; ++s) {
-          const int g = gs + s;
-          if (!mbar_wait_warp(BAR(C::B_PFULL + (g & 1)), (g >> 1) & 1, wc, 14)) { ok = false; break; }
-          // the previous unit's dV must have been read out before it is overwritten
-          if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DVFREE), (uc - 1) & 1, wc, 19)) { ok = false; break; }
-          tc_fence_after();
-          issue_acc(tbase + C::ST_COL + 64 * (g & 1), sdesc_add(dDO_mn, stage_bytes(g)), tbase + C::DV_COL, s == 0);
-          if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
-          if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
-          tc_fence_after();
-          issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(g)), tbase + C::DK_COL, s == 0);
-          tc_commit_w(BAR(C::B_QEMPTY + g % C::NSTAGE));
-          if (g > 0) {
-            if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
+        if constexpr (C::HALVES) {
+          const int own = 2 * u.dh, oth = 2 - own;
+          // Sᵀ or dPᵀ over the two 64-column panels pn0, pn0 + 1 of the head dimension
+          auto issue_xt_half = [&](uint64_t da0, uint64_t db0, uint32_t dtm, int pn0, bool first) {
+#pragma unroll
+            for (int j = 0; j < 2; ++j)
+#pragma unroll
+              for (int kk = 0; kk < 4; ++kk)
+                mma_ss_w(dtm, sdesc_add(da0, (uint32_t)(pn0 + j) * C::KV_PANEL + kk * 32),
+                         sdesc_add(db0, (uint32_t)(pn0 + j) * C::Q_PANEL + kk * 32), C::IDESC_ST,
+                         (first && j == 0 && kk == 0) ? 0u : 1u);
+          };
+          for (int s = 0; s < n && ok; ++s) {
+            const int g = gs + s;
+            const uint32_t st_t = tbase + C::ST_COL + 64 * (g & 1);
+            if (!mbar_wait_warp(BAR(C::B_HAFULL), g & 1, wc, 42)) { ok = false; break; }
             tc_fence_after();
-          }
-          issue_dq();
-          tc_commit_w(BAR(C::B_DQFULL));
-          // dPᵀ of the next step first: the compute warps are waiting for it
-          if (s + 1 < n) {
-            if (C::LA == 1 && !wait_q(g + 1)) { ok = false; break; }
-            issue_xt(dV_k, do_off(g + 1), tbase + C::DP_COL);
+            issue_xt_half(dK_k, dQ_k, st_t, oth, true);
+            if (!mbar_wait_warp(BAR(C::B_QBFULL), g & 1, wc, 43)) { ok = false; break; }
+            tc_fence_after();
+            issue_xt_half(dK_k, dQ_k, st_t, own, false);
+            tc_commit_w(BAR(C::B_SFULL + (g & 1)));
+            issue_xt_half(dV_k, dDO_k, tbase + C::DP_COL, oth, true);
+            if (!mbar_wait_warp(BAR(C::B_DOBFULL), g & 1, wc, 44)) { ok = false; break; }
+            tc_fence_after();
+            issue_xt_half(dV_k, dDO_k, tbase + C::DP_COL, own, false);
             tc_commit_w(BAR(C::B_DPFULL));
+            tc_commit_w(BAR(C::B_HAEMPTY));
+            if (!mbar_wait_warp(BAR(C::B_PFULL + (g & 1)), (g >> 1) & 1, wc, 14)) { ok = false; break; }
+            if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DVFREE), (uc - 1) & 1, wc, 19)) { ok = false; break; }
+            tc_fence_after();
+            issue_acc(st_t, dDO_mn, tbase + C::DV_COL, s == 0);
+            if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
+            if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
+            tc_fence_after();
+            issue_acc(tbase + C::DP_COL, dQ_mn, tbase + C::DK_COL, s == 0);
+            tc_commit_w(BAR(C::B_HBEMPTY));
+            if (g > 0) {
+              if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_dq();
+            tc_commit_w(BAR(C::B_DQFULL));
           }
-          if (s + C::LA < n) {
-            const int g2 = g + C::LA;
-            if (C::LA > 1 && !wait_q(g2)) { ok = false; break; }
-            issue_xt(dK_k, q_off(g2), tbase + C::ST_COL + 64 * (g2 & 1));
-            tc_commit_w(BAR(C::B_SFULL + (g2 & 1)));
+        } else {
+          for (int k = 0; k < C::LA && k < n && ok; ++k) {
+            ok = wait_q(gs + k);
+            if (!ok) break;
+            issue_xt(dK_k, q_off(gs + k), tbase + C::ST_COL + 64 * ((gs + k) & 1));
+            tc_commit_w(BAR(C::B_SFULL + ((gs + k) & 1)));
+          }
+          if (!ok) break;
+          issue_xt(dV_k, do_off(gs), tbase + C::DP_COL);
+          tc_commit_w(BAR(C::B_DPFULL));
+          for (int s = 0; s < n && ok; ++s) {
+            const int g = gs + s;
+            if (!mbar_wait_warp(BAR(C::B_PFULL + (g & 1)), (g >> 1) & 1, wc, 14)) { ok = false; break; }
+            // the previous unit's dV must have been read out before it is overwritten
+            if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DVFREE), (uc - 1) & 1, wc, 19)) { ok = false; break; }
+            tc_fence_after();
+            issue_acc(tbase + C::ST_COL + 64 * (g & 1), sdesc_add(dDO_mn, stage_bytes(g)), tbase + C::DV_COL, s == 0);
+            if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
+            if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
+            tc_fence_after();
+            issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(g)), tbase + C::DK_COL, s == 0);
+            tc_commit_w(BAR(C::B_QEMPTY + g % C::NSTAGE));
+            if (g > 0) {
+              if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
+              tc_fence_after();
+            }
+            issue_dq();
+            tc_commit_w(BAR(C::B_DQFULL));
+            // dPᵀ of the next step first: the compute warps are waiting for it
+            if (s + 1 < n) {
+              if (C::LA == 1 && !wait_q(g + 1)) { ok = false; break; }
+              issue_xt(dV_k, do_off(g + 1), tbase + C::DP_COL);
+              tc_commit_w(BAR(C::B_DPFULL));
+            }
+            if (s + C::LA < n) {
+              const int g2 = g + C::LA;
+              if (C::LA > 1 && !wait_q(g2)) { ok = false; break; }
+              issue_xt(dK_k, q_off(g2), tbase + C::ST_COL + 64 * (g2 & 1));
+              tc_commit_w(BAR(C::B_SFULL + (g2 & 1)));
+            }
           }
         }
         if (!ok) break;
@@ -543,7 +631,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int g = gs + s;
         const int st = g % C::NSTAGE;
         const int q0 = step_q0(u, s);
-        if (!mbar_wait_warp(BAR(C::B_QFULL + st), (g / C::NSTAGE) & 1, wc, 21)) { ok = false; break; }
+        const uint32_t stats_bar = C::HALVES ? BAR(C::B_QBFULL) : BAR(C::B_QFULL + st);
+        if (!mbar_wait_warp(stats_bar, (g / C::NSTAGE) & 1, wc, 21)) { ok = false; break; }
         if (!mbar_wait_warp(BAR(C::B_SFULL + (g & 1)), (g >> 1) & 1, wc, 22)) { ok = false; break; }
         tc_fence_after();
         const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512);

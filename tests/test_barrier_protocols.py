@@ -74,15 +74,24 @@ def _run(gens, engines, rnd, max_steps=20_000_000):
 
 
 # ---------------------------------------------------------------- backward
-def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
+def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halves=False):
     """fa_bwd_kernel: ``n_ctas`` persistent CTAs claim units (``unit_len[i]`` query
     steps each) from one counter.  Roles per CTA: the producer (lane 0 of warp
     0), the MMA warp, four compute warps and four drain warps.  ``lookahead`` is
-    how many Sᵀ products run ahead (2 with several Q/dO stages, 1 with one)."""
+    how many Sᵀ products run ahead (2 with several Q/dO stages, 1 with one).
+
+    ``halves`` models the one-stage layout of d = 256, where a step's Q and dO
+    tiles are loaded in two halves: half A (the head-dimension panels outside
+    the CTA's own output columns, last read by dPᵀ) and half B (the CTA's own
+    panels and the per-row statistics, last read by the dK product); half B's
+    Q and dO complete on separate barriers.  Each step issues Sᵀ and dPᵀ over
+    half A, then over half B, and then dV, dK, dQᵀ."""
     rnd = random.Random(seed)
     counter = [0]
     done_units = []
     gens, engines = {}, {}
+    # with halves, each unit owns one half of the output columns, chosen at random
+    unit_dh = [rnd.randrange(2) for _ in unit_len]
 
     def make_cta(c):
         bars = {}
@@ -93,6 +102,8 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
         for i in range(n_stage):
             bars["QFULL", i] = _Bar(1)
             bars["QEMPTY", i] = _Bar(1)
+        for nm in ("HAFULL", "HAEMPTY", "QBFULL", "DOBFULL", "HBEMPTY"):
+            bars[nm] = _Bar(1)
         for i in range(2):
             bars["SFULL", i] = _Bar(1)
             bars["PFULL", i] = _Bar(4)
@@ -106,16 +117,23 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
         slot_readers = [set(), set()]
         kv_readers, stage_readers, acc_writers = {}, {}, {}
         acc_read = {}               # (kind, uc) -> warps that read it out
+        half_readers = {}           # (panel pair, g) -> products reading those panels of step g
+        step_dh = {}                # g -> the output-column half of step g's unit
+        stats_read = {}             # g -> compute warps done with step g's row statistics
         prod_id = [0]
 
         def issue(kind, uc, g):
             prod_id[0] += 1
             i = prod_id[0]
             tc.append(("mma", i))
-            if kind in ("S", "dP", "dQ"):
+            if kind in ("S", "dP", "dQ", "S_A", "S_B", "dP_A", "dP_B"):
                 kv_readers.setdefault(uc, set()).add(i)
             if kind in ("S", "dP", "dV", "dK"):
                 stage_readers.setdefault(g, set()).add(i)
+            if kind in ("S_A", "dP_A"):
+                half_readers.setdefault((1 - step_dh[g], g), set()).add(i)
+            if kind in ("S_B", "dP_B") or (halves and kind in ("dV", "dK")):
+                half_readers.setdefault((step_dh[g], g), set()).add(i)
             if kind in ("dV", "dK"):
                 acc_writers.setdefault(uc, set()).add(i)
                 if uc > 0:
@@ -149,14 +167,38 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
                 if idx >= len(unit_len):
                     return
                 n = unit_len[idx]
+                dh = unit_dh[idx]
+
+                def load_halves(s):
+                    # the unit's dh picks which panel pair is half A (1 - dh) and half B (dh)
+                    g = gs + s
+                    step_dh[g] = dh
+                    if g >= 1:
+                        yield from wait("HAEMPTY", g - 1)
+                        if s == 0 and mistake != "no_unit_start_half_b_wait":
+                            # the previous unit's half B may be this half A
+                            yield from wait("HBEMPTY", g - 1)
+                        assert half_readers.get((1 - dh, g - 1), set()) <= completed, \
+                            f"panels {1 - dh} of step {g} reused"
+                    tma.append(("HAFULL", ("QA", g)))
+                    if g >= 1:
+                        if mistake != "no_half_b_empty_wait":
+                            yield from wait("HBEMPTY", g - 1)
+                        assert half_readers.get((dh, g - 1), set()) <= completed, f"panels {dh} of step {g} reused"
+                        assert stats_read.get(g - 1, 0) == 4, f"statistics of step {g} overwritten while read"
+                    tma.append(("QBFULL", ("QB", g)))
+                    tma.append(("DOBFULL", ("DOB", g)))
 
                 def load_q(s):
+                    if halves:
+                        yield from load_halves(s)
+                        return
                     g = gs + s
                     if g >= n_stage:
                         yield from wait(("QEMPTY", g % n_stage), g // n_stage - 1)
                         assert stage_readers.get(g - n_stage, set()) <= completed, f"stage of step {g} reused"
                     tma.append((("QFULL", g % n_stage), ("Q", g)))
-                pre = min(n_stage, n)
+                pre = min(1 if halves else n_stage, n)
                 for s in range(pre):
                     yield from load_q(s)
                 if uc > 0:
@@ -181,6 +223,41 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
                 def wait_q(g):
                     yield from wait(("QFULL", g % n_stage), g // n_stage)
                     assert ("Q", g) in loaded
+                if halves:
+                    for s in range(n):
+                        g = gs + s
+                        yield from wait("HAFULL", g)
+                        assert ("QA", g) in loaded
+                        issue("S_A", uc, g)
+                        yield from wait("QBFULL", g)
+                        assert ("QB", g) in loaded
+                        issue("S_B", uc, g)
+                        commit(("SFULL", g & 1))
+                        issue("dP_A", uc, g)
+                        yield from wait("DOBFULL", g)
+                        assert ("DOB", g) in loaded
+                        issue("dP_B", uc, g)
+                        commit("DPFULL")
+                        commit("HAEMPTY")
+                        yield from wait(("PFULL", g & 1), g >> 1)
+                        if s == 0 and uc > 0 and mistake != "no_dvfree_wait":
+                            yield from wait("DVFREE", uc - 1)
+                        issue("dV", uc, g)
+                        yield from wait("DSFULL", g)
+                        if s == 0 and uc > 0:
+                            yield from wait("DKFREE", uc - 1)
+                        issue("dK", uc, g)
+                        commit("HBEMPTY")
+                        if g > 0:
+                            yield from wait("DQEMPTY", g - 1)
+                        issue("dQ", uc, g)
+                        commit("DQFULL")
+                    commit("ACC")
+                    commit("KVEMPTY")
+                    done_units.append(idx)
+                    gs += n
+                    uc += 1
+                    continue
                 for k in range(min(lookahead, n)):
                     yield from wait_q(gs + k)
                     issue("S", uc, gs + k)
@@ -230,7 +307,11 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
                 for s in range(n):
                     g = gs + s
                     if kind == "dK":
-                        yield from wait(("QFULL", g % n_stage), g // n_stage)
+                        if halves:
+                            yield from wait("QBFULL", g)
+                            assert ("QB", g) in loaded
+                        else:
+                            yield from wait(("QFULL", g % n_stage), g // n_stage)
                         yield from wait(("SFULL", g & 1), g >> 1)
                         yield
                         bars["PFULL", g & 1].arrive()
@@ -238,6 +319,7 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None):
                         if g > 0:
                             yield from wait("DQFULL", g - 1)
                         yield
+                        stats_read[g] = stats_read.get(g, 0) + 1
                         bars["DSFULL"].arrive()
                     else:
                         yield from wait("DQFULL", g)
@@ -289,12 +371,30 @@ def test_backward_protocol(n_stage, lookahead, n_ctas):
             simulate_bwd(units, n_ctas, n_stage, lookahead, seed)
 
 
+@pytest.mark.parametrize("n_ctas", [1, 3])
+def test_backward_protocol_half_stages(n_ctas):
+    for units in BWD_UNITS:
+        for seed in range(4):
+            simulate_bwd(units, n_ctas, 1, 1, seed, halves=True)
+
+
 @pytest.mark.parametrize("mistake", ["no_unit_empty_wait", "no_dvfree_wait"])
 def test_backward_model_catches_a_missing_wait(mistake):
     caught = 0
     for seed in range(40):
         try:
             simulate_bwd([1, 1, 1, 1, 1, 1], 2, 3, 2, seed, mistake)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+@pytest.mark.parametrize("mistake", ["no_half_b_empty_wait", "no_unit_start_half_b_wait"])
+def test_backward_half_stage_model_catches_a_missing_wait(mistake):
+    caught = 0
+    for seed in range(40):
+        try:
+            simulate_bwd([2, 3, 1, 2, 1, 2], 2, 1, 1, seed, mistake, halves=True)
         except AssertionError:
             caught += 1
     assert caught > 0
