@@ -8,17 +8,21 @@
 // the next item's Q/K loads and first QKᵀ overlap the running item:
 //   * each query tile has its own Q buffer; it is reloaded as soon as the
 //     tile's last QKᵀ of the item has completed;
-//   * the MMA warp issues the next item's first QKᵀ for a tile right after the
-//     tile's last PV product, so the tensor pipe is fed while the softmax
-//     warpgroup writes the finished tile out;
+//   * the next item's first QKᵀ for a tile is issued right after the tile's
+//     last PV product, so the tensor pipe is fed while the softmax warpgroup
+//     writes the finished tile out;
+//   * at d = 64, P has TMEM columns of its own and each tile has its own MMA
+//     warp, so a tile's next QKᵀ is issued as soon as its softmax has read S;
 //   * with a causal mask the second tile of a pair sees one more K/V block
 //     than the first (its diagonal block).  That block is processed first, so
 //     both tiles finish an item in the same iteration;
 //   * causal items are ordered heaviest first, dealt to CTAs in alternating
 //     directions round by round; non-causal items are ordered head by head, so
 //     concurrently running CTAs share K/V tiles in L2.
-// Roles: warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 2-3 idle,
-// warps 4-7 / 8-11 softmax of query tile 0 / 1 (thread = query row).
+// Roles: warp 0 TMA producer, warp 1 MMA issuer and TMEM owner (at d = 64
+// the MMA issuer of query tile 0, warp 2 that of tile 1), the other control
+// warps idle, warps 4-7 / 8-11 softmax of query tile 0 / 1 (thread = query
+// row).
 #pragma once
 
 #include "fa_fwd.cuh"
@@ -46,12 +50,26 @@ struct FwdPCfg {
   static constexpr int B_PFULL2 = B_PFULL + 2;       // + tile: P keys 64..127 in TMEM
   static constexpr int B_ODONE = B_PFULL2 + 2;       // + tile
   static constexpr int B_DRAIN = B_ODONE + 2;
-  static constexpr int NBAR = B_DRAIN + 1;
+  static constexpr int B_SFREE = B_DRAIN + 1;        // + tile: S read out of TMEM (SEP_P)
+  static constexpr int NBAR = B_SFREE + 2;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int SMEM_BYTES = MISC_OFF + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int S_COL = 0;    // S of tile t at S_COL + 128·t (P over its first 64 columns)
+  static constexpr int S_COL = 0;    // S of tile t at S_COL + 128·t
   static constexpr int O_COL = 256;  // O of tile t at O_COL + t·D
+  // P (bf16, 64 columns for 128 keys): over the first 64 columns of its S
+  // buffer, or, at d = 64 where TMEM has room, in columns of its own
+  // (SEP_P).  Then a tile's next QKᵀ need not follow the PV that reads P: it
+  // is issued as soon as the softmax has loaded S into registers.
+  static constexpr bool SEP_P = (D == 64);
+  static constexpr int P_COL = O_COL + 2 * D;  // SEP_P: P of tile t at P_COL + 64·t
+  // One MMA warp per query tile (warps 1, 2) goes with SEP_P: each tile's
+  // next QKᵀ is issued as soon as its softmax has read S, whatever the other
+  // tile is doing.  Without SEP_P one MMA warp issues both tiles' products in
+  // strict alternation, which keeps the two softmax warpgroups half a block
+  // apart (measured faster at d = 128 than two independent issuers).
+  static constexpr bool PER_TILE = SEP_P;
+  static constexpr int MMA_WARPS = PER_TILE ? 2 : 1;
   static constexpr uint32_t IDESC_S = B::IDESC_S;
   static constexpr uint32_t IDESC_PV = B::IDESC_PV;
   // Register split (setmaxnreg): the item bookkeeping of the producer and MMA
@@ -70,6 +88,7 @@ struct FwdPCfg {
   static constexpr int kPolyPairs = (D == 64) ? 4 : 0;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(O_COL + 2 * D <= TMEM_COLS, "TMEM budget");
+  static_assert(!SEP_P || P_COL + 128 <= TMEM_COLS, "TMEM budget (separate P)");
 };
 
 struct FwdPParams {
@@ -192,12 +211,13 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       mbar_init(BAR(C::B_PFULL + t), 4);
       mbar_init(BAR(C::B_PFULL2 + t), 4);
       mbar_init(BAR(C::B_ODONE + t), 1);
+      mbar_init(BAR(C::B_SFREE + t), 4);
     }
     for (int i = 0; i < C::NSLOT; ++i) {
       mbar_init(BAR(C::B_KVFULL + i), 1);
-      mbar_init(BAR(C::B_KVEMPTY + i), 1);
+      mbar_init(BAR(C::B_KVEMPTY + i), C::MMA_WARPS);  // released by every MMA warp
     }
-    mbar_init(BAR(C::B_DRAIN), 1);
+    mbar_init(BAR(C::B_DRAIN), C::MMA_WARPS);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -258,119 +278,252 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         useq += 2 * w.nit;
       }
     }
-  } else if (warp == 1) {
-    // ---------------------------------------------------------- MMA issuer
-    // (the whole warp runs this role; one elected lane issues each instruction)
-    setmaxnreg_dec<C::CTRL_REGS>();
-    bool ok = true;
-    int waited = -1;           // K/V units whose arrival has been observed, in load order
-    int qfull_seen[2] = {0, 0};
-    int p_seen[2] = {0, 0};    // P hand-overs consumed per tile
-    // Wait for every unit up to U in load order: a unit's slot barrier is only
-    // ever waited on for its current fill, so the parity test is unambiguous.
-    auto wait_upto = [&](int U) -> bool {
-      while (waited < U) {
-        ++waited;
-#pragma unroll
+  } else if (warp == 1 || (C::PER_TILE && warp == 2)) {
+    if constexpr (C::PER_TILE) {
+      // ------------------------------------------------ MMA issuers, one per tile
+      // Warp 1 + t issues query tile t's products only (the whole warp runs the
+      // role; one elected lane issues each instruction).  Both warps walk every
+      // K/V unit of their items in load order and release each one (the slot's
+      // empty barrier counts two arrivals); a unit the tile does not read (the
+      // other tile's diagonal block, an item without tile 1) is released once
+      // this fill of its slot has landed, so that no release can count towards
+      // the slot's previous fill.
+      setmaxnreg_dec<C::CTRL_REGS>();
+      const int t = warp - 1;
+      bool ok = true;
+      int qfull_seen = 0;
+      int p_seen = 0;  // P hand-overs consumed
+      int s_cnt = 0;   // QKᵀ products issued into this tile's S buffer
+      // Wait for the fill of unit U: a warp never lags a full fill behind a
+      // slot, because the slot is refilled only after both warps released it.
+      auto wait_unit = [&](int U) -> bool {
+  #pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
-          const int seq = waited * C::NCH + c;
+          const int seq = U * C::NCH + c;
           if (!mbar_wait_warp(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 43)) return false;
         }
-      }
-      tc_fence_after();
-      return true;
-    };
-    auto release = [&](int U) {
-#pragma unroll
-      for (int c = 0; c < C::NCH; ++c) tc_commit_w(BAR(C::B_KVEMPTY + (U * C::NCH + c) % C::NSLOT));
-    };
-    const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
-    const uint64_t dKV_k = sdesc_sw128(sbase + C::KV_OFF, 16, 1024);
-    const uint64_t dKV_mn = sdesc_sw128(sbase + C::KV_OFF, C::PANEL, 1024);
-    // S_t = Q_t · Kᵀ for iteration jj of item w (its K unit is base + 2·jj)
-    auto issue_s = [&](int t, const FwdItem& w, int base, int jj) -> bool {
-      if (jj == w.first(t)) {
-        if (!mbar_wait_warp(BAR(C::B_QFULL + t), qfull_seen[t] & 1, wc, 44)) return false;
-        ++qfull_seen[t];
-      }
-      const int U = base + 2 * jj;
-      if (!wait_upto(U)) return false;
-      const uint64_t da0 = sdesc_add(dQ_k, t * C::Q_BYTES);
-      uint64_t db0[C::NCH];
-#pragma unroll
-      for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
-#pragma unroll
-      for (int kk = 0; kk < D / 16; ++kk) {
-        const int col = kk * 16;
-        mma_ss_w(tbase + C::S_COL + 128 * t, sdesc_add(da0, (kk >> 2) * C::PANEL + (kk & 3) * 32),
-                 sdesc_add(db0[col / C::CH], ((col % C::CH) / 64) * C::PANEL + (kk & 3) * 32), C::IDESC_S,
-                 kk > 0 ? 1u : 0u);
-      }
-      tc_commit_w(BAR(C::B_SFULL + t));
-      if (jj == w.nit - 1) tc_commit_w(BAR(C::B_QEMPTY + t));  // last QKᵀ of this tile in the item
-      if (t == 1 || w.n1 == 0) release(U);                      // last reader of this K unit
-      return true;
-    };
-    // O_t (+)= P_t · V for one 64-key half of the P tile
-    auto issue_pv = [&](int t, int U, bool first, int half) {
-#pragma unroll
-      for (int c = 0; c < C::NCH; ++c) {
-        const uint64_t db0 = sdesc_add(dKV_mn, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
-#pragma unroll
-        for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
-          mma_ts_w(tbase + C::O_COL + t * D + c * C::CH, tbase + C::S_COL + 128 * t + kk * 8,
-                   sdesc_add(db0, kk * 2048), C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
-      }
-    };
+        tc_fence_after();
+        return true;
+      };
+      auto release = [&](int U) {
+  #pragma unroll
+        for (int c = 0; c < C::NCH; ++c) tc_commit_w(BAR(C::B_KVEMPTY + (U * C::NCH + c) % C::NSLOT));
+      };
+      const uint64_t dQ_t = sdesc_add(sdesc_sw128(sbase + C::Q_OFF, 16, 1024), t * C::Q_BYTES);
+      const uint64_t dKV_k = sdesc_sw128(sbase + C::KV_OFF, 16, 1024);
+      const uint64_t dKV_mn = sdesc_sw128(sbase + C::KV_OFF, C::PANEL, 1024);
+      const uint32_t s_tm = tbase + C::S_COL + 128 * t;
+      const uint32_t p_tm = tbase + (C::SEP_P ? C::P_COL + 64 * t : C::S_COL + 128 * t);
+      const uint32_t o_tm = tbase + C::O_COL + t * D;
+      // S_t = Q_t · Kᵀ for iteration jj of item w (its K unit is base + 2·jj)
+      auto issue_s = [&](const FwdItem& w, int base, int jj) -> bool {
+        // SEP_P: the softmax must have read the previous S out of the buffer
+        // (otherwise the PV issued before this QKᵀ orders it after that read)
+        if (C::SEP_P && s_cnt > 0) {
+          if (!mbar_wait_warp(BAR(C::B_SFREE + t), (s_cnt - 1) & 1, wc, 51)) return false;
+          tc_fence_after();
+        }
+        ++s_cnt;
+        if (jj == w.first(t)) {
+          if (!mbar_wait_warp(BAR(C::B_QFULL + t), qfull_seen & 1, wc, 44)) return false;
+          ++qfull_seen;
+        }
+        const int U = base + 2 * jj;
+        if (!wait_unit(U)) return false;
+        uint64_t db0[C::NCH];
+  #pragma unroll
+        for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
+  #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int col = kk * 16;
+          mma_ss_w(s_tm, sdesc_add(dQ_t, (kk >> 2) * C::PANEL + (kk & 3) * 32),
+                   sdesc_add(db0[col / C::CH], ((col % C::CH) / 64) * C::PANEL + (kk & 3) * 32), C::IDESC_S,
+                   kk > 0 ? 1u : 0u);
+        }
+        tc_commit_w(BAR(C::B_SFULL + t));
+        if (jj == w.nit - 1) tc_commit_w(BAR(C::B_QEMPTY + t));  // last QKᵀ of this tile in the item
+        release(U);
+        return true;
+      };
+      // O_t (+)= P_t · V for one 64-key half of the P tile
+      auto issue_pv = [&](int U, bool first, int half) {
+  #pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const uint64_t db0 = sdesc_add(dKV_mn, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
+  #pragma unroll
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+            mma_ts_w(o_tm + c * C::CH, p_tm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_PV,
+                     (!first || kk > 0) ? 1u : 0u);
+        }
+      };
 
-    int k = 0;
-    while (k < n_rounds && fwd_item_index<CAUSAL>(k, cta, G) >= n_items) ++k;
-    if (k < n_rounds) {
-      FwdItem w = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k, cta, G), p, ne);
-      int base = 0;
-      for (int t = 0; t < 2 && ok; ++t)
-        if (w.has(t)) ok = issue_s(t, w, base, w.first(t));
-      while (ok) {
-        int k2 = k + 1;
-        while (k2 < n_rounds && fwd_item_index<CAUSAL>(k2, cta, G) >= n_items) ++k2;
-        const bool has_next = k2 < n_rounds;
-        FwdItem w2 = w;
-        if (has_next) w2 = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k2, cta, G), p, ne);
-        const int base2 = base + 2 * w.nit;
-        for (int jj = 0; jj < w.nit && ok; ++jj) {
-          for (int t = 0; t < 2; ++t) {
-            if (!w.has(t) || jj < w.first(t)) continue;
+      int k = 0;
+      while (k < n_rounds && fwd_item_index<CAUSAL>(k, cta, G) >= n_items) ++k;
+      if (k < n_rounds) {
+        FwdItem w = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k, cta, G), p, ne);
+        int base = 0;
+        if (w.has(t)) ok = issue_s(w, base, w.first(t));
+        while (ok) {
+          int k2 = k + 1;
+          while (k2 < n_rounds && fwd_item_index<CAUSAL>(k2, cta, G) >= n_items) ++k2;
+          const bool has_next = k2 < n_rounds;
+          FwdItem w2 = w;
+          if (has_next) w2 = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k2, cta, G), p, ne);
+          const int base2 = base + 2 * w.nit;
+          for (int jj = 0; jj < w.nit && ok; ++jj) {
+            if (!w.has(t) || jj < w.first(t)) {
+              // K and V units of this iteration that this tile does not read
+              if (!wait_unit(base + 2 * jj) || !wait_unit(base + 2 * jj + 1)) { ok = false; break; }
+              release(base + 2 * jj);
+              release(base + 2 * jj + 1);
+              continue;
+            }
+            // SEP_P: the tile's next QKᵀ of this item goes before its PV (the
+            // next item's first one stays after it: it may wait for a Q load)
+            if (C::SEP_P && jj + 1 < w.nit && !(ok = issue_s(w, base, jj + 1))) break;
             const int Uv = base + 2 * jj + 1;
             const bool first = (jj == w.first(t));
-            if (!mbar_wait_warp(BAR(C::B_PFULL + t), p_seen[t] & 1, wc, 45)) { ok = false; break; }
-            if (!wait_upto(Uv)) { ok = false; break; }
-            issue_pv(t, Uv, first, 0);
-            if (!mbar_wait_warp(BAR(C::B_PFULL2 + t), p_seen[t] & 1, wc, 46)) { ok = false; break; }
+            if (!mbar_wait_warp(BAR(C::B_PFULL + t), p_seen & 1, wc, 45)) { ok = false; break; }
+            if (!wait_unit(Uv)) { ok = false; break; }
+            issue_pv(Uv, first, 0);
+            if (!mbar_wait_warp(BAR(C::B_PFULL2 + t), p_seen & 1, wc, 46)) { ok = false; break; }
             tc_fence_after();
-            issue_pv(t, Uv, first, 1);
+            issue_pv(Uv, first, 1);
             tc_commit_w(BAR(C::B_ODONE + t));
-            ++p_seen[t];
-            if (t == 1 || w.n1 == 0) release(Uv);  // last reader of this V unit
+            ++p_seen;
+            release(Uv);
             // this tile's next QKᵀ: the item's next iteration, or the next item's first
             if (jj + 1 < w.nit) {
-              ok = issue_s(t, w, base, jj + 1);
+              if (!C::SEP_P) ok = issue_s(w, base, jj + 1);
             } else if (has_next && w2.has(t)) {
-              ok = issue_s(t, w2, base2, w2.first(t));
+              ok = issue_s(w2, base2, w2.first(t));
             }
-            if (!ok) break;
+          }
+          if (!ok || !has_next) break;
+          // the tile had no rows in this item, so its first QKᵀ of the next one is still due
+          if (!w.has(t) && w2.has(t)) ok = issue_s(w2, base2, w2.first(t));
+          w = w2;
+          base = base2;
+          k = k2;
+        }
+      }
+      // no MMA of either warp may still be running when TMEM is released
+      tc_commit_w(BAR(C::B_DRAIN));
+      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 47);
+    } else {
+      // ---------------------------------------------------------- MMA issuer
+      // (the whole warp runs this role; one elected lane issues each instruction)
+      setmaxnreg_dec<C::CTRL_REGS>();
+      bool ok = true;
+      int waited = -1;           // K/V units whose arrival has been observed, in load order
+      int qfull_seen[2] = {0, 0};
+      int p_seen[2] = {0, 0};    // P hand-overs consumed per tile
+      // Wait for every unit up to U in load order: a unit's slot barrier is only
+      // ever waited on for its current fill, so the parity test is unambiguous.
+      auto wait_upto = [&](int U) -> bool {
+        while (waited < U) {
+          ++waited;
+  #pragma unroll
+          for (int c = 0; c < C::NCH; ++c) {
+            const int seq = waited * C::NCH + c;
+            if (!mbar_wait_warp(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 43)) return false;
           }
         }
-        if (!ok || !has_next) break;
-        // tile 1 had no rows in this item, so its first QKᵀ of the next one is still due
-        if (!w.has(1) && w2.has(1)) ok = issue_s(1, w2, base2, 0);
-        w = w2;
-        base = base2;
-        k = k2;
+        tc_fence_after();
+        return true;
+      };
+      auto release = [&](int U) {
+  #pragma unroll
+        for (int c = 0; c < C::NCH; ++c) tc_commit_w(BAR(C::B_KVEMPTY + (U * C::NCH + c) % C::NSLOT));
+      };
+      const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
+      const uint64_t dKV_k = sdesc_sw128(sbase + C::KV_OFF, 16, 1024);
+      const uint64_t dKV_mn = sdesc_sw128(sbase + C::KV_OFF, C::PANEL, 1024);
+      // S_t = Q_t · Kᵀ for iteration jj of item w (its K unit is base + 2·jj)
+      auto issue_s = [&](int t, const FwdItem& w, int base, int jj) -> bool {
+        if (jj == w.first(t)) {
+          if (!mbar_wait_warp(BAR(C::B_QFULL + t), qfull_seen[t] & 1, wc, 44)) return false;
+          ++qfull_seen[t];
+        }
+        const int U = base + 2 * jj;
+        if (!wait_upto(U)) return false;
+        const uint64_t da0 = sdesc_add(dQ_k, t * C::Q_BYTES);
+        uint64_t db0[C::NCH];
+  #pragma unroll
+        for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
+  #pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const int col = kk * 16;
+          mma_ss_w(tbase + C::S_COL + 128 * t, sdesc_add(da0, (kk >> 2) * C::PANEL + (kk & 3) * 32),
+                   sdesc_add(db0[col / C::CH], ((col % C::CH) / 64) * C::PANEL + (kk & 3) * 32), C::IDESC_S,
+                   kk > 0 ? 1u : 0u);
+        }
+        tc_commit_w(BAR(C::B_SFULL + t));
+        if (jj == w.nit - 1) tc_commit_w(BAR(C::B_QEMPTY + t));  // last QKᵀ of this tile in the item
+        if (t == 1 || w.n1 == 0) release(U);                      // last reader of this K unit
+        return true;
+      };
+      // O_t (+)= P_t · V for one 64-key half of the P tile
+      auto issue_pv = [&](int t, int U, bool first, int half) {
+  #pragma unroll
+        for (int c = 0; c < C::NCH; ++c) {
+          const uint64_t db0 = sdesc_add(dKV_mn, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
+  #pragma unroll
+          for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
+            mma_ts_w(tbase + C::O_COL + t * D + c * C::CH, tbase + C::S_COL + 128 * t + kk * 8,
+                     sdesc_add(db0, kk * 2048), C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
+        }
+      };
+
+      int k = 0;
+      while (k < n_rounds && fwd_item_index<CAUSAL>(k, cta, G) >= n_items) ++k;
+      if (k < n_rounds) {
+        FwdItem w = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k, cta, G), p, ne);
+        int base = 0;
+        for (int t = 0; t < 2 && ok; ++t)
+          if (w.has(t)) ok = issue_s(t, w, base, w.first(t));
+        while (ok) {
+          int k2 = k + 1;
+          while (k2 < n_rounds && fwd_item_index<CAUSAL>(k2, cta, G) >= n_items) ++k2;
+          const bool has_next = k2 < n_rounds;
+          FwdItem w2 = w;
+          if (has_next) w2 = fwd_item<CAUSAL, VARLEN>(fwd_item_index<CAUSAL>(k2, cta, G), p, ne);
+          const int base2 = base + 2 * w.nit;
+          for (int jj = 0; jj < w.nit && ok; ++jj) {
+            for (int t = 0; t < 2; ++t) {
+              if (!w.has(t) || jj < w.first(t)) continue;
+              const int Uv = base + 2 * jj + 1;
+              const bool first = (jj == w.first(t));
+              if (!mbar_wait_warp(BAR(C::B_PFULL + t), p_seen[t] & 1, wc, 45)) { ok = false; break; }
+              if (!wait_upto(Uv)) { ok = false; break; }
+              issue_pv(t, Uv, first, 0);
+              if (!mbar_wait_warp(BAR(C::B_PFULL2 + t), p_seen[t] & 1, wc, 46)) { ok = false; break; }
+              tc_fence_after();
+              issue_pv(t, Uv, first, 1);
+              tc_commit_w(BAR(C::B_ODONE + t));
+              ++p_seen[t];
+              if (t == 1 || w.n1 == 0) release(Uv);  // last reader of this V unit
+              // this tile's next QKᵀ: the item's next iteration, or the next item's first
+              if (jj + 1 < w.nit) {
+                ok = issue_s(t, w, base, jj + 1);
+              } else if (has_next && w2.has(t)) {
+                ok = issue_s(t, w2, base2, w2.first(t));
+              }
+              if (!ok) break;
+            }
+          }
+          if (!ok || !has_next) break;
+          // tile 1 had no rows in this item, so its first QKᵀ of the next one is still due
+          if (!w.has(1) && w2.has(1)) ok = issue_s(1, w2, base2, 0);
+          w = w2;
+          base = base2;
+          k = k2;
+        }
       }
+      // no MMA may still be running when TMEM is released
+      tc_commit_w(BAR(C::B_DRAIN));
+      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 47);
     }
-    // no MMA may still be running when TMEM is released
-    tc_commit_w(BAR(C::B_DRAIN));
-    mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 47);
   } else if (warp < 4) {
     // idle warps of the control warpgroup: hand their registers to the softmax
     setmaxnreg_dec<C::CTRL_REGS>();
@@ -384,6 +537,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
     const float sl2 = p.scale_log2;
     const int scol = C::S_COL + 128 * t;
     const int ocol = C::O_COL + t * D;
+    const int pcol = C::SEP_P ? C::P_COL + 64 * t : scol;
     int done = 0;  // S tiles this warpgroup has finished (phase count of its barriers)
     bool ok = true;
     for (int k = 0; k < n_rounds && ok; ++k) {
@@ -409,6 +563,12 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         reg_fence(r1);
         reg_fence(r2);
         reg_fence(r3);
+        if (C::SEP_P) {
+          // S is in registers: the tile's next QKᵀ may overwrite the buffer
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(BAR(C::B_SFREE + t));
+        }
         float s[128];
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
@@ -466,6 +626,11 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         {
           uint32_t pk[32];
           exp_half(0, pk);
+          if (C::SEP_P && j > 0 && !warp_rescale) {
+            // the previous block's PV must be done reading P before it is overwritten
+            if (!mbar_wait_warp(BAR(C::B_ODONE + t), (done + j - 1) & 1, wc, 52)) { ok = false; break; }
+            tc_fence_after();
+          }
           if (warp_rescale) {
             // O must hold the previous block's product before it is scaled,
             // and be scaled before this block's first PV half accumulates
@@ -482,7 +647,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
               tmem_st32(tl + ocol + oc * 32, ov);
             }
           }
-          tmem_st32(tl + scol, pk);
+          tmem_st32(tl + pcol, pk);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();
@@ -491,7 +656,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         {
           uint32_t pk[32];
           exp_half(64, pk);
-          tmem_st32(tl + scol + 32, pk);
+          tmem_st32(tl + pcol + 32, pk);
           tmem_st_wait();
           tc_fence_before();
           __syncwarp();

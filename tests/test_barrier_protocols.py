@@ -401,11 +401,11 @@ def test_backward_half_stage_model_catches_a_missing_wait(mistake):
 
 
 # ----------------------------------------------------------------- forward
-def simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed, mistake=None):
-    """fa_fwd_persistent_kernel: items are pairs of 128-row query tiles of one
-    (b, h), dealt to ``n_ctas`` CTAs in a fixed order.  Roles per CTA: the
-    producer, the MMA warp and the two softmax warpgroups (one per query
-    tile).  K and V blocks are separate "units" streamed through ``n_slot``
+def simulate_fwd_single(n_qtiles, BH, causal, n_ctas, n_slot, seed, mistake=None):
+    """fa_fwd_persistent_kernel at d = 128: items are pairs of 128-row query
+    tiles of one (b, h), dealt to ``n_ctas`` CTAs in a fixed order.  Roles
+    per CTA: the producer, one MMA warp for both tiles and the two softmax
+    warpgroups (one per query tile).  K and V blocks are separate "units" streamed through ``n_slot``
     slots; with a causal mask the second tile's diagonal block comes first."""
     rnd = random.Random(seed)
     n_pairs = (n_qtiles + 1) // 2
@@ -610,23 +610,293 @@ def simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed, mistake=None):
 
 @pytest.mark.parametrize("causal", [False, True])
 @pytest.mark.parametrize("n_slot", [5, 8])
-def test_forward_protocol(causal, n_slot):
+def test_forward_single_mma_warp_protocol(causal, n_slot):
     for n_qtiles in (1, 2, 3, 5, 8):
         for BH, n_ctas in ((1, 1), (3, 2), (5, 3)):
-            simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed=n_qtiles * 7 + BH)
+            simulate_fwd_single(n_qtiles, BH, causal, n_ctas, n_slot, seed=n_qtiles * 7 + BH)
 
 
-def test_forward_model_catches_a_missing_wait():
+def test_forward_single_mma_warp_model_catches_a_missing_wait():
     caught = 0
     for seed in range(20):
         try:
-            simulate_fwd(4, 3, True, 1, 5, seed, mistake="no_qempty_wait")
+            simulate_fwd_single(4, 3, True, 1, 5, seed, mistake="no_qempty_wait")
         except AssertionError:
             caught += 1
     assert caught > 0
 
 
 # ------------------------------------------------------------ forward, CTA pair
+def simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed, sep_p=False, mistake=None, max_steps=20_000_000):
+    """fa_fwd_persistent_kernel: items are pairs of 128-row query tiles of one
+    (b, h), dealt to ``n_ctas`` CTAs in a fixed order.  Roles per CTA: the
+    producer, one MMA warp and one softmax warpgroup per query tile.  K and V
+    blocks are separate "units" streamed through ``n_slot`` slots; with a
+    causal mask the second tile's diagonal block comes first.
+
+    At d = 64, MMA warp t issues tile t's QKᵀ and PV products only.  Both warps walk every K/V unit
+    in load order and commit its release (the slot's empty barrier counts two
+    arrivals), so the producer refills a slot only after both are done with
+    it; a warp waits only for the units its tile reads.  ``sep_p`` (d = 64):
+    P has its own TMEM columns, so a tile's next QKᵀ of the same item is
+    issued as soon as the softmax has read S (SFREE), and the softmax waits
+    for the previous PV before it writes P."""
+    rnd = random.Random(seed)
+    n_pairs = (n_qtiles + 1) // 2
+    n_items = n_pairs * BH
+    issued = {"S": [], "PV": []}
+
+    def item(idx):
+        if causal:
+            pair, bh = n_pairs - 1 - idx // BH, idx % BH
+        else:
+            bh, pair = idx // n_pairs, idx % n_pairs
+        qt0 = 2 * pair
+        has1 = qt0 + 1 < n_qtiles
+        n0 = qt0 + 1 if causal else n_qtiles
+        n1 = (qt0 + 2 if causal else n_qtiles) if has1 else 0
+        skew = 1 if (causal and has1) else 0
+        return dict(qt0=qt0, n0=n0, n1=n1, skew=skew, nit=n0 + skew)
+
+    def kv_block(w, jj):
+        return w["qt0"] + 1 if (w["skew"] and jj == 0) else jj - w["skew"]
+
+    def first(w, t):
+        return w["skew"] if t == 0 else 0
+
+    def has(w, t):
+        return t == 0 or w["n1"] > 0
+
+    def deal(k, c):
+        return k * n_ctas + ((n_ctas - 1 - c) if (causal and (k & 1)) else c)
+
+    n_rounds = (n_items + n_ctas - 1) // n_ctas
+    gens, engines = {}, {}
+    all_items = []
+
+    def make_cta(c):
+        items = [deal(k, c) for k in range(n_rounds) if deal(k, c) < n_items]
+        all_items.extend(items)
+        bars = {}
+        for t in range(2):
+            for nm in ("QFULL", "QEMPTY", "SFULL", "ODONE"):
+                bars[nm, t] = _Bar(1)
+            bars["PFULL", t] = _Bar(4)
+            bars["PFULL2", t] = _Bar(4)
+            bars["SFREE", t] = _Bar(4)
+        for s in range(n_slot):
+            bars["KVFULL", s] = _Bar(1)
+            bars["KVEMPTY", s] = _Bar(2)
+        wait = _waiter(bars)
+        tc, tma = [], []
+        slot_unit, loaded = {}, set()
+        q_tile = {0: None, 1: None}
+        unit_readers = {}           # unit -> ids of products that read it
+        completed = set()
+        commits = {}                # unit -> release commits that completed
+        s_issued, s_read = [0, 0], [0, 0]
+        p_written, pv_done = [0, 0], [0, 0]
+        prod_id = [0]
+        unit_of = {}
+        u_acc = 0
+        for idx in items:
+            for u in range(2 * item(idx)["nit"]):
+                unit_of[u_acc + u] = (idx, u)
+            u_acc += 2 * item(idx)["nit"]
+
+        def producer():
+            useq = 0
+            q_loads = [0, 0]
+            for idx in items:
+                w = item(idx)
+                for t in range(2):
+                    if not has(w, t):
+                        continue
+                    if q_loads[t] > 0 and mistake != "no_qempty_wait":
+                        yield from wait(("QEMPTY", t), q_loads[t] - 1)
+                    q_tile[t] = (idx, t)
+                    tma.append((("QFULL", t), None))
+                    q_loads[t] += 1
+                for u in range(2 * w["nit"]):
+                    U = useq + u
+                    s = U % n_slot
+                    if U >= n_slot:
+                        yield from wait(("KVEMPTY", s), U // n_slot - 1)
+                    if s in slot_unit:
+                        old = slot_unit[s]
+                        assert commits.get(old, 0) == 2, f"slot {s} refilled before both warps released unit {old}"
+                        assert unit_readers.get(old, set()) <= completed, f"slot {s} refilled while unit {old} is read"
+                    slot_unit[s] = U
+                    tma.append((("KVFULL", s), U))
+                useq += 2 * w["nit"]
+
+        def mma(t):
+            q_seen = [0]
+            p_seen = [0]
+
+            def wait_unit(U):
+                yield from wait(("KVFULL", U % n_slot), U // n_slot)
+                assert U in loaded and slot_unit[U % n_slot] == U
+
+            def product(kind, U):
+                prod_id[0] += 1
+                unit_readers.setdefault(U, set()).add(prod_id[0])
+                tc.append(("mma", prod_id[0]))
+
+            def release(U):
+                if mistake == "one_release_only" and t == 0:
+                    return
+                tc.append(("release", U))
+
+            def issue_s(w, idx, base, jj):
+                if sep_p and s_issued[t] > 0 and mistake != "no_sfree_wait":
+                    yield from wait(("SFREE", t), s_issued[t] - 1)
+                assert s_read[t] == s_issued[t], f"S buffer {t} overwritten before it was read"
+                s_issued[t] += 1
+                if jj == first(w, t):
+                    yield from wait(("QFULL", t), q_seen[0])
+                    q_seen[0] += 1
+                assert q_tile[t] == (idx, t), f"Q tile {t} overwritten: {q_tile[t]} for item {idx}"
+                U = base + 2 * jj
+                yield from wait_unit(U)
+                assert unit_of[U] == (idx, 2 * jj)
+                product("S", U)
+                issued["S"].append((idx, t, kv_block(w, jj)))
+                tc.append(("commit", ("SFULL", t)))
+                if jj == w["nit"] - 1:
+                    tc.append(("commit", ("QEMPTY", t)))
+                release(U)
+
+            if not items:
+                return
+            idx, w, base = items[0], item(items[0]), 0
+            if has(w, t):
+                yield from issue_s(w, idx, base, first(w, t))
+            for pos in range(len(items)):
+                nxt = items[pos + 1] if pos + 1 < len(items) else None
+                w2 = item(nxt) if nxt is not None else None
+                base2 = base + 2 * w["nit"]
+                for jj in range(w["nit"]):
+                    if not has(w, t) or jj < first(w, t):
+                        # units this tile does not read: release each once it
+                        # holds this fill (a release ahead of the load would
+                        # count towards the slot's previous fill)
+                        for U in (base + 2 * jj, base + 2 * jj + 1):
+                            if mistake != "release_before_load":
+                                yield from wait_unit(U)
+                            release(U)
+                        continue
+                    if sep_p and jj + 1 < w["nit"]:
+                        yield from issue_s(w, idx, base, jj + 1)
+                    Uv = base + 2 * jj + 1
+                    yield from wait(("PFULL", t), p_seen[0])
+                    yield from wait_unit(Uv)
+                    yield from wait(("PFULL2", t), p_seen[0])
+                    product("PV", Uv)
+                    issued["PV"].append((idx, t, kv_block(w, jj)))
+                    tc.append(("pv", t))
+                    tc.append(("commit", ("ODONE", t)))
+                    p_seen[0] += 1
+                    release(Uv)
+                    if jj + 1 < w["nit"]:
+                        if not sep_p:
+                            yield from issue_s(w, idx, base, jj + 1)
+                    elif nxt is not None and has(w2, t):
+                        yield from issue_s(w2, nxt, base2, first(w2, t))
+                if nxt is None:
+                    break
+                if not has(w, t) and has(w2, t):
+                    yield from issue_s(w2, nxt, base2, first(w2, t))
+                idx, w, base = nxt, w2, base2
+
+        def softmax(t):
+            done = 0
+            for idx in items:
+                w = item(idx)
+                if not has(w, t):
+                    continue
+                n = w["n0"] if t == 0 else w["n1"]
+                for j in range(n):
+                    yield from wait(("SFULL", t), done + j)
+                    yield
+                    s_read[t] += 1
+                    if sep_p:
+                        for _ in range(4):
+                            bars["SFREE", t].arrive()
+                        if j > 0:
+                            yield from wait(("ODONE", t), done + j - 1)
+                        assert pv_done[t] == p_written[t], f"P buffer {t} overwritten while a PV reads it"
+                    elif j > 0 and rnd.random() < 0.3:
+                        yield from wait(("ODONE", t), done + j - 1)
+                    p_written[t] += 1
+                    for _ in range(4):
+                        bars["PFULL", t].arrive()
+                    yield
+                    for _ in range(4):
+                        bars["PFULL2", t].arrive()
+                yield from wait(("ODONE", t), done + n - 1)
+                done += n
+
+        def tc_done(entry):
+            kind, x = entry
+            if kind == "mma":
+                completed.add(x)
+            elif kind == "pv":
+                pv_done[x] += 1
+            elif kind == "release":
+                commits[x] = commits.get(x, 0) + 1
+                bars["KVEMPTY", x % n_slot].arrive()
+            else:
+                bars[x].arrive()
+
+        def tma_done(entry):
+            bar, unit = entry
+            if unit is not None:
+                loaded.add(unit)
+            bars[bar].arrive()
+
+        gens[c, "producer"] = producer()
+        for t in range(2):
+            gens[c, "mma", t] = mma(t)
+            gens[c, "softmax", t] = softmax(t)
+        engines[c, "tc"] = (tc, tc_done)
+        engines[c, "tma"] = (tma, tma_done)
+
+    for c in range(n_ctas):
+        make_cta(c)
+    _run(gens, engines, rnd, max_steps)
+    assert sorted(all_items) == list(range(n_items))
+    for kind in ("S", "PV"):
+        got = sorted(issued[kind])
+        want = []
+        for idx in range(n_items):
+            w = item(idx)
+            for t in range(2):
+                if has(w, t):
+                    qt = w["qt0"] + t
+                    want += [(idx, t, j) for j in (range(qt + 1) if causal else range(n_qtiles))]
+        assert got == sorted(want), kind
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("n_slot", [8, 5])
+def test_forward_per_tile_mma_warp_protocol(causal, n_slot):
+    for n_qtiles in (1, 2, 3, 5, 8):
+        for BH, n_ctas in ((1, 1), (3, 2), (5, 3)):
+            simulate_fwd(n_qtiles, BH, causal, n_ctas, n_slot, seed=n_qtiles * 7 + BH, sep_p=True)
+
+
+@pytest.mark.parametrize("mistake", ["no_qempty_wait", "no_sfree_wait", "one_release_only", "release_before_load"])
+def test_forward_per_tile_model_catches_a_missing_wait(mistake):
+    caught = 0
+    for seed in range(30):
+        try:
+            simulate_fwd(3, 3, seed % 2 == 1, 1, 5, seed, True, mistake, max_steps=200_000)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
 def simulate_fwd_pair(n0, n1, n_slot, seed, mistake=None, max_steps=20_000_000):
     """fa_fwd_pair_kernel: one cluster of two CTAs, each with two query tiles;
     tile pair t (one tile in each CTA) multiplies K/V blocks 0 .. n_t - 1,
