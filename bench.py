@@ -525,8 +525,9 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
     copies that step's Q, K, V, dO from pinned host memory to the device, runs
     fa_fwd and fa_bwd, and copies O, LSE, dQ, dK, dV back.  As in a training
     loop, the copies of neighbouring steps overlap the kernels: H2D and D2H run
-    on their own streams (the GPU's copy engines) over two sets of device
-    buffers, with events ordering each buffer's reuse.  The timed region runs
+    on their own streams (the GPU's copy engines) over three sets of device
+    buffers, with events ordering each buffer's reuse, so that both copy
+    directions can stay busy while the kernels run.  The timed region runs
     from the first H2D to the last D2H."""
     import torch
 
@@ -535,29 +536,30 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
     B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
     q0, k0, v0, do0, o0, lse0, dq0, dk0, dv0, ws0 = bufs0
     host_in = [t.cpu().pin_memory() for t in (q0, k0, v0, do0)]
-    sets = [bufs0, tuple(torch.empty_like(t) for t in bufs0)]
+    n_sets = 3
+    sets = [bufs0] + [tuple(torch.empty_like(t) for t in bufs0) for _ in range(n_sets - 1)]
     host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o0, lse0, dq0, dk0, dv0)]
-                for _ in range(2)]
+                for _ in range(n_sets)]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out[0])
     s_h2d = torch.cuda.Stream(device=dev)
     s_d2h = torch.cuda.Stream(device=dev)
     ev = lambda: torch.cuda.Event(enable_timing=False)  # noqa: E731
-    in_ready = [ev(), ev()]
-    comp_done = [ev(), ev()]
-    out_done = [ev(), ev()]
+    in_ready = [ev() for _ in range(n_sets)]
+    comp_done = [ev() for _ in range(n_sets)]
+    out_done = [ev() for _ in range(n_sets)]
 
     def step(i):
-        b = i % 2
+        b = i % n_sets
         q, k, v, do, o, lse, dq, dk, dv, ws = sets[b]
         with torch.cuda.stream(s_h2d):
-            if i >= 2:
+            if i >= n_sets:
                 s_h2d.wait_event(comp_done[b])  # this buffer's previous step no longer reads its inputs
             for hsrc, ddst in zip(host_in, (q, k, v, do)):
                 ddst.copy_(hsrc, non_blocking=True)
             in_ready[b].record(s_h2d)
         stream.wait_event(in_ready[b])
-        if i >= 2:
+        if i >= n_sets:
             stream.wait_event(out_done[b])  # its previous outputs have reached the host
         st = binding.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, w.causal, w.scale, stream)
         if st:
@@ -574,7 +576,7 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
             out_done[b].record(s_d2h)
 
     ke = max(3, min(K, 30))
-    for i in range(2):  # warm-up
+    for i in range(n_sets):  # warm-up
         step(i)
     torch.cuda.synchronize()
     barrier()
@@ -592,7 +594,7 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
     ms = max_over_ranks(t0.elapsed_time(t1)) / ke
     return {"value": step_flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
-            "overlap": "H2D of step i+1 and D2H of step i-1 overlap the kernels of step i (2 buffer sets)"}
+            "overlap": "H2D of later steps and D2H of earlier ones overlap the kernels of step i (3 buffer sets)"}
 
 
 # ------------------------------------------------------------------- ours
