@@ -469,32 +469,23 @@ def run_varlen(args, w, rank, world, local_rank):
 
     e2e = None
     if not args.no_e2e:
-        host_in = [t.cpu().pin_memory() for t in (q, k, v, do)]
-        host_out = [torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o, lse, dq, dk, dv)]
-        host_cu = cu.cpu().pin_memory()
+        def e2e_compute(ins, outs, extra):
+            q_, k_, v_, do_, cu_ = ins
+            o_, lse_, dq_, dk_, dv_ = outs
+            fw_, bw_ = extra
+            st = binding.fa_fwd_varlen(q_, k_, v_, o_, lse_, cu_, nseq, w.Hq, w.Hkv, T, w.max_seqlen, w.d, w.causal,
+                                       w.scale, fw_, fws, stream)
+            if st:
+                raise binding.FAError(st, "fa_fwd_varlen")
+            st = binding.fa_bwd_varlen(q_, k_, v_, o_, lse_, do_, dq_, dk_, dv_, cu_, nseq, w.Hq, w.Hkv, T,
+                                       w.max_seqlen, w.d, w.causal, w.scale, bw_, bws, stream)
+            if st:
+                raise binding.FAError(st, "fa_bwd_varlen")
 
-        def e2e_step():
-            for hsrc, ddst in zip(host_in, (q, k, v, do)):
-                ddst.copy_(hsrc, non_blocking=True)
-            cu.copy_(host_cu, non_blocking=True)
-            step()
-            for hdst, dsrc in zip(host_out, (o, lse, dq, dk, dv)):
-                hdst.copy_(dsrc, non_blocking=True)
-
-        e2e_step()
-        ke = max(3, min(K, 20))
-        barrier()
-        a, b = ev(), ev()
-        a.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        b.record(stream)
-        barrier()
-        ms_e2e = mo(a.elapsed_time(b)) / ke
-        e2e = {"value": 3.5 * F * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": sum(t.numel() * t.element_size() for t in host_in) + host_cu.numel() * 4,
-               "d2h_bytes_per_step": sum(t.numel() * t.element_size() for t in host_out), "steps": ke,
-               "overlap": "none: copies and kernels of a step in order on one stream"}
+        e2e = run_e2e(dev, stream, (q, k, v, do, cu), (o, lse, dq, dk, dv), (fw, bw), e2e_compute, 3.5 * F,
+                      world, barrier, mo, K)
+        if binding.fa_device_status(stream) != 0:
+            raise RuntimeError("device error in the end-to-end region")
     line = {
         "metric": METRIC, "value": value, "unit": "TFLOPS", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
@@ -520,26 +511,25 @@ def run_varlen(args, w, rank, world, local_rank):
 
 
 # ------------------------------------------------------------------- e2e
-def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ranks, K):
+def run_e2e(dev, stream, ins0, outs0, extra0, compute, step_flops, world, barrier, max_over_ranks, K):
     """The step through the public C ABI with its data on the host: every step
-    copies that step's Q, K, V, dO from pinned host memory to the device, runs
-    fa_fwd and fa_bwd, and copies O, LSE, dQ, dK, dV back.  As in a training
-    loop, the copies of neighbouring steps overlap the kernels: H2D and D2H run
-    on their own streams (the GPU's copy engines) over three sets of device
-    buffers, with events ordering each buffer's reuse, so that both copy
-    directions can stay busy while the kernels run.  The timed region runs
-    from the first H2D to the last D2H."""
+    copies that step's inputs from pinned host memory to the device, runs the
+    step's kernels (``compute(ins, outs, extra)`` enqueues them on ``stream``)
+    and copies its outputs back.  As in a training loop, the copies of
+    neighbouring steps overlap the kernels: H2D and D2H run on their own
+    streams (the GPU's copy engines) over three sets of device buffers, with
+    events ordering each buffer's reuse, so that both copy directions can stay
+    busy while the kernels run.  The timed region runs from the first H2D to
+    the last D2H."""
     import torch
 
-    from exact_attention_104_b200 import binding
-
-    B, Hq, Hkv, N, d = w.B, w.Hq, w.Hkv, w.N, w.d
-    q0, k0, v0, do0, o0, lse0, dq0, dk0, dv0, ws0 = bufs0
-    host_in = [t.cpu().pin_memory() for t in (q0, k0, v0, do0)]
+    host_in = [t.cpu().pin_memory() for t in ins0]
     n_sets = 3
-    sets = [bufs0] + [tuple(torch.empty_like(t) for t in bufs0) for _ in range(n_sets - 1)]
-    host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in (o0, lse0, dq0, dk0, dv0)]
-                for _ in range(n_sets)]
+    sets = [(list(ins0), list(outs0), list(extra0))]
+    for _ in range(n_sets - 1):
+        sets.append(([torch.empty_like(t) for t in ins0], [torch.empty_like(t) for t in outs0],
+                     [torch.empty_like(t) for t in extra0]))
+    host_out = [[torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for t in outs0] for _ in range(n_sets)]
     h2d = sum(t.numel() * t.element_size() for t in host_in)
     d2h = sum(t.numel() * t.element_size() for t in host_out[0])
     s_h2d = torch.cuda.Stream(device=dev)
@@ -551,27 +541,21 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
 
     def step(i):
         b = i % n_sets
-        q, k, v, do, o, lse, dq, dk, dv, ws = sets[b]
+        ins, outs, extra = sets[b]
         with torch.cuda.stream(s_h2d):
             if i >= n_sets:
                 s_h2d.wait_event(comp_done[b])  # this buffer's previous step no longer reads its inputs
-            for hsrc, ddst in zip(host_in, (q, k, v, do)):
+            for hsrc, ddst in zip(host_in, ins):
                 ddst.copy_(hsrc, non_blocking=True)
             in_ready[b].record(s_h2d)
         stream.wait_event(in_ready[b])
         if i >= n_sets:
             stream.wait_event(out_done[b])  # its previous outputs have reached the host
-        st = binding.fa_fwd(q, k, v, o, lse, B, Hq, Hkv, N, d, w.causal, w.scale, stream)
-        if st:
-            raise binding.FAError(st, "fa_fwd")
-        st = binding.fa_bwd(q, k, v, o, lse, do, dq, dk, dv, B, Hq, Hkv, N, d, w.causal, w.scale, ws,
-                            ws.numel(), stream)
-        if st:
-            raise binding.FAError(st, "fa_bwd")
+        compute(ins, outs, extra)
         comp_done[b].record(stream)
         with torch.cuda.stream(s_d2h):
             s_d2h.wait_event(comp_done[b])
-            for hdst, dsrc in zip(host_out[b], (o, lse, dq, dk, dv)):
+            for hdst, dsrc in zip(host_out[b], outs):
                 hdst.copy_(dsrc, non_blocking=True)
             out_done[b].record(s_d2h)
 
@@ -589,8 +573,6 @@ def run_e2e(args, w, dev, stream, bufs0, step_flops, world, barrier, max_over_ra
     t1.record(s_d2h)
     torch.cuda.synchronize()
     barrier()
-    if binding.fa_device_status(stream) != 0:
-        raise RuntimeError("device error in the end-to-end region")
     ms = max_over_ranks(t0.elapsed_time(t1)) / ke
     return {"value": step_flops * world / (ms * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms,
             "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h, "steps": ke,
@@ -754,8 +736,22 @@ def run_ours(args, w, rank, world, local_rank):
     # end to end through the public API with host buffers
     e2e = None
     if not args.no_e2e:
-        e2e = run_e2e(args, w, dev, stream, (q, k, v, do, o, lse, dq, dk, dv, ws), step_flops, world, barrier,
-                      max_over_ranks, K)
+        def e2e_compute(ins, outs, extra):
+            q_, k_, v_, do_ = ins
+            o_, lse_, dq_, dk_, dv_ = outs
+            (ws_,) = extra
+            st = binding.fa_fwd(q_, k_, v_, o_, lse_, B, Hq, Hkv, N, d, w.causal, scale, stream)
+            if st:
+                raise binding.FAError(st, "fa_fwd")
+            st = binding.fa_bwd(q_, k_, v_, o_, lse_, do_, dq_, dk_, dv_, B, Hq, Hkv, N, d, w.causal, scale, ws_,
+                                ws_bytes, stream)
+            if st:
+                raise binding.FAError(st, "fa_bwd")
+
+        e2e = run_e2e(dev, stream, (q, k, v, do), (o, lse, dq, dk, dv), (ws,), e2e_compute, step_flops, world,
+                      barrier, max_over_ranks, K)
+        if binding.fa_device_status(stream) != 0:
+            raise RuntimeError("device error in the end-to-end region")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
