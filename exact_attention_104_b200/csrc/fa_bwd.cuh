@@ -388,6 +388,9 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       tma_prefetch_desc(&tmV);
       tma_prefetch_desc(&tmDO);
       int gs = 0;  // steps loaded before this unit
+      // loads issued so far: K/V tiles (one per unit), steps' Q/dO tiles (one
+      // count per stage, or per half at d = 256)
+      int kv_loads = 0, q_issued = 0, ha_issued = 0, qb_issued = 0, dob_issued = 0;
       bool ok = true;
       for (int uc = 0; ok; ++uc) {
         // claim the next unit and publish its index (an index past the end
@@ -416,6 +419,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
               tma_load_2d(sbase + C::Q_OFF + pn * C::Q_PANEL, &tmQ, BAR(C::B_HAFULL), pn * 64, q_row);
               tma_load_2d(sbase + C::DO_OFF + pn * C::Q_PANEL, &tmDO, BAR(C::B_HAFULL), pn * 64, q_row);
             }
+            ha_issued = g + 1;
             if (!mbar_wait(BAR(C::B_HBEMPTY), (g & 1) ^ 1, wc, 41)) return false;
             mbar_expect_tx(BAR(C::B_QBFULL), 2 * C::Q_PANEL + 512);
 #pragma unroll
@@ -423,11 +427,13 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
               tma_load_2d(sbase + C::Q_OFF + (own + j) * C::Q_PANEL, &tmQ, BAR(C::B_QBFULL), (own + j) * 64, q_row);
             bulk_load(sbase + C::LS_OFF, p.lse2 + q_row_p, 256, BAR(C::B_QBFULL));
             bulk_load(sbase + C::LS_OFF + 256, p.dvec + q_row_p, 256, BAR(C::B_QBFULL));
+            qb_issued = g + 1;
             mbar_expect_tx(BAR(C::B_DOBFULL), 2 * C::Q_PANEL);
 #pragma unroll
             for (int j = 0; j < 2; ++j)
               tma_load_2d(sbase + C::DO_OFF + (own + j) * C::Q_PANEL, &tmDO, BAR(C::B_DOBFULL), (own + j) * 64,
                           q_row);
+            dob_issued = g + 1;
             return true;
           }
           const int st = g % C::NSTAGE;
@@ -443,6 +449,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           }
           bulk_load(sbase + C::LS_OFF + st * 512, p.lse2 + q_row_p, 256, bar);
           bulk_load(sbase + C::LS_OFF + st * 512 + 256, p.dvec + q_row_p, 256, bar);
+          q_issued = g + 1;
           return true;
         };
         // the first steps' tiles only need free stages: load them before K, V,
@@ -458,8 +465,22 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
           tma_load_2d(sbase + C::K_OFF + pn * C::KV_PANEL, &tmK, BAR(C::B_KVFULL), pn * 64, kv_row);
           tma_load_2d(sbase + C::V_OFF + pn * C::KV_PANEL, &tmV, BAR(C::B_KVFULL), pn * 64, kv_row);
         }
+        ++kv_loads;
         for (int s = pre; s < u.n && ok; ++s) ok = load_q(s);
         gs += u.n;
+      }
+      // every load issued has landed before the CTA may exit (immediate unless
+      // the CTA stopped early on a failed wait)
+      if (kv_loads > 0) mbar_wait_inflight(BAR(C::B_KVFULL), (kv_loads - 1) & 1, wc, 36);
+      if constexpr (C::HALVES) {
+        if (ha_issued > 0) mbar_wait_inflight(BAR(C::B_HAFULL), (ha_issued - 1) & 1, wc, 37);
+        if (qb_issued > 0) mbar_wait_inflight(BAR(C::B_QBFULL), (qb_issued - 1) & 1, wc, 38);
+        if (dob_issued > 0) mbar_wait_inflight(BAR(C::B_DOBFULL), (dob_issued - 1) & 1, wc, 39);
+      } else {
+        for (int st = 0; st < C::NSTAGE && st < q_issued; ++st) {
+          const int last = q_issued - 1 - (q_issued - 1 - st) % C::NSTAGE;  // last step loaded into stage st
+          mbar_wait_inflight(BAR(C::B_QFULL + st), (last / C::NSTAGE) & 1, wc, 10);
+        }
       }
     }
   } else if (warp == 1) {
@@ -607,7 +628,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         gs += n;
       }
       tc_commit_w(BAR(C::B_DRAIN));
-      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 17);
+      mbar_wait_inflight(BAR(C::B_DRAIN), 0, wc, 17);
     }
   } else if (warp < 4) {
     // idle warps of the control warpgroup

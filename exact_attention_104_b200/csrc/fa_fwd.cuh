@@ -236,6 +236,7 @@ __global__ void __launch_bounds__(FwdCfg<D, 1>::THREADS, 1)
         tma_load_2d_hint(sbase + C::Q_OFF + pn * C::PANEL, &tmQ, BAR(C::B_QFULL), pn * 64, q_row_base + qt * C::BM,
                          pol_q);
       bool ok = true;
+      int kv_issued = 0;  // K/V chunk loads issued (sequence numbers 0 .. kv_issued − 1)
       for (int u = 0; u < 2 * n && ok; ++u) {
         bool is_v;
         int j;
@@ -251,7 +252,15 @@ __global__ void __launch_bounds__(FwdCfg<D, 1>::THREADS, 1)
           for (int pp = 0; pp < C::CH / 64; ++pp)
             tma_load_2d_hint(sbase + C::KV_OFF + slot * C::SLOT_BYTES + pp * C::PANEL, is_v ? &tmV : &tmK,
                              BAR(C::B_KVFULL + slot), c * C::CH + pp * 64, kv_row_base + j * C::BN, pol_kv);
+          kv_issued = seq + 1;
         }
+      }
+      // every load issued has landed before the CTA may exit (immediate unless
+      // the CTA stopped early on a failed wait)
+      mbar_wait_inflight(BAR(C::B_QFULL), 0, wc, 12);
+      for (int sl = 0; sl < C::NSLOT && sl < kv_issued; ++sl) {
+        const int last = kv_issued - 1 - (kv_issued - 1 - sl) % C::NSLOT;  // last chunk loaded into slot sl
+        mbar_wait_inflight(BAR(C::B_KVFULL + sl), (last / C::NSLOT) & 1, wc, 13);
       }
     }
   } else if (warp == 1) {
@@ -356,7 +365,7 @@ __global__ void __launch_bounds__(FwdCfg<D, 1>::THREADS, 1)
       }
       // no MMA may still be running when TMEM is released
       tc_commit_w(BAR(C::B_DRAIN));
-      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 8);
+      mbar_wait_inflight(BAR(C::B_DRAIN), 0, wc, 8);
     }
   } else if (warp >= 4) {
     // ------------------------------------------------------------- softmax

@@ -153,6 +153,7 @@ __global__ void __launch_bounds__(FwdPairCfg::THREADS, 1)
                            q_base + (4 * item + 2 * t + (int)rank) * C::BM, pol_q);
       // units: K(0), V(0), K(1), V(1), ... of the blocks of tile pair 1
       bool ok = true;
+      int kv_issued = 0;  // units whose loads this CTA issued
       for (int u = 0; u < 2 * n1 && ok; ++u) {
         const int j = u >> 1;
         const int slot = u % C::NSLOT;
@@ -168,6 +169,17 @@ __global__ void __launch_bounds__(FwdPairCfg::THREADS, 1)
           for (int pn = 0; pn < D / 64; ++pn)
             tma_load_2d_pair(dst + pn * C::KH_PANEL, &tmK, LBAR(C::B_KVFULL + slot), pn * 64,
                              kv_base + j * C::BN + 64 * (int)rank, pol_kv);
+        }
+        kv_issued = u + 1;
+      }
+      // both CTAs' loads complete on the leader's barriers: the leader waits
+      // for every fill it armed before the pair's final cluster barrier
+      // (immediate unless a CTA stopped early on a failed wait)
+      if (leader) {
+        mbar_wait_inflight(BAR(C::B_QFULL), 0, wc, 70);
+        for (int sl = 0; sl < C::NSLOT && sl < kv_issued; ++sl) {
+          const int last = kv_issued - 1 - (kv_issued - 1 - sl) % C::NSLOT;  // last unit loaded into slot sl
+          mbar_wait_inflight(BAR(C::B_KVFULL + sl), (last / C::NSLOT) & 1, wc, 71);
         }
       }
     }
@@ -234,7 +246,7 @@ __global__ void __launch_bounds__(FwdPairCfg::THREADS, 1)
       }
       // no MMA may still be running when either CTA releases its TMEM
       tc_commit_pair_w(BAR(C::B_DRAIN));
-      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 66);
+      mbar_wait_inflight(BAR(C::B_DRAIN), 0, wc, 66);
     }
   } else if (warp < 4) {
     // idle warps of the control warpgroup: hand their registers to the softmax

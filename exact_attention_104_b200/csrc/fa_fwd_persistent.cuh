@@ -242,6 +242,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       const uint64_t pol_q = policy_evict_first();
       int useq = 0;               // K/V units loaded so far (a unit is NCH chunks)
       int qloads[2] = {0, 0};     // Q tiles loaded so far, per tile buffer
+      int kv_issued = 0;          // K/V chunk loads issued (chunk sequence numbers 0 .. kv_issued − 1)
       bool ok = true;
       for (int k = 0; k < n_rounds && ok; ++k) {
         const int idx = fwd_item_index<CAUSAL>(k, cta, G);
@@ -273,9 +274,18 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
             for (int pp = 0; pp < C::CH / 64; ++pp)
               tma_load_2d_hint(sbase + C::KV_OFF + slot * C::SLOT_BYTES + pp * C::PANEL, is_v ? &tmV : &tmK,
                                BAR(C::B_KVFULL + slot), c * C::CH + pp * 64, kv_row_base + kb * C::BN, pol_kv);
+            kv_issued = seq + 1;
           }
         }
         useq += 2 * w.nit;
+      }
+      // every load issued has landed before the CTA may exit (immediate unless
+      // the CTA stopped early on a failed wait)
+      for (int t = 0; t < 2; ++t)
+        if (qloads[t] > 0) mbar_wait_inflight(BAR(C::B_QFULL + t), (qloads[t] - 1) & 1, wc, 53);
+      for (int sl = 0; sl < C::NSLOT && sl < kv_issued; ++sl) {
+        const int last = kv_issued - 1 - (kv_issued - 1 - sl) % C::NSLOT;  // last chunk loaded into slot sl
+        mbar_wait_inflight(BAR(C::B_KVFULL + sl), (last / C::NSLOT) & 1, wc, 54);
       }
     }
   } else if (warp == 1 || (C::PER_TILE && warp == 2)) {
@@ -409,7 +419,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       }
       // no MMA of either warp may still be running when TMEM is released
       tc_commit_w(BAR(C::B_DRAIN));
-      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 47);
+      mbar_wait_inflight(BAR(C::B_DRAIN), 0, wc, 47);
     } else {
       // ---------------------------------------------------------- MMA issuer
       // (the whole warp runs this role; one elected lane issues each instruction)
@@ -522,7 +532,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       }
       // no MMA may still be running when TMEM is released
       tc_commit_w(BAR(C::B_DRAIN));
-      mbar_wait_warp(BAR(C::B_DRAIN), 0, wc, 47);
+      mbar_wait_inflight(BAR(C::B_DRAIN), 0, wc, 47);
     }
   } else if (warp < 4) {
     // idle warps of the control warpgroup: hand their registers to the softmax

@@ -91,6 +91,27 @@ __device__ __forceinline__ bool mbar_wait(uint32_t bar, uint32_t parity, const W
   }
 }
 
+// For work already in flight when a CTA stops (its own TMA loads and tensor
+// products complete by themselves): wait for phase `parity` of `bar` whether
+// or not the CTA has been aborted, so that the CTA neither frees TMEM under a
+// running product nor exits while a copy into its shared memory is still
+// landing.  The limit is the wait cap but at least 2^30 cycles (about half a
+// second), far beyond any copy's latency, so that a short cap set for a test
+// cannot cut it short; a timeout is recorded like any other.
+__device__ __forceinline__ bool mbar_wait_inflight(uint32_t bar, uint32_t parity, const WaitCtx& w, int site) {
+  if (mbar_try_wait(bar, parity)) return true;
+  const long long cap = w.cap > (1LL << 30) ? w.cap : (1LL << 30);
+  const long long t0 = clock64();
+  while (true) {
+    if (mbar_try_wait(bar, parity)) return true;
+    if (clock64() - t0 > cap) {
+      *w.abort_flag = 1;
+      atomicCAS(w.err, 0, kDevTimeout | (site << 8));
+      return false;
+    }
+  }
+}
+
 // Warp-collective form: every lane waits, and the warp proceeds only if all
 // lanes saw the phase complete (keeps .sync.aligned tcgen05 ops convergent).
 __device__ __forceinline__ bool mbar_wait_warp(uint32_t bar, uint32_t parity, const WaitCtx& w, int site) {
