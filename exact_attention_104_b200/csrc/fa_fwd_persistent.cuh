@@ -307,7 +307,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       // Wait for the fill of unit U: a warp never lags a full fill behind a
       // slot, because the slot is refilled only after both warps released it.
       auto wait_unit = [&](int U) -> bool {
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const int seq = U * C::NCH + c;
           if (!mbar_wait_warp(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 43)) return false;
@@ -316,7 +316,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         return true;
       };
       auto release = [&](int U) {
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) tc_commit_w(BAR(C::B_KVEMPTY + (U * C::NCH + c) % C::NSLOT));
       };
       const uint64_t dQ_t = sdesc_add(sdesc_sw128(sbase + C::Q_OFF, 16, 1024), t * C::Q_BYTES);
@@ -341,9 +341,9 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         const int U = base + 2 * jj;
         if (!wait_unit(U)) return false;
         uint64_t db0[C::NCH];
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
-  #pragma unroll
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int col = kk * 16;
           mma_ss_w(s_tm, sdesc_add(dQ_t, (kk >> 2) * C::PANEL + (kk & 3) * 32),
@@ -357,10 +357,10 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       };
       // O_t (+)= P_t · V for one 64-key half of the P tile
       auto issue_pv = [&](int U, bool first, int half) {
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const uint64_t db0 = sdesc_add(dKV_mn, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
-  #pragma unroll
+#pragma unroll
           for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
             mma_ts_w(o_tm + c * C::CH, p_tm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_PV,
                      (!first || kk > 0) ? 1u : 0u);
@@ -433,7 +433,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       auto wait_upto = [&](int U) -> bool {
         while (waited < U) {
           ++waited;
-  #pragma unroll
+#pragma unroll
           for (int c = 0; c < C::NCH; ++c) {
             const int seq = waited * C::NCH + c;
             if (!mbar_wait_warp(BAR(C::B_KVFULL + seq % C::NSLOT), (seq / C::NSLOT) & 1, wc, 43)) return false;
@@ -443,7 +443,7 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         return true;
       };
       auto release = [&](int U) {
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) tc_commit_w(BAR(C::B_KVEMPTY + (U * C::NCH + c) % C::NSLOT));
       };
       const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
@@ -459,9 +459,9 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
         if (!wait_upto(U)) return false;
         const uint64_t da0 = sdesc_add(dQ_k, t * C::Q_BYTES);
         uint64_t db0[C::NCH];
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) db0[c] = sdesc_add(dKV_k, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
-  #pragma unroll
+#pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const int col = kk * 16;
           mma_ss_w(tbase + C::S_COL + 128 * t, sdesc_add(da0, (kk >> 2) * C::PANEL + (kk & 3) * 32),
@@ -475,10 +475,10 @@ __global__ void __launch_bounds__(FwdPCfg<D>::THREADS, 1)
       };
       // O_t (+)= P_t · V for one 64-key half of the P tile
       auto issue_pv = [&](int t, int U, bool first, int half) {
-  #pragma unroll
+#pragma unroll
         for (int c = 0; c < C::NCH; ++c) {
           const uint64_t db0 = sdesc_add(dKV_mn, ((U * C::NCH + c) % C::NSLOT) * C::SLOT_BYTES);
-  #pragma unroll
+#pragma unroll
           for (int kk = 4 * half; kk < 4 * half + 4; ++kk)
             mma_ts_w(tbase + C::O_COL + t * D + c * C::CH, tbase + C::S_COL + 128 * t + kk * 8,
                      sdesc_add(db0, kk * 2048), C::IDESC_PV, (!first || kk > 0) ? 1u : 0u);
