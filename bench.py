@@ -312,30 +312,18 @@ def run_decode(args, w, rank, world, local_rank):
     if not args.no_e2e:
         # a decoding step's own data is its query rows and its outputs; the K/V
         # cache stays on the device between steps
-        hq = q.cpu().pin_memory()
-        ho = torch.empty(o.shape, dtype=o.dtype, pin_memory=True)
-        hl = torch.empty(lse.shape, dtype=lse.dtype, pin_memory=True)
+        def e2e_compute(ins, outs, extra):
+            (q_,) = ins
+            o_, lse_ = outs
+            (ws_,) = extra
+            st = binding.fa_fwd_decode(q_, k, v, o_, lse_, w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, w.scale,
+                                       ws_, ws_bytes, stream)
+            if st:
+                raise binding.FAError(st, "fa_fwd_decode")
 
-        def e2e_step():
-            q.copy_(hq, non_blocking=True)
-            step()
-            ho.copy_(o, non_blocking=True)
-            hl.copy_(lse, non_blocking=True)
-
-        e2e_step()
-        ke = max(3, min(K, 50))
-        barrier()
-        a, b = ev(), ev()
-        a.record(stream)
-        for _ in range(ke):
-            e2e_step()
-        b.record(stream)
-        barrier()
-        ms_e2e = max_over_ranks(a.elapsed_time(b)) / ke
-        e2e = {"value": F * world / (ms_e2e * 1e-3) / 1e12, "unit": "TFLOPS", "ms_per_step": ms_e2e,
-               "h2d_bytes_per_step": hq.numel() * hq.element_size(),
-               "d2h_bytes_per_step": ho.numel() * ho.element_size() + hl.numel() * hl.element_size(),
-               "steps": ke}
+        e2e = run_e2e(dev, stream, (q,), (o, lse), (ws,), e2e_compute, F, world, barrier, max_over_ranks, K)
+        if binding.fa_device_status(stream) != 0:
+            raise RuntimeError("device error in the end-to-end region")
 
     cpu = None
     if rank == 0 and world == 1 and not args.no_cpu_baseline:
