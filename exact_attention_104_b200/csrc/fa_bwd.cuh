@@ -37,7 +37,12 @@ struct BwdCfg {
   static constexpr int NDH = D / DH;            // CTAs per key tile
   static constexpr int BR = 64;                 // query rows per step
   static constexpr int BC = 128;                // keys per CTA
-  static constexpr int THREADS = 384;
+  // compute warpgroups: two at d = 64, where the compute warps rather than the
+  // tensor pipe bound a step (each group takes 32 of a step's 64 query columns)
+  static constexpr int NCG = (D == 64) ? 2 : 1;
+  static constexpr int CG_COLS = BR / NCG;
+  static constexpr int A_HALF = NCG == 2 ? 32 : 16;  // TMEM columns between the two 16-query halves of Pᵀ / dSᵀ
+  static constexpr int THREADS = 256 + 128 * NCG;
   static constexpr int KV_PANEL = BC * 128;     // 64 columns x 128 rows (bytes)
   static constexpr int Q_PANEL = BR * 128;      // 64 columns x 64 rows
   static constexpr int KV_BYTES = BC * D * 2;
@@ -103,12 +108,13 @@ struct BwdCfg {
   // Register split between the warpgroups (control: setmaxnreg.dec; compute
   // and drain: setmaxnreg.inc).  Valid for a launch allocation R with
   // CTRL_REGS <= R <= min(COMPUTE_REGS, DRAIN_REGS) and
-  // 128·(CTRL_REGS + COMPUTE_REGS + DRAIN_REGS) <= 384·R; checked on the host.
-  static constexpr int CTRL_REGS = 104;
-  static constexpr int COMPUTE_REGS = 208;
-  static constexpr int DRAIN_REGS = 168;
+  // 128·(CTRL_REGS + NCG·COMPUTE_REGS + DRAIN_REGS) <= THREADS·R; checked on the host.
+  static constexpr int CTRL_REGS = NCG == 2 ? 96 : 104;
+  static constexpr int COMPUTE_REGS = NCG == 2 ? 136 : 208;
+  static constexpr int DRAIN_REGS = NCG == 2 ? 136 : 168;
   static constexpr bool REG_SPLIT = (D <= 128);  // d = 256 needs more than 104 in the MMA warp
-  static constexpr int MIN_LAUNCH_REGS = (128 * (CTRL_REGS + COMPUTE_REGS + DRAIN_REGS) + THREADS - 1) / THREADS;
+  static constexpr int MIN_LAUNCH_REGS =
+      (128 * (CTRL_REGS + NCG * COMPUTE_REGS + DRAIN_REGS) + THREADS - 1) / THREADS;
   static constexpr int MAX_LAUNCH_REGS = COMPUTE_REGS < DRAIN_REGS ? COMPUTE_REGS : DRAIN_REGS;
 };
 
@@ -336,20 +342,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
     mbar_init(BAR(C::B_SFULL + 0), 1);
     mbar_init(BAR(C::B_SFULL + 1), 1);
     mbar_init(BAR(C::B_DPFULL), 1);
-    mbar_init(BAR(C::B_PFULL + 0), 4);
-    mbar_init(BAR(C::B_PFULL + 1), 4);
-    mbar_init(BAR(C::B_DSFULL), 4);
+    mbar_init(BAR(C::B_PFULL + 0), 4 * C::NCG);
+    mbar_init(BAR(C::B_PFULL + 1), 4 * C::NCG);
+    mbar_init(BAR(C::B_DSFULL), 4 * C::NCG);
     mbar_init(BAR(C::B_DQFULL), 1);
     mbar_init(BAR(C::B_DQEMPTY), 4);
     mbar_init(BAR(C::B_STGFREE), 1);
     mbar_init(BAR(C::B_STGFULL), 128);
     mbar_init(BAR(C::B_ACC), 1);
     mbar_init(BAR(C::B_KVEMPTY), 1);
-    mbar_init(BAR(C::B_DKFREE), 4);
+    mbar_init(BAR(C::B_DKFREE), 4 * C::NCG);
     mbar_init(BAR(C::B_DVFREE), 4);
     for (int i = 0; i < 2; ++i) {
       mbar_init(BAR(C::B_UNITFULL + i), 1);
-      mbar_init(BAR(C::B_UNITEMPTY + i), 9);  // MMA warp, four compute warps, four drain warps
+      mbar_init(BAR(C::B_UNITEMPTY + i), 5 + 4 * C::NCG);  // MMA warp, the compute warps, four drain warps
     }
     mbar_init(BAR(C::B_DRAIN), 1);
     for (int i = C::B_HAFULL; i <= C::B_HBEMPTY; ++i) mbar_init(BAR(i), 1);
@@ -512,7 +518,8 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       auto issue_acc = [&](uint32_t atm, uint64_t db0, uint32_t dtm, bool first) {
 #pragma unroll
         for (int kk = 0; kk < C::BR / 16; ++kk)
-          mma_ts_w(dtm, atm + kk * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV, (!first || kk > 0) ? 1u : 0u);
+          mma_ts_w(dtm, atm + (kk >> 1) * C::A_HALF + (kk & 1) * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV,
+                   (!first || kk > 0) ? 1u : 0u);
       };
       auto stage_bytes = [&](int g) -> uint32_t { return (uint32_t)(g % C::NSTAGE) * C::Q_BYTES; };
       auto q_off = [&](int g) -> uint64_t { return sdesc_add(dQ_k, stage_bytes(g)); };
@@ -633,9 +640,17 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
   } else if (warp < 4) {
     // idle warps of the control warpgroup
     if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
-  } else if (warp >= 4 && warp < 8) {
+  } else if ((warp >= 4 && warp < 8) || warp >= 12) {
     // ------------------------------------------- compute: Pᵀ and dSᵀ rows
+    // With two compute warpgroups (d = 64), warps 4-7 take query columns 0..31
+    // of each step and warps 12-15 columns 32..63; each group writes its bf16
+    // Pᵀ and dSᵀ into TMEM columns of its own Sᵀ / dPᵀ range (the products
+    // read the two 16-query halves A_HALF columns apart), so neither group
+    // overwrites columns the other has not read yet.
     if (C::REG_SPLIT) setmaxnreg_inc<C::COMPUTE_REGS>();
+    constexpr int NC = C::CG_COLS;                      // query columns of this group
+    const int cg = warp >= 12 ? 1 : 0;
+    const int col0 = C::NCG == 2 ? 32 * cg : 0;         // first query column of this group
     const int quarter = warp & 3;
     const int r = quarter * 32 + lane;  // key row within the tile
     const uint32_t tl = tbase + ((uint32_t)(quarter * 32) << 16);
@@ -651,42 +666,46 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       for (int s = 0; s < u.n; ++s) {
         const int g = gs + s;
         const int st = g % C::NSTAGE;
-        const int q0 = step_q0(u, s);
+        const int q0 = step_q0(u, s) + col0;  // first query row of this group's columns
         const uint32_t stats_bar = C::HALVES ? BAR(C::B_QBFULL) : BAR(C::B_QFULL + st);
         if (!mbar_wait_warp(stats_bar, (g / C::NSTAGE) & 1, wc, 21)) { ok = false; break; }
         if (!mbar_wait_warp(BAR(C::B_SFULL + (g & 1)), (g >> 1) & 1, wc, 22)) { ok = false; break; }
         tc_fence_after();
-        const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512);
+        const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512) + col0;
         const float* dv = lse2 + 64;
         uint32_t x0[32], x1[32];
         const int scol = C::ST_COL + 64 * (g & 1);
-        tmem_ld32(tl + scol, x0);
-        tmem_ld32(tl + scol + 32, x1);
+        tmem_ld32(tl + scol + col0, x0);
+        if (NC == 64) tmem_ld32(tl + scol + 32, x1);
         tmem_ld_wait();
         reg_fence(x0);
-        reg_fence(x1);
-        float pr[64];
+        if (NC == 64) reg_fence(x1);
+        float pr[NC];
         const bool diag = CAUSAL && (q0 < u.jt * C::BC + C::BC);
 #pragma unroll
         for (int c = 0; c < 32; ++c) {
           pr[c] = ex2(fmaf(__uint_as_float(x0[c]), sl2, -lse2[c]));
-          pr[32 + c] = ex2(fmaf(__uint_as_float(x1[c]), sl2, -lse2[32 + c]));
+          if (NC == 64) pr[(32 + c) % NC] = ex2(fmaf(__uint_as_float(x1[c]), sl2, -lse2[32 + c]));
         }
         if (diag) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < NC; ++c)
             if (key > q0 + c) pr[c] = 0.f;
         }
         // ragged N: keys and queries past the end of the sequence contribute nothing
-        if (TAIL && (key >= u.len || q0 + C::BR > u.len)) {
+        if (TAIL && (key >= u.len || q0 + NC > u.len)) {
 #pragma unroll
-          for (int c = 0; c < 64; ++c)
+          for (int c = 0; c < NC; ++c)
             if (key >= u.len || q0 + c >= u.len) pr[c] = 0.f;
         }
-        uint32_t pk[32];
+        uint32_t pk[NC / 2];
 #pragma unroll
-        for (int c = 0; c < 32; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
-        tmem_st32(tl + scol, pk);
+        for (int c = 0; c < NC / 2; ++c) pk[c] = pack_bf16(pr[2 * c], pr[2 * c + 1]);
+        if constexpr (NC == 64) {
+          tmem_st32(tl + scol, pk);
+        } else {
+          tmem_st16(tl + scol + col0, pk);
+        }
         tmem_st_wait();
         tc_fence_before();
         __syncwarp();
@@ -700,19 +719,20 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: bf16 over the
         // consumed dPᵀ columns (A operand of dK) and into the smem tile (dQᵀ)
 #pragma unroll
-        for (int hf = 0; hf < 2; ++hf) {
+        for (int h = 0; h < NC / 32; ++h) {
+          const int hf = C::NCG == 2 ? cg : h;  // which 32 of the step's 64 query columns
           tmem_ld32(tl + C::DP_COL + 32 * hf, x0);
           tmem_ld_wait();
           reg_fence(x0);
           uint32_t dk16[16];
 #pragma unroll
           for (int c = 0; c < 16; ++c) {
-            const int q = 32 * hf + 2 * c;
+            const int q = 32 * h + 2 * c;  // this group's column index
             const float d0 = pr[q] * (__uint_as_float(x0[2 * c]) - dv[q]);
             const float d1 = pr[q + 1] * (__uint_as_float(x0[2 * c + 1]) - dv[q + 1]);
             dk16[c] = pack_bf16(d0, d1);
           }
-          tmem_st16(tl + C::DP_COL + 16 * hf, dk16);
+          tmem_st16(tl + C::DP_COL + C::A_HALF * hf, dk16);
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int lch = 4 * hf + ch;
@@ -727,18 +747,21 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         if (lane == 0) mbar_arrive(BAR(C::B_DSFULL));
       }
       if (!ok) break;
-      // dK epilogue (scaled by s); tcgen05.ld is warp-collective: every lane
-      // loads, only rows < N are stored
+      // dK epilogue (scaled by s), this group's 32-column chunks of the CTA's
+      // output columns; tcgen05.ld is warp-collective: every lane loads, only
+      // rows < N are stored
       if (!mbar_wait_warp(BAR(C::B_ACC), uc & 1, wc, 25)) { ok = false; break; }
       tc_fence_after();
       __nv_bfloat16* dst = p.dk + ((size_t)bwd_kvrow<VARLEN>(u, p) + key) * D + u.dh * C::DH;
+      constexpr int NOC = C::DH / 32 / C::NCG;  // chunks per group
 #pragma unroll
-      for (int oc = 0; oc < C::DH / 32; ++oc) {
+      for (int h = 0; h < NOC; ++h) {
+        const int oc = cg * NOC + h;
         uint32_t v[32];
         tmem_ld32(tl + C::DK_COL + oc * 32, v);
         tmem_ld_wait();
         reg_fence(v);
-        if (oc == C::DH / 32 - 1) {
+        if (h == NOC - 1) {
           // dK has been read out of TMEM: the next unit may overwrite it
           tc_fence_before();
           __syncwarp();
@@ -757,7 +780,7 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
       gs += u.n;
     }
     tc_fence_before();
-  } else if (warp >= 8) {
+  } else {
     // ------------------------- drain: dQᵀ -> smem staging -> TMA reduce-add
     if (C::REG_SPLIT) setmaxnreg_inc<C::DRAIN_REGS>();
     const int quarter = warp & 3;
