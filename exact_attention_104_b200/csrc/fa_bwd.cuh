@@ -62,10 +62,15 @@ struct BwdCfg {
   static constexpr int Q_OFF = DS_OFF + 16384;
   static constexpr int DO_OFF = Q_OFF + NSTAGE * Q_BYTES;
   static constexpr int LS_OFF = DO_OFF + NSTAGE * Q_BYTES;  // per stage: lse2[64], Dvec[64]
-  // dQᵀ staging for the TMA reduce-add: STG_ROWS query rows x DH fp32, row-major
+  // dQᵀ staging for the TMA reduce-add: STG_ROWS query rows x DH fp32,
+  // row-major; at d = 64, where shared memory has room, two such buffers used
+  // alternately, so that the next step's dQᵀ is staged while the previous
+  // reduce still reads its buffer
   static constexpr int STG_ROWS = (D == 256) ? 32 : 64;
+  static constexpr int STG_NBUF = (D == 64) ? 2 : 1;
   static constexpr int STG_OFF = LS_OFF + NSTAGE * 512 + ((1024 - (NSTAGE * 512) % 1024) % 1024);
-  static constexpr int STG_BYTES = STG_ROWS * DH * 4;
+  static constexpr int STG_BUF = STG_ROWS * DH * 4;
+  static constexpr int STG_BYTES = STG_NBUF * STG_BUF;
   static constexpr int BAR_OFF = STG_OFF + STG_BYTES;
   static constexpr int B_KVFULL = 0;
   static constexpr int B_QFULL = 1;                  // + stage
@@ -813,24 +818,27 @@ __global__ void __launch_bounds__(BwdCfg<D>::THREADS, 1)
         const int q_row = bwd_qprow<VARLEN>(u, step_head(u, s), p) + step_q0(u, s);  // padded accumulator row
 #pragma unroll
         for (int sub = 0; sub < 64 / C::STG_ROWS; ++sub) {
-          // the previous reduce must have finished reading the staging tile
+          const int buf = C::STG_NBUF == 2 ? (sub_seq & 1) : 0;
+          // the reduce that last read this staging buffer must be done reading
+          // it (with two buffers the previous reduce may still be in flight)
           if (dt == 0) {
-            bulk_wait_read_all();
+            bulk_wait_read<C::STG_NBUF - 1>();
             mbar_arrive(BAR(C::B_STGFREE));
           }
           if (!mbar_wait_warp(BAR(C::B_STGFREE), sub_seq & 1, wc, 33)) { ok = false; break; }
+          float* sb = stg + buf * (C::STG_BUF / 4);
           if (r < C::DH) {
 #pragma unroll
             for (int qq = 0; qq < C::STG_ROWS; ++qq) {
               const int c = sub * C::STG_ROWS + qq;
-              stg[qq * C::DH + r] = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
+              sb[qq * C::DH + r] = __uint_as_float(c < 32 ? x0[c] : x1[c - 32]);
             }
           }
           fence_proxy_async_smem();
           mbar_arrive(BAR(C::B_STGFULL));
           if (dt == 0) {
             if (!mbar_wait(BAR(C::B_STGFULL), sub_seq & 1, wc, 34)) { ok = false; break; }
-            tma_reduce_add_2d(&tmDQ, sbase + C::STG_OFF, u.dh * C::DH, q_row + sub * C::STG_ROWS);
+            tma_reduce_add_2d(&tmDQ, sbase + C::STG_OFF + buf * C::STG_BUF, u.dh * C::DH, q_row + sub * C::STG_ROWS);
             bulk_commit_group();
           }
           ++sub_seq;
