@@ -273,7 +273,7 @@ template <int D, bool CAUSAL, bool TAIL, bool VARLEN>
 fa_status launch_bwd_kernel(const CUtensorMap& tq, const CUtensorMap& tk, const CUtensorMap& tv,
                             const CUtensorMap& tdo, const fa::BwdParams& p, uint64_t dq_rows, long long units,
                             int sms, cudaStream_t stream) {
-  using C = fa::BwdCfg<D>;
+  using C = fa::BwdCfgOf<D, CAUSAL>;
   auto kern = fa::fa_bwd_kernel<D, CAUSAL, TAIL, VARLEN>;
   if (C::REG_SPLIT && !reg_split_fits<C>(kern)) return FA_ERR_UNSUPPORTED;
   CUtensorMap tdq;
