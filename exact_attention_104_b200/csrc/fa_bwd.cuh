@@ -570,9 +570,13 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
           for (int s = 0; s < n && ok; ++s) {
             const int g = gs + s;
             const uint32_t st_t = tbase + C::ST_COL + 64 * (g & 1);
-            if (!mbar_wait_warp(BAR(C::B_HAFULL), g & 1, wc, 42)) { ok = false; break; }
-            tc_fence_after();
-            issue_xt_half(dK_k, dQ_k, st_t, oth, true);
+            if (s == 0) {
+              // a unit's first step; later steps' Sᵀ over half A was issued
+              // during the step before, after its dV product
+              if (!mbar_wait_warp(BAR(C::B_HAFULL), g & 1, wc, 42)) { ok = false; break; }
+              tc_fence_after();
+              issue_xt_half(dK_k, dQ_k, st_t, oth, true);
+            }
             if (!mbar_wait_warp(BAR(C::B_QBFULL), g & 1, wc, 43)) { ok = false; break; }
             tc_fence_after();
             issue_xt_half(dK_k, dQ_k, st_t, own, false);
@@ -587,6 +591,14 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
             if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DVFREE), (uc - 1) & 1, wc, 19)) { ok = false; break; }
             tc_fence_after();
             issue_acc(st_t, dDO_mn, tbase + C::DV_COL, s == 0);
+            if (s + 1 < n) {
+              // the next step's Sᵀ over half A (into the other Sᵀ buffer, whose
+              // Pᵀ the dV product two steps back has read) while the compute
+              // warps form dSᵀ: the tensor pipe would otherwise wait for them
+              if (!mbar_wait_warp(BAR(C::B_HAFULL), (g + 1) & 1, wc, 48)) { ok = false; break; }
+              tc_fence_after();
+              issue_xt_half(dK_k, dQ_k, tbase + C::ST_COL + 64 * ((g + 1) & 1), oth, true);
+            }
             if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
             if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
             tc_fence_after();

@@ -84,8 +84,9 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
     tiles are loaded in two halves: half A (the head-dimension panels outside
     the CTA's own output columns, last read by dPᵀ) and half B (the CTA's own
     panels and the per-row statistics, last read by the dK product); half B's
-    Q and dO complete on separate barriers.  Each step issues Sᵀ and dPᵀ over
-    half A, then over half B, and then dV, dK, dQᵀ."""
+    Q and dO complete on separate barriers.  Each step issues Sᵀ over half B,
+    dPᵀ over half A and B, dV, then the next step's Sᵀ over half A, then dK and
+    dQᵀ (a unit's first step issues its own Sᵀ over half A first)."""
     rnd = random.Random(seed)
     counter = [0]
     done_units = []
@@ -226,9 +227,11 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                 if halves:
                     for s in range(n):
                         g = gs + s
-                        yield from wait("HAFULL", g)
-                        assert ("QA", g) in loaded
-                        issue("S_A", uc, g)
+                        if s == 0:
+                            # later steps' Sᵀ over half A was issued during the previous step
+                            yield from wait("HAFULL", g)
+                            assert ("QA", g) in loaded
+                            issue("S_A", uc, g)
                         yield from wait("QBFULL", g)
                         assert ("QB", g) in loaded
                         issue("S_B", uc, g)
@@ -243,6 +246,11 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                         if s == 0 and uc > 0 and mistake != "no_dvfree_wait":
                             yield from wait("DVFREE", uc - 1)
                         issue("dV", uc, g)
+                        if s + 1 < n and mistake != "s_a_before_dv":
+                            # the next step's Sᵀ over half A fills the wait for dSᵀ
+                            yield from wait("HAFULL", g + 1)
+                            assert ("QA", g + 1) in loaded
+                            issue("S_A", uc, g + 1)
                         yield from wait("DSFULL", g)
                         if s == 0 and uc > 0:
                             yield from wait("DKFREE", uc - 1)
