@@ -20,7 +20,9 @@
 //   dV += Pᵀ dO, dK += dSᵀ Q       (A = bf16 Pᵀ / dSᵀ written back to TMEM)
 //   dQᵀ = Kᵀ dSᵀ                   (A = K tile read MN-major, B = dSᵀ in smem)
 // Roles: warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 4-7 compute
-// (thread = key row: Pᵀ, dSᵀ), warps 8-11 drain (thread = d row of dQᵀ).
+// (thread = key row: Pᵀ, dSᵀ), warps 8-11 drain (thread = d row of dQᵀ); at
+// d = 64 and for causal d = 128 warps 12-15 form a second compute warpgroup,
+// the two groups taking 32 query columns of each step each.
 // For d = 256, dK/dV/dQ do not fit TMEM for a full row, so two CTAs share a
 // key tile, each owning 128 of the 256 output columns and both recomputing Sᵀ
 // and dPᵀ over the full head dimension.
