@@ -54,6 +54,7 @@ __all__ = [
     "safe_softmax",
     "online_softmax",
     "blockwise_online_attention",
+    "blockwise_attention_lazy_rescale",
     "attention_forward",
     "attention_backward",
     "head_forward_rows",
@@ -166,6 +167,81 @@ def blockwise_online_attention(q, k, v, scale, kv_block, causal=False):
         m_prev, d_prev, o_prev = m_new, d_new, o_new
         start += size
     return o_prev, m_prev, d_prev
+
+
+def _lazy_rescale(o, l, m_ref, m_new):
+    """Move a row's accumulated output and normaliser from reference maximum
+    m_ref to m_new (both scaled by e^{m_ref - m_new}); rows without any term
+    yet (m_ref = -inf) hold zeros and stay zero."""
+    alpha = np.where(np.isfinite(m_ref), np.exp(np.where(np.isfinite(m_ref), m_ref, 0.0) - m_new), 0.0)
+    return alpha[:, None] * o, alpha * l
+
+
+def blockwise_attention_lazy_rescale(q, k, v, scale, kv_block, tau, causal=False):
+    """Blockwise attention with conditional rescaling, the FA4 technique that
+    P1 "Key observations" names without giving its rule.  The reading taken:
+    every row keeps a reference maximum m_ref and un-normalised accumulators
+    O and l, all relative to m_ref.  For each KV block j:
+
+      1. S_j = s·Q K_jᵀ (masked entries -inf), m_j = rowmax(S_j)
+      2. if m_ref = -inf or m_j > m_ref + tau: rescale O and l by
+         e^{m_ref - m_new} and set m_ref = m_new = max(m_ref, m_j)
+         (otherwise keep the stale m_ref)
+      3. O += exp(S_j - m_ref) V_j ;  l += Σ exp(S_j - m_ref)
+
+    and at the end O/l, LSE = m_ref + ln l.  Because O and l always share one
+    reference the result is the exact softmax for any tau >= 0; tau only
+    bounds every term exp(S_j - m_ref) by e^tau.  The pages give no threshold:
+    the kernels use 8 in base-2 units of the scaled scores, i.e.
+    tau = 8·ln 2 here.  ``kv_block`` is an int or a list of block sizes.
+    q: [M, d], k, v: [N, d].  Returns (O, LSE, rescales, max_term): the number
+    of rescalings of each row after its first term, and the largest term
+    exp(S_j - m_ref) met."""
+    q = np.asarray(q, np.float64)
+    k = np.asarray(k, np.float64)
+    v = np.asarray(v, np.float64)
+    n_keys = k.shape[0]
+    if isinstance(kv_block, int):
+        sizes = [kv_block] * (n_keys // kv_block)
+        if n_keys % kv_block:
+            sizes.append(n_keys % kv_block)
+    else:
+        sizes = list(kv_block)
+    assert sum(sizes) == n_keys and tau >= 0
+    rows = q.shape[0]
+    m_ref = np.full(rows, -np.inf)
+    l = np.zeros(rows)
+    o = np.zeros((rows, v.shape[1]))
+    rescales = np.zeros(rows, np.int64)
+    max_term = 0.0
+    start = 0
+    for size in sizes:
+        kj, vj = k[start:start + size], v[start:start + size]
+        s_j = scale * (q @ kj.T)                                       # step 1
+        if causal:
+            qi = np.arange(rows)[:, None]
+            kj_idx = (start + np.arange(size))[None, :]
+            s_j = np.where(kj_idx > qi, -np.inf, s_j)
+        m_j = s_j.max(axis=1)
+        need = np.isfinite(m_j) & (~np.isfinite(m_ref) | (m_j > m_ref + tau))   # step 2
+        if need.any():
+            m_new = np.where(need, np.maximum(m_ref, m_j), m_ref)
+            o_s, l_s = _lazy_rescale(o, l, m_ref, m_new)
+            o = np.where(need[:, None], o_s, o)
+            l = np.where(need, l_s, l)
+            rescales += (need & np.isfinite(m_ref)).astype(np.int64)
+            m_ref = m_new
+        live = np.isfinite(m_ref)
+        e = np.where(live[:, None], np.exp(s_j - np.where(live, m_ref, 0.0)[:, None]), 0.0)   # step 3
+        if e.size:
+            max_term = max(max_term, float(e.max()))
+        o = o + e @ vj
+        l = l + e.sum(axis=1)
+        start += size
+    with np.errstate(invalid="ignore", divide="ignore"):
+        out = np.where((l > 0)[:, None], o / l[:, None], 0.0)
+        lse = np.where(l > 0, m_ref + np.log(l), -np.inf)
+    return out, lse, rescales, max_term
 
 
 # ---------------------------------------------------------------------------

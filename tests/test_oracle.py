@@ -12,6 +12,9 @@ fix rather than against the oracle itself:
   and its autograd (the handbook page "FlashAttention", "如何使用 FlashAttention",
   names PyTorch SDPA as the standard entry point);
 * central finite differences and gradient invariants for the backward pass;
+* the conditional-rescale form of the blockwise update (the FA4 technique the
+  concept page lists) against the plain definition for several thresholds,
+  with both branches exercised and the e^tau bound on its terms;
 * planted mistakes in the oracle, which must make at least one pin fail.
 """
 
@@ -120,6 +123,66 @@ def test_blockwise_update_running_max_and_normaliser():
     s = 0.5 * q @ k.T
     np.testing.assert_allclose(m, s.max(axis=1), rtol=1e-15)
     np.testing.assert_allclose(dsum, np.exp(s - s.max(axis=1, keepdims=True)).sum(axis=1), rtol=1e-13)
+
+
+def _growing_logits(seed, N=48, d=8):
+    # keys whose scores against every query grow from block to block, so the
+    # row maximum moves up by several units per block (the rescale branch)
+    rng = np.random.default_rng(seed)
+    q = rng.normal(0, 1, (N, d))
+    q[:, 0] = np.abs(q[:, 0]) + 1.0
+    k = rng.normal(0, 1, (N, d))
+    k[:, 0] = np.linspace(0.0, 40.0, N)
+    v = rng.normal(0, 1, (N, d))
+    return q, k, v
+
+
+@pytest.mark.parametrize("causal", [False, True])
+@pytest.mark.parametrize("tau", [0.0, 0.7, 8 * math.log(2), 1e3])
+def test_lazy_rescale_equals_two_pass(causal, tau):
+    # conditional rescaling keeps O and l on one reference, so the result is
+    # the plain definition for any threshold (exactness, P1 "Core idea")
+    cases = [_growing_logits(11), (_rand((40, 8), 12, 3.0), _rand((40, 8), 13, 3.0), _rand((40, 8), 14))]
+    for q, k, v in cases:
+        scale = 1 / math.sqrt(q.shape[1])
+        o_ref, lse_ref, _ = oracle.head_forward_rows(q, k, v, scale, causal)
+        ragged = [5, 11, 7, 1, q.shape[0] - 24]  # uneven blocks, one of a single key
+        for sizes in (16, ragged, 1):
+            o, lse, _, _ = oracle.blockwise_attention_lazy_rescale(q, k, v, scale, sizes, tau, causal)
+            np.testing.assert_allclose(o, o_ref, rtol=1e-11, atol=1e-12)
+            np.testing.assert_allclose(lse, lse_ref, rtol=1e-12, atol=1e-12)
+
+
+def test_lazy_rescale_branches_and_term_bound():
+    q, k, v = _growing_logits(21)
+    scale = 1 / math.sqrt(q.shape[1])
+    # tau = 0: a rescale at every block whose row maximum is larger
+    _, _, r0, t0 = oracle.blockwise_attention_lazy_rescale(q, k, v, scale, 8, 0.0)
+    assert r0.min() >= 1 and t0 <= 1.0 + 1e-12
+    # a threshold above the whole score range: the first block's maximum stays
+    # the reference, and terms then exceed 1 (up to e^tau)
+    _, _, r1, t1 = oracle.blockwise_attention_lazy_rescale(q, k, v, scale, 8, 1e3)
+    assert r1.max() == 0 and t1 > 1.0
+    # the kernels' threshold: some rows rescale, fewer times than with tau = 0,
+    # and no term exceeds e^tau
+    tau = 8 * math.log(2)
+    _, _, r2, t2 = oracle.blockwise_attention_lazy_rescale(q, k, v, scale, 8, tau)
+    assert 0 < r2.sum() < r0.sum() and t2 <= math.exp(tau) * (1 + 1e-12)
+
+
+def test_planted_lazy_rescale_mistake_is_caught(monkeypatch):
+    # rescaling O but not the normaliser l must break exactness
+    def only_o(o, l, m_ref, m_new):
+        o2, _ = _orig_lazy_rescale(o, l, m_ref, m_new)
+        return o2, l
+    _orig_lazy_rescale = oa._lazy_rescale
+    monkeypatch.setattr(oa, "_lazy_rescale", only_o)
+    q, k, v = _growing_logits(31)
+    scale = 1 / math.sqrt(q.shape[1])
+    o_ref, lse_ref, _ = oracle.head_forward_rows(q, k, v, scale, False)
+    o, lse, r, _ = oracle.blockwise_attention_lazy_rescale(q, k, v, scale, 8, 0.0)
+    assert r.sum() > 0
+    assert np.abs(lse - lse_ref).max() > 1e-3 or np.abs(o - o_ref).max() > 1e-3
 
 
 # ---------------------------------------------------------------------------
