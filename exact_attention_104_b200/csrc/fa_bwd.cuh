@@ -18,11 +18,13 @@
 // In fa_bwd_kernel every product runs on tcgen05 with fp32 TMEM accumulators:
 //   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ        (A, B from shared memory)
 //   dV += Pᵀ dO, dK += dSᵀ Q       (A = bf16 Pᵀ / dSᵀ written back to TMEM)
-//   dQᵀ = Kᵀ dSᵀ                   (A = K tile read MN-major, B = dSᵀ in smem)
+//   dQᵀ = Kᵀ dSᵀ                   (B = dSᵀ in smem; A = Kᵀ in TMEM at d <= 128,
+//                                  the K tile read MN-major at d = 256)
 // Roles: warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 4-7 compute
-// (thread = key row: Pᵀ, dSᵀ), warps 8-11 drain (thread = d row of dQᵀ); at
-// d = 64 and for causal d = 128 warps 12-15 form a second compute warpgroup,
-// the two groups taking 32 query columns of each step each.
+// (thread = key row: Pᵀ, dSᵀ), warps 8-11 drain (thread = d row of dQᵀ; at
+// d <= 128 they also write each unit's Kᵀ into TMEM); at d = 64 and for
+// causal d = 128 warps 12-15 form a second compute warpgroup, the two groups
+// taking 32 query columns of each step each.
 // For d = 256, dK/dV/dQ do not fit TMEM for a full row, so two CTAs share a
 // key tile, each owning 128 of the 256 output columns and both recomputing Sᵀ
 // and dPᵀ over the full head dimension.
@@ -51,7 +53,15 @@ struct BwdCfg {
   static constexpr int KV_BYTES = BC * D * 2;
   static constexpr int Q_BYTES = BR * D * 2;
   static constexpr int NSTAGE = (D == 64) ? 4 : (D == 128 ? 3 : 1);
-  static constexpr int LA = NSTAGE >= 2 ? 2 : 1;  // Sᵀ lookahead in steps
+  // dQᵀ = Kᵀ dSᵀ reads Kᵀ from TMEM (A operand of a TS product) instead of the
+  // K tile in shared memory at every step: the drain warps write it once per
+  // unit (32 KB less shared-memory traffic per step at d = 128).  At d = 64
+  // TMEM has 64 columns to spare; at d = 128 they are the second Sᵀ buffer,
+  // so Sᵀ is single-buffered there and each step's Sᵀ is issued right after
+  // the previous step's dV product (the last reader of the buffer).
+  static constexpr bool KT_TMEM = (D <= 128);
+  static constexpr int ST_NBUF = (D == 128) ? 1 : 2;
+  static constexpr int LA = (NSTAGE >= 2 && ST_NBUF == 2) ? 2 : 1;  // Sᵀ lookahead in steps
   // d = 256 (one stage): a step's Q and dO tiles load in two halves.  Half A
   // is the two 64-column panels outside the CTA's own output columns (read
   // only by Sᵀ and dPᵀ, so it is free once dPᵀ is done); half B is the CTA's
@@ -98,21 +108,27 @@ struct BwdCfg {
   static constexpr int B_QBFULL = B_HAEMPTY + 1;  // half B of Q and the row statistics loaded
   static constexpr int B_DOBFULL = B_QBFULL + 1;  // half B of dO loaded
   static constexpr int B_HBEMPTY = B_DOBFULL + 1; // half B read by the dV and dK products
-  static constexpr int NBAR = B_HBEMPTY + 1;
+  static constexpr int B_KTFULL = B_HBEMPTY + 1;  // a unit's Kᵀ written into TMEM
+  static constexpr int NBAR = B_KTFULL + 1;
   static constexpr int MISC_OFF = BAR_OFF + NBAR * 8;
   static constexpr int UNIT_OFF = MISC_OFF + 16;   // two unit-index slots
   static constexpr int SMEM_BYTES = UNIT_OFF + 16 + 1024;
   static constexpr int TMEM_COLS = 512;
   static constexpr int DK_COL = 0;
   static constexpr int DV_COL = DH;
-  static constexpr int ST_COL = 2 * DH;        // two 64-column Sᵀ buffers
+  static constexpr int ST_COL = 2 * DH;        // ST_NBUF 64-column Sᵀ buffers
   static constexpr int DP_COL = 2 * DH + 128;  // dPᵀ (later dSᵀ bf16)
   static constexpr int DQ_COL = 2 * DH + 192;  // dQᵀ
+  // Kᵀ (bf16, two keys per column): the free columns after dQᵀ at d = 64, the
+  // unused second Sᵀ buffer at d = 128
+  static constexpr int KT_COL = ST_NBUF == 2 ? 2 * DH + 256 : 2 * DH + 64;
   static constexpr uint32_t IDESC_ST = idesc_bf16_f32(128, BR, false, false);
   static constexpr uint32_t IDESC_DKV = idesc_bf16_f32(128, DH, false, true);
   static constexpr uint32_t IDESC_DQ = idesc_bf16_f32(128, BR, true, true);
+  static constexpr uint32_t IDESC_DQ_TS = idesc_bf16_f32(128, BR, false, true);
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
   static_assert(DQ_COL + 64 <= TMEM_COLS, "TMEM budget");
+  static_assert(!KT_TMEM || (KT_COL + 64 <= TMEM_COLS && (ST_NBUF == 1 || KT_COL >= DQ_COL + 64)), "TMEM budget (Kᵀ)");
   // Register split between the warpgroups (control: setmaxnreg.dec; compute
   // and drain: setmaxnreg.inc).  Valid for a launch allocation R with
   // CTRL_REGS <= R <= min(COMPUTE_REGS, DRAIN_REGS) and
@@ -373,6 +389,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
     }
     mbar_init(BAR(C::B_DRAIN), 1);
     for (int i = C::B_HAFULL; i <= C::B_HBEMPTY; ++i) mbar_init(BAR(i), 1);
+    mbar_init(BAR(C::B_KTFULL), 4);
     *abort_flag = 0;
     fence_mbar_init();
   }
@@ -551,10 +568,17 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
         // dQᵀ [128 d-rows x 64 queries] = K[:, dh half]ᵀ · dSᵀ over the 128 keys
         auto issue_dq = [&]() {
 #pragma unroll
-          for (int kk = 0; kk < C::BC / 16; ++kk)
-            mma_ss_w(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
-                   kk > 0 ? 1u : 0u);
+          for (int kk = 0; kk < C::BC / 16; ++kk) {
+            if constexpr (C::KT_TMEM)
+              mma_ts_w(tbase + C::DQ_COL, tbase + C::KT_COL + kk * 8, sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ_TS,
+                       kk > 0 ? 1u : 0u);
+            else
+              mma_ss_w(tbase + C::DQ_COL, sdesc_add(dKT_mn, kk * 2048), sdesc_add(dDS_mn, kk * 2048), C::IDESC_DQ,
+                       kk > 0 ? 1u : 0u);
+          }
         };
+        // Sᵀ buffer of step g
+        auto st_col = [&](int g) -> uint32_t { return tbase + C::ST_COL + (C::ST_NBUF == 2 ? 64 * (g & 1) : 0); };
         if (!mbar_wait_warp(BAR(C::B_KVFULL), uc & 1, wc, 12)) { ok = false; break; }
         tc_fence_after();
         if constexpr (C::HALVES) {
@@ -617,7 +641,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
           for (int k = 0; k < C::LA && k < n && ok; ++k) {
             ok = wait_q(gs + k);
             if (!ok) break;
-            issue_xt(dK_k, q_off(gs + k), tbase + C::ST_COL + 64 * ((gs + k) & 1));
+            issue_xt(dK_k, q_off(gs + k), st_col(gs + k));
             tc_commit_w(BAR(C::B_SFULL + ((gs + k) & 1)));
           }
           if (!ok) break;
@@ -629,7 +653,14 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
             // the previous unit's dV must have been read out before it is overwritten
             if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DVFREE), (uc - 1) & 1, wc, 19)) { ok = false; break; }
             tc_fence_after();
-            issue_acc(tbase + C::ST_COL + 64 * (g & 1), sdesc_add(dDO_mn, stage_bytes(g)), tbase + C::DV_COL, s == 0);
+            issue_acc(st_col(g), sdesc_add(dDO_mn, stage_bytes(g)), tbase + C::DV_COL, s == 0);
+            if (C::ST_NBUF == 1 && s + 1 < n) {
+              // one Sᵀ buffer: the next step's Sᵀ right after dV, the last
+              // reader of this step's Pᵀ in it
+              if (!wait_q(g + 1)) { ok = false; break; }
+              issue_xt(dK_k, q_off(g + 1), st_col(g + 1));
+              tc_commit_w(BAR(C::B_SFULL + ((g + 1) & 1)));
+            }
             if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
             if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
             tc_fence_after();
@@ -639,15 +670,20 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
               if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
               tc_fence_after();
             }
+            if (C::KT_TMEM && s == 0) {
+              // this unit's Kᵀ is in TMEM
+              if (!mbar_wait_warp(BAR(C::B_KTFULL), uc & 1, wc, 28)) { ok = false; break; }
+              tc_fence_after();
+            }
             issue_dq();
             tc_commit_w(BAR(C::B_DQFULL));
             // dPᵀ of the next step first: the compute warps are waiting for it
             if (s + 1 < n) {
-              if (C::LA == 1 && !wait_q(g + 1)) { ok = false; break; }
+              if (C::LA == 1 && C::ST_NBUF == 2 && !wait_q(g + 1)) { ok = false; break; }
               issue_xt(dV_k, do_off(g + 1), tbase + C::DP_COL);
               tc_commit_w(BAR(C::B_DPFULL));
             }
-            if (s + C::LA < n) {
+            if (C::ST_NBUF == 2 && s + C::LA < n) {
               const int g2 = g + C::LA;
               if (C::LA > 1 && !wait_q(g2)) { ok = false; break; }
               issue_xt(dK_k, q_off(g2), tbase + C::ST_COL + 64 * (g2 & 1));
@@ -700,7 +736,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
         const float* lse2 = reinterpret_cast<const float*>(smem + C::LS_OFF + st * 512) + col0;
         const float* dv = lse2 + 64;
         uint32_t x0[32], x1[32];
-        const int scol = C::ST_COL + 64 * (g & 1);
+        const int scol = C::ST_COL + (C::ST_NBUF == 2 ? 64 * (g & 1) : 0);
         tmem_ld32(tl + scol + col0, x0);
         if (NC == 64) tmem_ld32(tl + scol + 32, x1);
         tmem_ld_wait();
@@ -823,6 +859,33 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
       if (idx < 0) { ok = false; break; }
       if (idx >= n_units) break;
       const BwdUnit u = bwd_unit<D, CAUSAL, VARLEN>(idx, p, ne);
+      if constexpr (C::KT_TMEM) {
+        // Kᵀ into TMEM, the A operand of the unit's dQᵀ products: lane r holds
+        // column r of the K tile, keys 2c and 2c + 1 in column c (low half
+        // first), gathered from the 128B-swizzled tile.  The previous unit's
+        // last dQᵀ is complete: its K tile was replaced only after that.
+        if (!mbar_wait_warp(BAR(C::B_KVFULL), uc & 1, wc, 29)) { ok = false; break; }
+        if (quarter * 32 < C::DH) {
+          const uint8_t* kp = smem + C::K_OFF + (r >> 6) * C::KV_PANEL + (r & 7) * 2;
+          const int cb = (r & 63) >> 3;  // 16-byte chunk of column r in a key row
+#pragma unroll
+          for (int h = 0; h < 2; ++h) {
+            uint32_t w[32];
+#pragma unroll
+            for (int c = 0; c < 32; ++c) {
+              const int k0 = 64 * h + 2 * c;
+              const uint32_t lo = *reinterpret_cast<const uint16_t*>(kp + k0 * 128 + ((cb ^ (k0 & 7)) << 4));
+              const uint32_t hi = *reinterpret_cast<const uint16_t*>(kp + (k0 + 1) * 128 + ((cb ^ ((k0 + 1) & 7)) << 4));
+              w[c] = lo | (hi << 16);
+            }
+            tmem_st32(tl + C::KT_COL + 32 * h, w);
+          }
+          tmem_st_wait();
+        }
+        tc_fence_before();
+        __syncwarp();
+        if (lane == 0) mbar_arrive(BAR(C::B_KTFULL));
+      }
       for (int s = 0; s < u.n && ok; ++s) {
         const int g = gs + s;
         if (!mbar_wait_warp(BAR(C::B_DQFULL), g & 1, wc, 31)) { ok = false; break; }

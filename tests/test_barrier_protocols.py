@@ -74,7 +74,8 @@ def _run(gens, engines, rnd, max_steps=20_000_000):
 
 
 # ---------------------------------------------------------------- backward
-def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halves=False):
+def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halves=False, kt_tmem=False,
+                 st_single=False):
     """fa_bwd_kernel: ``n_ctas`` persistent CTAs claim units (``unit_len[i]`` query
     steps each) from one counter.  Roles per CTA: the producer (lane 0 of warp
     0), the MMA warp, four compute warps and four drain warps.  ``lookahead`` is
@@ -86,7 +87,17 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
     panels and the per-row statistics, last read by the dK product); half B's
     Q and dO complete on separate barriers.  Each step issues Sᵀ over half B,
     dPᵀ over half A and B, dV, then the next step's Sᵀ over half A, then dK and
-    dQᵀ (a unit's first step issues its own Sᵀ over half A first)."""
+    dQᵀ (a unit's first step issues its own Sᵀ over half A first).
+
+    ``kt_tmem`` models Kᵀ in TMEM: at the start of each unit the four drain
+    warps wait for the unit's K tile, write Kᵀ into TMEM and arrive on KTFULL,
+    which the MMA warp waits for before the unit's first dQᵀ; the model checks
+    that no dQᵀ reads a Kᵀ not yet fully written and that no Kᵀ is overwritten
+    while a dQᵀ of the unit before may still read it.  ``st_single`` models one
+    Sᵀ buffer (lookahead 1): each step's Sᵀ is issued right after the previous
+    step's dV.  For both Sᵀ layouts the model checks that an Sᵀ product
+    completes only after the compute warps handed over the Pᵀ it overwrites and
+    the dV product that read it completed."""
     rnd = random.Random(seed)
     counter = [0]
     done_units = []
@@ -105,6 +116,7 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
             bars["QEMPTY", i] = _Bar(1)
         for nm in ("HAFULL", "HAEMPTY", "QBFULL", "DOBFULL", "HBEMPTY"):
             bars[nm] = _Bar(1)
+        bars["KTFULL"] = _Bar(4)
         for i in range(2):
             bars["SFULL", i] = _Bar(1)
             bars["PFULL", i] = _Bar(4)
@@ -121,12 +133,22 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
         half_readers = {}           # (panel pair, g) -> products reading those panels of step g
         step_dh = {}                # g -> the output-column half of step g's unit
         stats_read = {}             # g -> compute warps done with step g's row statistics
+        p_handed = {}               # g -> compute warps that handed over step g's Pᵀ
+        dv_prod = {}                # g -> id of step g's dV product
+        kt_writes = {}              # uc -> drain warps that wrote the unit's Kᵀ
+        kt_readers = {}             # uc -> the unit's dQᵀ products
+        prod_info = {}
         prod_id = [0]
 
         def issue(kind, uc, g):
             prod_id[0] += 1
             i = prod_id[0]
             tc.append(("mma", i))
+            prod_info[i] = (kind, uc, g)
+            if kind == "dV":
+                dv_prod[g] = i
+            if kind == "dQ" and kt_tmem:
+                kt_readers.setdefault(uc, set()).add(i)
             if kind in ("S", "dP", "dQ", "S_A", "S_B", "dP_A", "dP_B"):
                 kv_readers.setdefault(uc, set()).add(i)
             if kind in ("S", "dP", "dV", "dK"):
@@ -274,10 +296,19 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                 commit("DPFULL")
                 for s in range(n):
                     g = gs + s
+                    if st_single and mistake == "s_before_dv" and s + 1 < n:
+                        yield from wait_q(g + 1)
+                        issue("S", uc, g + 1)
+                        commit(("SFULL", (g + 1) & 1))
                     yield from wait(("PFULL", g & 1), g >> 1)
                     if s == 0 and uc > 0 and mistake != "no_dvfree_wait":
                         yield from wait("DVFREE", uc - 1)
                     issue("dV", uc, g)
+                    if st_single and mistake != "s_before_dv" and s + 1 < n:
+                        # one Sᵀ buffer: the next step's Sᵀ right after dV
+                        yield from wait_q(g + 1)
+                        issue("S", uc, g + 1)
+                        commit(("SFULL", (g + 1) & 1))
                     yield from wait("DSFULL", g)
                     if s == 0 and uc > 0:
                         yield from wait("DKFREE", uc - 1)
@@ -285,14 +316,16 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                     commit(("QEMPTY", g % n_stage))
                     if g > 0:
                         yield from wait("DQEMPTY", g - 1)
+                    if kt_tmem and s == 0 and mistake != "no_ktfull_wait":
+                        yield from wait("KTFULL", uc)
                     issue("dQ", uc, g)
                     commit("DQFULL")
                     if s + 1 < n:
-                        if lookahead == 1:
+                        if lookahead == 1 and not st_single:
                             yield from wait_q(g + 1)
                         issue("dP", uc, g + 1)
                         commit("DPFULL")
-                    if s + lookahead < n:
+                    if not st_single and s + lookahead < n:
                         g2 = g + lookahead
                         if lookahead > 1:
                             yield from wait_q(g2)
@@ -312,6 +345,14 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                 if idx >= len(unit_len):
                     return
                 n = unit_len[idx]
+                if kind == "dV" and kt_tmem:
+                    if mistake != "kt_before_kvfull":
+                        yield from wait("KVFULL", uc)
+                    assert ("KV", uc) in loaded, f"Kᵀ of unit {uc} read from an unloaded K tile"
+                    assert kt_readers.get(uc - 1, set()) <= completed, f"Kᵀ of unit {uc - 1} overwritten while read"
+                    yield
+                    kt_writes[uc] = kt_writes.get(uc, 0) + 1
+                    bars["KTFULL"].arrive()
                 for s in range(n):
                     g = gs + s
                     if kind == "dK":
@@ -322,6 +363,7 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                             yield from wait(("QFULL", g % n_stage), g // n_stage)
                         yield from wait(("SFULL", g & 1), g >> 1)
                         yield
+                        p_handed[g] = p_handed.get(g, 0) + 1
                         bars["PFULL", g & 1].arrive()
                         yield from wait("DPFULL", g)
                         if g > 0:
@@ -341,12 +383,23 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                 gs += n
                 uc += 1
 
+        nbuf = 1 if st_single else 2
+
         def tc_done(item):
             kind, x = item
             if kind == "commit":
                 bars[x].arrive()
-            else:
-                completed.add(x)
+                return
+            pk, puc, pg = prod_info[x]
+            if pk == "S":
+                # the Sᵀ buffer's previous content: Pᵀ of step pg - nbuf
+                gp = pg - nbuf
+                if gp in dv_prod or p_handed.get(gp, 0):
+                    assert p_handed.get(gp, 0) == 4, f"Sᵀ of step {pg} overwrites Pᵀ of step {gp} being written"
+                    assert dv_prod.get(gp) in completed, f"Sᵀ of step {pg} overwrites Pᵀ of step {gp} before dV read it"
+            if pk == "dQ" and kt_tmem:
+                assert kt_writes.get(puc, 0) == 4, f"dQᵀ of unit {puc} read a Kᵀ not fully written"
+            completed.add(x)
 
         def tma_done(item):
             bar, what = item
@@ -392,6 +445,26 @@ def test_backward_model_catches_a_missing_wait(mistake):
     for seed in range(40):
         try:
             simulate_bwd([1, 1, 1, 1, 1, 1], 2, 3, 2, seed, mistake)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
+
+
+@pytest.mark.parametrize("n_stage,kt_tmem,st_single", [(4, True, False), (3, True, True), (3, False, True)])
+@pytest.mark.parametrize("n_ctas", [1, 3])
+def test_backward_protocol_kt_tmem_and_single_s_buffer(n_stage, kt_tmem, st_single, n_ctas):
+    # d = 64: Kᵀ in TMEM, two Sᵀ buffers; d = 128: Kᵀ in TMEM, one Sᵀ buffer
+    for units in BWD_UNITS:
+        for seed in range(4):
+            simulate_bwd(units, n_ctas, n_stage, 1 if st_single else 2, seed, kt_tmem=kt_tmem, st_single=st_single)
+
+
+@pytest.mark.parametrize("mistake", ["no_ktfull_wait", "kt_before_kvfull", "s_before_dv"])
+def test_backward_kt_tmem_model_catches_a_missing_wait(mistake):
+    caught = 0
+    for seed in range(40):
+        try:
+            simulate_bwd([2, 1, 3, 1, 2, 1], 2, 3, 1, seed, mistake, kt_tmem=True, st_single=True)
         except AssertionError:
             caught += 1
     assert caught > 0
