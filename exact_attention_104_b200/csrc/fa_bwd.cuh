@@ -17,7 +17,8 @@
 //
 // In fa_bwd_kernel every product runs on tcgen05 with fp32 TMEM accumulators:
 //   Sᵀ = K Qᵀ, dPᵀ = V dOᵀ        (A, B from shared memory)
-//   dV += Pᵀ dO, dK += dSᵀ Q       (A = bf16 Pᵀ / dSᵀ written back to TMEM)
+//   dV += Pᵀ dO, dK += dSᵀ Q       (A = bf16 Pᵀ / dSᵀ written back to TMEM; at
+//                                  d = 64 dK reads dSᵀ from shared memory)
 //   dQᵀ = Kᵀ dSᵀ                   (B = dSᵀ in smem; A = Kᵀ in TMEM at d <= 128,
 //                                  the K tile read MN-major at d = 256)
 // Roles: warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 4-7 compute
@@ -62,6 +63,11 @@ struct BwdCfg {
   static constexpr bool KT_TMEM = (D <= 128);
   static constexpr int ST_NBUF = (D == 128) ? 1 : 2;
   static constexpr int LA = (NSTAGE >= 2 && ST_NBUF == 2) ? 2 : 1;  // Sᵀ lookahead in steps
+  // dK += dSᵀ Q with dSᵀ read from the shared-memory tile the dQᵀ product uses
+  // (an SS product) instead of a bf16 copy in TMEM: at d = 64 this saved the
+  // compute warps' TMEM store and was 2.7 % faster; at d = 128 it was no
+  // faster (C3, C4) or slower (C2 +3.5 %), same box, alternated.
+  static constexpr bool DK_SS = (D == 64);
   // d = 256 (one stage): a step's Q and dO tiles load in two halves.  Half A
   // is the two 64-column panels outside the CTA's own output columns (read
   // only by Sᵀ and dPᵀ, so it is free once dPᵀ is done); half B is the CTA's
@@ -538,6 +544,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
       const uint64_t dQ_k = sdesc_sw128(sbase + C::Q_OFF, 16, 1024);
       const uint64_t dDO_k = sdesc_sw128(sbase + C::DO_OFF, 16, 1024);
       const uint64_t dDS_mn = sdesc_sw128(sbase + C::DS_OFF, 16384, 1024);
+      const uint64_t dDS_k = sdesc_sw128(sbase + C::DS_OFF, 16, 1024);
       // Sᵀ / dPᵀ: [128 keys x 64 queries] = (K or V tile) · (Q or dO tile)ᵀ over D
       auto issue_xt = [&](uint64_t da0, uint64_t db0, uint32_t dtm) {
 #pragma unroll
@@ -551,6 +558,17 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
         for (int kk = 0; kk < C::BR / 16; ++kk)
           mma_ts_w(dtm, atm + (kk >> 1) * C::A_HALF + (kk & 1) * 8, sdesc_add(db0, kk * 2048), C::IDESC_DKV,
                    (!first || kk > 0) ? 1u : 0u);
+      };
+      // dK += dSᵀ · Q tile[:, dh half], dSᵀ from TMEM or (DK_SS) from shared memory
+      auto issue_dk = [&](uint64_t db0, bool first) {
+        if constexpr (C::DK_SS) {
+#pragma unroll
+          for (int kk = 0; kk < C::BR / 16; ++kk)
+            mma_ss_w(tbase + C::DK_COL, sdesc_add(dDS_k, kk * 32), sdesc_add(db0, kk * 2048), C::IDESC_DKV,
+                     (!first || kk > 0) ? 1u : 0u);
+        } else {
+          issue_acc(tbase + C::DP_COL, db0, tbase + C::DK_COL, first);
+        }
       };
       auto stage_bytes = [&](int g) -> uint32_t { return (uint32_t)(g % C::NSTAGE) * C::Q_BYTES; };
       auto q_off = [&](int g) -> uint64_t { return sdesc_add(dQ_k, stage_bytes(g)); };
@@ -628,7 +646,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
             if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
             if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
             tc_fence_after();
-            issue_acc(tbase + C::DP_COL, dQ_mn, tbase + C::DK_COL, s == 0);
+            issue_dk(dQ_mn, s == 0);
             tc_commit_w(BAR(C::B_HBEMPTY));
             if (g > 0) {
               if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
@@ -664,7 +682,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
             if (!mbar_wait_warp(BAR(C::B_DSFULL), g & 1, wc, 15)) { ok = false; break; }
             if (s == 0 && uc > 0 && !mbar_wait_warp(BAR(C::B_DKFREE), (uc - 1) & 1, wc, 20)) { ok = false; break; }
             tc_fence_after();
-            issue_acc(tbase + C::DP_COL, sdesc_add(dQ_mn, stage_bytes(g)), tbase + C::DK_COL, s == 0);
+            issue_dk(sdesc_add(dQ_mn, stage_bytes(g)), s == 0);
             tc_commit_w(BAR(C::B_QEMPTY + g % C::NSTAGE));
             if (g > 0) {
               if (!mbar_wait_warp(BAR(C::B_DQEMPTY), (g - 1) & 1, wc, 16)) { ok = false; break; }
@@ -778,8 +796,9 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
         if (g > 0 && !mbar_wait_warp(BAR(C::B_DQFULL), (g - 1) & 1, wc, 24)) { ok = false; break; }
         tc_fence_after();
         uint8_t* rowp = smem + C::DS_OFF + r * 128;
-        // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: bf16 over the
-        // consumed dPᵀ columns (A operand of dK) and into the smem tile (dQᵀ)
+        // dSᵀ = Pᵀ ∘ (dPᵀ − D), 32 query columns at a time: bf16 into the smem
+        // tile (B operand of dQᵀ; A operand of dK with DK_SS) and, without
+        // DK_SS, over the consumed dPᵀ columns (A operand of dK)
 #pragma unroll
         for (int h = 0; h < NC / 32; ++h) {
           const int hf = C::NCG == 2 ? cg : h;  // which 32 of the step's 64 query columns
@@ -794,7 +813,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
             const float d1 = pr[q + 1] * (__uint_as_float(x0[2 * c + 1]) - dv[q + 1]);
             dk16[c] = pack_bf16(d0, d1);
           }
-          tmem_st16(tl + C::DP_COL + C::A_HALF * hf, dk16);
+          if (!C::DK_SS) tmem_st16(tl + C::DP_COL + C::A_HALF * hf, dk16);
 #pragma unroll
           for (int ch = 0; ch < 4; ++ch) {
             const int lch = 4 * hf + ch;

@@ -75,7 +75,7 @@ def _run(gens, engines, rnd, max_steps=20_000_000):
 
 # ---------------------------------------------------------------- backward
 def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halves=False, kt_tmem=False,
-                 st_single=False):
+                 st_single=False, dk_ss=False):
     """fa_bwd_kernel: ``n_ctas`` persistent CTAs claim units (``unit_len[i]`` query
     steps each) from one counter.  Roles per CTA: the producer (lane 0 of warp
     0), the MMA warp, four compute warps and four drain warps.  ``lookahead`` is
@@ -97,7 +97,10 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
     Sᵀ buffer (lookahead 1): each step's Sᵀ is issued right after the previous
     step's dV.  For both Sᵀ layouts the model checks that an Sᵀ product
     completes only after the compute warps handed over the Pᵀ it overwrites and
-    the dV product that read it completed."""
+    the dV product that read it completed.  The compute warps overwrite the
+    shared-memory dSᵀ tile of a step only after the previous step's readers of
+    it completed: its dQᵀ product and, with ``dk_ss`` (dK reading dSᵀ from
+    shared memory), its dK product."""
     rnd = random.Random(seed)
     counter = [0]
     done_units = []
@@ -137,6 +140,7 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
         dv_prod = {}                # g -> id of step g's dV product
         kt_writes = {}              # uc -> drain warps that wrote the unit's Kᵀ
         kt_readers = {}             # uc -> the unit's dQᵀ products
+        ds_readers = {}             # g -> products reading step g's shared-memory dSᵀ tile
         prod_info = {}
         prod_id = [0]
 
@@ -149,6 +153,8 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                 dv_prod[g] = i
             if kind == "dQ" and kt_tmem:
                 kt_readers.setdefault(uc, set()).add(i)
+            if kind == "dQ" or (kind == "dK" and dk_ss):
+                ds_readers.setdefault(g, set()).add(i)
             if kind in ("S", "dP", "dQ", "S_A", "S_B", "dP_A", "dP_B"):
                 kv_readers.setdefault(uc, set()).add(i)
             if kind in ("S", "dP", "dV", "dK"):
@@ -312,8 +318,10 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                     yield from wait("DSFULL", g)
                     if s == 0 and uc > 0:
                         yield from wait("DKFREE", uc - 1)
-                    issue("dK", uc, g)
-                    commit(("QEMPTY", g % n_stage))
+                    late_dk = mistake == "dk_after_next_dp"
+                    if not late_dk:
+                        issue("dK", uc, g)
+                        commit(("QEMPTY", g % n_stage))
                     if g > 0:
                         yield from wait("DQEMPTY", g - 1)
                     if kt_tmem and s == 0 and mistake != "no_ktfull_wait":
@@ -325,6 +333,9 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                             yield from wait_q(g + 1)
                         issue("dP", uc, g + 1)
                         commit("DPFULL")
+                    if late_dk:
+                        issue("dK", uc, g)
+                        commit(("QEMPTY", g % n_stage))
                     if not st_single and s + lookahead < n:
                         g2 = g + lookahead
                         if lookahead > 1:
@@ -368,6 +379,7 @@ def simulate_bwd(unit_len, n_ctas, n_stage, lookahead, seed, mistake=None, halve
                         yield from wait("DPFULL", g)
                         if g > 0:
                             yield from wait("DQFULL", g - 1)
+                            assert ds_readers.get(g - 1, set()) <= completed, f"dSᵀ tile of step {g - 1} overwritten while read"
                         yield
                         stats_read[g] = stats_read.get(g, 0) + 1
                         bars["DSFULL"].arrive()
@@ -457,6 +469,24 @@ def test_backward_protocol_kt_tmem_and_single_s_buffer(n_stage, kt_tmem, st_sing
     for units in BWD_UNITS:
         for seed in range(4):
             simulate_bwd(units, n_ctas, n_stage, 1 if st_single else 2, seed, kt_tmem=kt_tmem, st_single=st_single)
+
+
+@pytest.mark.parametrize("n_ctas", [1, 3])
+def test_backward_protocol_dk_from_shared_memory(n_ctas):
+    # d = 64: dK reads dSᵀ from the shared-memory tile, Kᵀ in TMEM, two Sᵀ buffers
+    for units in BWD_UNITS:
+        for seed in range(4):
+            simulate_bwd(units, n_ctas, 4, 2, seed, kt_tmem=True, dk_ss=True)
+
+
+def test_backward_dk_from_shared_memory_model_catches_a_late_dk():
+    caught = 0
+    for seed in range(40):
+        try:
+            simulate_bwd([2, 1, 3, 1, 2, 1], 2, 4, 2, seed, "dk_after_next_dp", kt_tmem=True, dk_ss=True)
+        except AssertionError:
+            caught += 1
+    assert caught > 0
 
 
 @pytest.mark.parametrize("mistake", ["no_ktfull_wait", "kt_before_kvfull", "s_before_dv"])
