@@ -23,9 +23,9 @@
 //                                  the K tile read MN-major at d = 256)
 // Roles: warp 0 TMA producer, warp 1 MMA issuer + TMEM owner, warps 4-7 compute
 // (thread = key row: Pᵀ, dSᵀ), warps 8-11 drain (thread = d row of dQᵀ; at
-// d <= 128 they also write each unit's Kᵀ into TMEM); at d = 64 and for
-// causal d = 128 warps 12-15 form a second compute warpgroup, the two groups
-// taking 32 query columns of each step each.
+// d <= 128 they also write each unit's Kᵀ into TMEM); at d <= 128 warps 12-15
+// form a second compute warpgroup, the two groups taking 32 query columns of
+// each step each.
 // For d = 256, dK/dV/dQ do not fit TMEM for a full row, so two CTAs share a
 // key tile, each owning 128 of the 256 output columns and both recomputing Sᵀ
 // and dPᵀ over the full head dimension.
@@ -148,11 +148,12 @@ struct BwdCfg {
   static constexpr int MAX_LAUNCH_REGS = COMPUTE_REGS < DRAIN_REGS ? COMPUTE_REGS : DRAIN_REGS;
 };
 
-// The configuration a kernel instance uses: two compute warpgroups at d = 64
-// and for causal d = 128 (measured, same box, backward main kernel: C3 −5.5 %,
-// C4 −8.6 %, C2 causal −3.3 % time; non-causal C2 +4.3 %, so it keeps one).
+// The configuration a kernel instance uses: two compute warpgroups at d <= 128
+// (measured, same box, backward main kernel: C3 −5.5 %, C4 −8.6 %, C2 causal
+// −3.3 % time; non-causal C2 +4.3 % with Kᵀ read from shared memory, −1.4 % and
+// −2.5 % with Kᵀ in TMEM), one at d = 256.
 template <int D, bool CAUSAL>
-using BwdCfgOf = BwdCfg<D, (D == 64 || (D == 128 && CAUSAL)) ? 2 : 1>;
+using BwdCfgOf = BwdCfg<D, (D <= 128) ? 2 : 1>;
 
 // ------------------------------------------------------------ preprocess
 // The per-row workspace arrays (D, lse2 and the fp32 dQ accumulator) use a
@@ -722,7 +723,7 @@ __global__ void __launch_bounds__(BwdCfgOf<D, CAUSAL>::THREADS, 1)
     if (C::REG_SPLIT) setmaxnreg_dec<C::CTRL_REGS>();
   } else if ((warp >= 4 && warp < 8) || warp >= 12) {
     // ------------------------------------------- compute: Pᵀ and dSᵀ rows
-    // With two compute warpgroups (d = 64), warps 4-7 take query columns 0..31
+    // With two compute warpgroups (d <= 128), warps 4-7 take query columns 0..31
     // of each step and warps 12-15 columns 32..63; each group writes its bf16
     // Pᵀ and dSᵀ into TMEM columns of its own Sᵀ / dPᵀ range (the products
     // read the two 16-query halves A_HALF columns apart), so neither group
