@@ -83,6 +83,43 @@ def test_varlen_equals_one_call_per_sequence(d, causal):
         assert rel_fro(f64(dq[0]), f64(g["dq"][:, lo:hi])) <= 1e-3, (b, "dq")
 
 
+def _random_batches(n, seed):
+    """Seeded random packed batches: 1..8 sequences of 0..599 tokens, d in
+    {64, 128, 256}, kv heads 1..2 with GQA ratio 1, 2 or 4, either mask."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        d = int(rng.choice([64, 128, 256]))
+        hkv = int(rng.integers(1, 3))
+        g = int(rng.choice([1, 2, 4]))
+        lens = tuple(int(x) for x in rng.integers(0, 600, size=int(rng.integers(1, 9))))
+        if sum(lens) < 2:
+            lens = lens + (5,)
+        causal = bool(rng.integers(0, 2))
+        out.append(VarlenWorkload(f"rand{i}_d{d}_hq{hkv * g}_hkv{hkv}_{'c' if causal else 'nc'}", lens, hkv * g, hkv,
+                                  d, causal, 9000 + i, 3.0 if d == 256 else 1.0))
+    return out
+
+
+def test_varlen_random_batches_match_oracle():
+    # 40 seeded random batches in one test (about 12 s); every failing batch is reported
+    failures = []
+    for w in _random_batches(40, 4242):
+        g = _run(w)
+        cu = w.cu_seqlens()
+        dq, dk, dv, o, lse = oracle.attention_backward_varlen(f64(g["q"]), f64(g["k"]), f64(g["v"]), f64(g["do"]), cu,
+                                                              w.scale, w.causal)
+        err_o = np.abs(f64(g["o"]) - o)
+        err = {"o_max": float(err_o.max()), "o_mean": float(err_o.mean()),
+               "lse_max": float(np.abs(f64(g["lse"]) - lse).max()),
+               "dq": rel_fro(f64(g["dq"]), dq), "dk": rel_fro(f64(g["dk"]), dk), "dv": rel_fro(f64(g["dv"]), dv)}
+        try:
+            assert_within_tolerance(err)
+        except AssertionError:
+            failures.append((w.name, w.lengths, err))
+    assert not failures, failures
+
+
 def _sampled_errors(w, g, seed, rows_per_seq=12):
     """Sampled rows of every sequence (its first and last rows, the rows
     around the first tile edge, the last tile's first row and random ones),
