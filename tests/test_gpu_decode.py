@@ -67,6 +67,34 @@ def test_decode_matches_oracle(case):
     _check(DecodeWorkload("dec", B, Hq, Hkv, Nq, Nk, d, causal, 300 + Nk + Nq))
 
 
+def _random_decode_cases(n, seed):
+    """Seeded random decode shapes: d in {64, 128, 256}, kv heads 1..3 with GQA
+    ratio 1, 2, 4 or 8, B in 1..2, Nk in 1..5999, Nq in 1..min(Nk, 256), either
+    mask: both decode kernels and partial, single and multiple row tiles."""
+    rng = np.random.default_rng(seed)
+    out = []
+    for i in range(n):
+        d = int(rng.choice([64, 128, 256]))
+        hkv = int(rng.integers(1, 4))
+        g = int(rng.choice([1, 2, 4, 8]))
+        B = int(rng.integers(1, 3))
+        Nk = int(rng.integers(1, 6000))
+        Nq = int(rng.integers(1, min(Nk, 256) + 1))
+        out.append(DecodeWorkload(f"rdec{i}", B, hkv * g, hkv, Nq, Nk, d, bool(rng.integers(0, 2)), 7000 + i))
+    return out
+
+
+def test_decode_random_shapes_match_oracle():
+    # 60 seeded random shapes in one test (a few seconds); every failing shape is reported
+    failures = []
+    for w in _random_decode_cases(60, 2718):
+        try:
+            _check(w)
+        except AssertionError as e:
+            failures.append((w.B, w.Hq, w.Hkv, w.Nq, w.Nk, w.d, w.causal, str(e)))
+    assert not failures, failures
+
+
 @pytest.mark.parametrize("name", list(DECODE_WORKLOADS))
 def test_decode_bench_workload_matches_oracle(name):
     _check(DECODE_WORKLOADS[name])
